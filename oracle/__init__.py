@@ -1,0 +1,109 @@
+"""fp64 CPU oracle for SegmentAttention -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline / reference
+legs of ``bench.py`` may import this package.  The product path never does.
+
+The arithmetic lives in ``seg_attn_oracle.c`` (plain two-pass softmax
+attention in double precision that walks the segment lists itself); this file
+compiles it with gcc on first use and marshals arguments through ctypes.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "seg_attn_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle into ``oracle/liboracle.so`` (gcc, OpenMP, IEEE double)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            P = ctypes.c_void_p
+            lib.oracle_rows.argtypes = [ctypes.c_int, P, P, P, P, P, P, P, ctypes.c_int,
+                                        ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int,
+                                        ctypes.c_int64, P, P, P, P]
+            lib.oracle_rows.restype = ctypes.c_int
+            lib.oracle_attention.argtypes = [ctypes.c_int, P, P, P, P, P, P, P, ctypes.c_int,
+                                             ctypes.c_int, ctypes.c_int, ctypes.c_double,
+                                             ctypes.c_int, P, P]
+            lib.oracle_attention.restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+def _i32(x):
+    return np.ascontiguousarray(np.asarray(x, dtype=np.int32).reshape(-1))
+
+
+def _bits(t: torch.Tensor) -> np.ndarray:
+    assert t.dtype == torch.bfloat16
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p) if a.size else ctypes.c_void_p(0)
+
+
+def attention(q_lens, seg_starts, seg_lens, q, k_pool, v_pool, scale, causal, rows=None):
+    """Oracle outputs for one batch.
+
+    ``seg_starts`` / ``seg_lens`` are per-request lists (logical order).
+    ``q`` is bf16 [sum q_lens, Hq, d]; pools are bf16 [S, Hkv, d] (CPU tensors).
+    ``rows``: optional (token_index int64 array, head int32 array); when given,
+    only those rows are computed and out is [n, d], lse [n].
+    Otherwise out is [sum q_lens, Hq, d] and lse [sum q_lens, Hq].  float64.
+    """
+    lib = _load()
+    counts = _i32([len(s) for s in seg_starts])
+    starts = _i32([x for s in seg_starts for x in s])
+    lens = _i32([x for s in seg_lens for x in s])
+    ql = _i32(q_lens)
+    qb, kb, vb = _bits(q), _bits(k_pool), _bits(v_pool)
+    hq, d = q.shape[1], q.shape[2]
+    hkv = k_pool.shape[1]
+    batch = len(q_lens)
+    if rows is None:
+        total = int(ql.sum())
+        out = np.zeros((total, hq, d), dtype=np.float64)
+        lse = np.zeros((total, hq), dtype=np.float64)
+        rc = lib.oracle_attention(batch, _ptr(ql), _ptr(counts), _ptr(starts), _ptr(lens),
+                                  _ptr(qb), _ptr(kb), _ptr(vb), hq, hkv, d, float(scale),
+                                  int(bool(causal)), _ptr(out), _ptr(lse))
+    else:
+        tok = np.ascontiguousarray(np.asarray(rows[0], dtype=np.int64))
+        head = np.ascontiguousarray(np.asarray(rows[1], dtype=np.int32))
+        out = np.zeros((tok.size, d), dtype=np.float64)
+        lse = np.zeros((tok.size,), dtype=np.float64)
+        rc = lib.oracle_rows(batch, _ptr(ql), _ptr(counts), _ptr(starts), _ptr(lens), _ptr(qb),
+                             _ptr(kb), _ptr(vb), hq, hkv, d, float(scale), int(bool(causal)),
+                             tok.size, _ptr(tok), _ptr(head), _ptr(out), _ptr(lse))
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments")
+    return torch.from_numpy(out), torch.from_numpy(lse)
+
+
+def batch_attention(wl, batch, rows=None):
+    """Convenience wrapper over a synthetic workload's batch."""
+    return attention(batch.q_lens, batch.seg_starts, batch.seg_lens, batch.q, wl.k_pool,
+                     wl.v_pool, wl.scale, batch.causal, rows=rows)

@@ -1,0 +1,207 @@
+"""Seeded synthetic workloads for SegmentAttention.
+
+This module only draws inputs: request lengths, segment lists, slot placement
+and the Q / K / V values.  It holds no attention arithmetic, so both the CUDA
+path and the fp64 oracle can take their inputs from it.
+
+The workloads follow the kernel benchmark of the Flood README ("Kernels >
+Seg-attn": 64 query heads, 8 kv heads, head_dim 128) and its segmentable
+KV cache ("Introduction": each request's cache is a few contiguous runs of
+token slots in a shared pool instead of fixed pages).
+
+Draw order, fixed for every config: lengths -> segment counts -> cut points
+-> placement -> Q -> K -> V.  Lengths, counts, cut points and placement always
+come from a CPU ``torch.Generator`` seeded with the config seed, so the table
+structure does not depend on the device.  Values come from a generator on the
+requested device seeded with the same seed; large pools are drawn on the GPU
+because drawing billions of normals on the host takes minutes.  Free pool
+slots are filled with NaN so that a read outside the segment lists poisons
+the output.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+from typing import List, Optional
+
+import torch
+
+__all__ = ["Batch", "Workload", "make_workload", "CONFIG_NAMES", "split_uniform_cuts",
+           "place_segments"]
+
+CONFIG_NAMES = {
+    1: "tiny causal prefill (2 req, q=k=16/33, 4/1 heads, d64)",
+    2: "pages-shaped prefill (1 req, q=k=1024, 64/8 heads, d128)",
+    3: "chunked prefill varlen (16 req, 2048 new tokens, prior 0-8192)",
+    4: "batched decode (128 req, k 1024-32768)",
+    5: "long-context mix (8 decode at k=131072 + 1 prefill chunk 2048 over 131072)",
+}
+
+
+@dataclass
+class Batch:
+    """One call's worth of requests over the shared pool."""
+    mode: str                      # "prefill" or "decode"
+    q_lens: List[int]
+    seg_starts: List[List[int]]    # per request, logical (list) order
+    seg_lens: List[List[int]]
+    causal: bool
+    q: Optional[torch.Tensor] = None   # bf16 [sum(q_lens), Hq, d]
+
+    @property
+    def batch(self) -> int:
+        return len(self.q_lens)
+
+    @property
+    def k_lens(self) -> List[int]:
+        return [sum(s) for s in self.seg_lens]
+
+    @property
+    def total_q(self) -> int:
+        return sum(self.q_lens)
+
+    def flat_segments(self):
+        counts = [len(s) for s in self.seg_starts]
+        starts = [x for s in self.seg_starts for x in s]
+        lens = [x for s in self.seg_lens for x in s]
+        return counts, starts, lens
+
+
+@dataclass
+class Workload:
+    config: int
+    name: str
+    q_heads: int
+    kv_heads: int
+    head_dim: int
+    num_slots: int
+    scale: float
+    batches: List[Batch]
+    k_pool: Optional[torch.Tensor] = None   # bf16 [S, Hkv, d]
+    v_pool: Optional[torch.Tensor] = None
+    live: Optional[torch.Tensor] = field(default=None, repr=False)  # bool [S]
+
+
+def split_uniform_cuts(total: int, nseg: int, gen: torch.Generator) -> List[int]:
+    """Split ``total`` tokens into ``nseg`` positive lengths at distinct uniform cut points."""
+    if total <= 0:
+        return []
+    nseg = max(1, min(nseg, total))
+    if nseg == 1:
+        return [total]
+    cuts = (torch.randperm(total - 1, generator=gen)[: nseg - 1] + 1).sort().values.tolist()
+    edges = [0] + cuts + [total]
+    return [edges[i + 1] - edges[i] for i in range(nseg)]
+
+
+def place_segments(all_lens: List[int], num_slots: int, gen: torch.Generator) -> List[int]:
+    """Random non-overlapping placement: shuffle every segment of every request,
+    cut the free slots into nseg+1 gaps at sorted uniform points, then lay gaps
+    and segments out alternately.  Returns the start slot of each segment."""
+    nseg = len(all_lens)
+    live = sum(all_lens)
+    free = num_slots - live
+    assert free >= 0, "pool too small"
+    order = torch.randperm(nseg, generator=gen).tolist()
+    cuts = torch.randint(0, free + 1, (nseg,), generator=gen).sort().values.tolist()
+    gaps = [cuts[0]] + [cuts[i] - cuts[i - 1] for i in range(1, nseg)]
+    starts = [0] * nseg
+    pos = 0
+    for i, s in enumerate(order):
+        pos += gaps[i]
+        starts[s] = pos
+        pos += all_lens[s]
+    assert pos <= num_slots
+    return starts
+
+
+def _values(shape, gen, device, std=1.0):
+    x = torch.randn(shape, generator=gen, device=device, dtype=torch.float32)
+    if std != 1.0:
+        x.mul_(std)
+    return x.to(torch.bfloat16)
+
+
+def _pool_values(num_slots, kv_heads, head_dim, live, gen, device, std):
+    """Pool values drawn in slices (bounded temporary memory), free slots NaN."""
+    pool = torch.empty((num_slots, kv_heads, head_dim), dtype=torch.bfloat16, device=device)
+    step = max(1, (1 << 26) // (kv_heads * head_dim))
+    for a in range(0, num_slots, step):
+        b = min(num_slots, a + step)
+        pool[a:b] = _values((b - a, kv_heads, head_dim), gen, device, std)
+    pool[~live.to(device)] = float("nan")
+    return pool
+
+
+def _structure(cfg: int, gen: torch.Generator):
+    """Lengths, segment counts and cut points of each config (no values)."""
+    if cfg == 1:
+        q_lens = [16, 33]
+        seg_lens = [[8, 8], [17, 16]]
+        return dict(q_heads=4, kv_heads=1, head_dim=64, num_slots=128,
+                    batches=[("prefill", q_lens, seg_lens, True)], qk_std=1.0)
+    if cfg == 2:
+        return dict(q_heads=64, kv_heads=8, head_dim=128, num_slots=65536,
+                    batches=[("prefill", [1024], [[256, 256, 256, 256]], True)], qk_std=1.0)
+    if cfg == 3:
+        B = 16
+        prior = torch.randint(0, 8193, (B,), generator=gen).tolist()
+        q_lens = torch.bincount(torch.randint(0, B, (2048,), generator=gen), minlength=B).tolist()
+        k_lens = [p + q for p, q in zip(prior, q_lens)]
+        nsegs = torch.randint(1, 7, (B,), generator=gen).tolist()
+        seg_lens = [split_uniform_cuts(k, n, gen) for k, n in zip(k_lens, nsegs)]
+        return dict(q_heads=64, kv_heads=8, head_dim=128, num_slots=262144,
+                    batches=[("prefill", q_lens, seg_lens, True)], qk_std=1.0)
+    if cfg == 4:
+        B = 128
+        k_lens = torch.randint(1024, 32769, (B,), generator=gen).tolist()
+        nsegs = torch.randint(1, 9, (B,), generator=gen).tolist()
+        seg_lens = [split_uniform_cuts(k, n, gen) for k, n in zip(k_lens, nsegs)]
+        slots = math.ceil(1.1 * sum(k_lens))
+        return dict(q_heads=64, kv_heads=8, head_dim=128, num_slots=slots,
+                    batches=[("decode", [1] * B, seg_lens, True)], qk_std=1.0)
+    if cfg == 5:
+        k_dec = [131072] * 8
+        k_pre = [131072 + 2048]
+        nsegs = torch.randint(4, 17, (9,), generator=gen).tolist()
+        lens_all = [split_uniform_cuts(k, n, gen) for k, n in zip(k_dec + k_pre, nsegs)]
+        slots = math.ceil(1.1 * (sum(k_dec) + sum(k_pre)))
+        return dict(q_heads=64, kv_heads=8, head_dim=128, num_slots=slots,
+                    batches=[("decode", [1] * 8, lens_all[:8], True),
+                             ("prefill", [2048], lens_all[8:], True)], qk_std=0.5)
+    raise ValueError(f"unknown config {cfg}")
+
+
+def make_workload(cfg: int, device: str = "cpu", values: bool = True,
+                  seed: Optional[int] = None) -> Workload:
+    """Build config ``cfg`` (1..5).  Seed defaults to cfg - 1."""
+    seed = cfg - 1 if seed is None else seed
+    gen = torch.Generator(device="cpu").manual_seed(seed)
+    st = _structure(cfg, gen)
+    batches = []
+    all_lens = []
+    for mode, q_lens, seg_lens, causal in st["batches"]:
+        batches.append(Batch(mode=mode, q_lens=list(q_lens), seg_starts=[], seg_lens=seg_lens,
+                             causal=causal))
+        for s in seg_lens:
+            all_lens.extend(s)
+    starts = place_segments(all_lens, st["num_slots"], gen)
+    it = iter(starts)
+    for b in batches:
+        b.seg_starts = [[next(it) for _ in s] for s in b.seg_lens]
+    live = torch.zeros(st["num_slots"], dtype=torch.bool)
+    for b in batches:
+        for ss, ll in zip(b.seg_starts, b.seg_lens):
+            for s, l in zip(ss, ll):
+                live[s:s + l] = True
+    wl = Workload(config=cfg, name=CONFIG_NAMES[cfg], q_heads=st["q_heads"],
+                  kv_heads=st["kv_heads"], head_dim=st["head_dim"], num_slots=st["num_slots"],
+                  scale=1.0 / math.sqrt(st["head_dim"]), batches=batches, live=live)
+    if values:
+        vgen = torch.Generator(device=device).manual_seed(seed)
+        for b in batches:
+            b.q = _values((b.total_q, wl.q_heads, wl.head_dim), vgen, device, st["qk_std"])
+        wl.k_pool = _pool_values(wl.num_slots, wl.kv_heads, wl.head_dim, live, vgen, device,
+                                 st["qk_std"])
+        wl.v_pool = _pool_values(wl.num_slots, wl.kv_heads, wl.head_dim, live, vgen, device, 1.0)
+    return wl

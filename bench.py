@@ -1,0 +1,496 @@
+"""Benchmark of the SegmentAttention hot path on B200.
+
+One step = one pass of the whole path over one batch of the long-context mix
+(8 decode requests at k = 131072, then one prefill chunk of 2048 queries over
+131072 prior tokens; 64 query / 8 kv heads, d = 128, shared segmented pool):
+table build is done once (host), then per step: decode split-K + merge and
+the tcgen05 prefill, all through the C ABI on one stream.
+
+Metric: prefill TFLOPS and decode HBM GB/s vs peak, as in the Flood README
+kernel table ("Kernels > Seg-attn", which reports both prefill and decode in
+TFLOPS).  `value` is the step's attention TFLOP/s: (prefill flops, causal
+4*d*Hq*sum(q*p + q^2/2), plus decode flops 4*d*Hq*sum(k)) / step time.  The
+per-leg numbers (prefill TFLOP/s, decode GB/s) and their fractions of the
+measured peaks are in `legs`.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config C]
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import segmented_kv_cache_b200 as sa  # noqa: E402
+from segmented_kv_cache_b200 import synth  # noqa: E402
+
+METRIC = "prefill TFLOPS and decode HBM GB/s (1 B200) vs peak; max-abs err vs oracle"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 1024 * 1024
+
+
+# ----------------------------------------------------------------------------- helpers
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def prefill_flops(batch, wl):
+    tot = 0.0
+    for q, k in zip(batch.q_lens, batch.k_lens):
+        p = k - q
+        tot += q * p + (q * q / 2.0 if batch.causal else q * q)
+    return 4.0 * wl.head_dim * wl.q_heads * tot
+
+
+def decode_flops(batch, wl):
+    return 4.0 * wl.head_dim * wl.q_heads * float(sum(batch.k_lens))
+
+
+def decode_bytes(batch, wl, table_bytes):
+    kv = 2 * 2 * wl.kv_heads * wl.head_dim * float(sum(batch.k_lens))
+    qo = 2 * 2 * batch.batch * wl.q_heads * wl.head_dim
+    return kv + qo + 4 * batch.batch * wl.q_heads + table_bytes
+
+
+def source_digest(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def profiled_traffic(kernel, workload_tag):
+    """DRAM bytes per launch from the committed ncu summary, if it still matches the source."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload_tag}.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m = re.search(r"dram bytes per launch \(read\+write\):\s*([0-9.eE+]+)", text)
+    h = re.search(r"source sha256\[:16\] of ([\w/.]+):\s*([0-9a-f]{16})", text)
+    if not m or not h:
+        return None
+    src = os.path.join(ROOT, h.group(1))
+    if not os.path.exists(src) or source_digest(src) != h.group(2):
+        return None  # kernel changed since the counters were taken
+    return float(m.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled while the timed region runs."""
+    FIELDS = ("index,timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def stop(self, t0, t1):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = [l for (t, l) in self.lines if t0 - 0.06 <= t <= t1 + 0.06] or \
+            [l for (_, l) in self.lines[-3:]]
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            f = [x.strip() for x in r.split(",")]
+            if len(f) < 10:
+                continue
+            try:
+                sm.append(float(f[2]))
+                mx.append(float(f[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[6:10]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+# ----------------------------------------------------------------------------- workload
+class Path:
+    """Device-resident buffers + tables of one workload, and the calls of one step."""
+
+    def __init__(self, wl, device):
+        self.wl = wl
+        self.device = device
+        self.legs = []
+        for b in wl.batches:
+            mode = sa.MODE_PREFILL if b.mode == "prefill" else sa.MODE_DECODE
+            tab = sa.SegTable.build(b.q_lens if mode == sa.MODE_PREFILL else None, b.seg_starts,
+                                    b.seg_lens, wl.num_slots, b.causal, mode, wl.q_heads,
+                                    wl.kv_heads, wl.head_dim, pin=True)
+            tab.to(device)
+            out = torch.empty_like(b.q)
+            lse = torch.empty(b.q.shape[0], wl.q_heads, dtype=torch.float32, device=device)
+            ws = (torch.empty(tab.workspace_bytes, dtype=torch.uint8, device=device)
+                  if tab.workspace_bytes else None)
+            launches = 1 + (1 if (mode == sa.MODE_DECODE and tab.workspace_bytes) else 0)
+            self.legs.append(dict(batch=b, mode=mode, tab=tab, out=out, lse=lse, ws=ws,
+                                  launches=launches))
+
+    def run_leg(self, leg, stream=None):
+        fn = sa.seg_attn_prefill if leg["mode"] == sa.MODE_PREFILL else sa.seg_attn_decode
+        fn(leg["batch"].q, self.wl.k_pool, self.wl.v_pool, leg["out"], leg["lse"],
+           leg["tab"].device, leg["tab"].desc, self.wl.scale, leg["ws"], stream)
+
+    def launches_per_step(self):
+        return sum(l["launches"] for l in self.legs)
+
+
+def workload_name(wl):
+    return {1: "tiny causal prefill", 2: "pages-shaped prefill q=k=1024",
+            3: "chunked prefill varlen (16 req, 2048 new tokens)",
+            4: "batched decode 128 req k=1024..32768",
+            5: "long-context mix: decode 8x131072 + prefill 2048 over 131072"}[wl.config]
+
+
+# ----------------------------------------------------------------------------- oracle legs
+def oracle_sample(wl, leg_batches, budget_rows, rng_seed=0):
+    """Bounded oracle sample: `budget_rows` (token, head) rows per batch of the workload.
+
+    Returns (flops, seconds, rows_desc, results) where results hold the oracle rows for a
+    parity spot check of the GPU outputs."""
+    import oracle
+    g = torch.Generator().manual_seed(rng_seed)
+    flops, secs, results, desc = 0.0, 0.0, [], []
+    for bi, b in enumerate(leg_batches):
+        n = min(budget_rows[bi], b.total_q * wl.q_heads)
+        toks = torch.randint(0, b.total_q, (n,), generator=g)
+        heads = torch.randint(0, wl.q_heads, (n,), generator=g)
+        q_off = np.concatenate([[0], np.cumsum(b.q_lens)])
+        reqs = sorted(set(int(np.searchsorted(q_off, int(t), side="right") - 1) for t in toks))
+        # compact pool: only the sampled requests' segments (relocation is result-neutral)
+        seg_s, seg_l, idx, pos = [], [], [], 0
+        for r in reqs:
+            ss, ll = [], []
+            for s, l in zip(b.seg_starts[r], b.seg_lens[r]):
+                ss.append(pos)
+                ll.append(l)
+                idx.append(torch.arange(s, s + l))
+                pos += l
+            seg_s.append(ss)
+            seg_l.append(ll)
+        ii = torch.cat(idx).to(wl.k_pool.device)
+        kp, vp = wl.k_pool[ii].cpu(), wl.v_pool[ii].cpu()
+        q_rows = torch.cat([torch.arange(q_off[r], q_off[r + 1]) for r in reqs])
+        qc = b.q[q_rows.to(b.q.device)].cpu()
+        new_off = np.concatenate([[0], np.cumsum([b.q_lens[r] for r in reqs])])
+        remap = {}
+        for j, r in enumerate(reqs):
+            for t in range(b.q_lens[r]):
+                remap[q_off[r] + t] = new_off[j] + t
+        ltok = np.array([remap[int(t)] for t in toks], dtype=np.int64)
+        for t in toks.tolist():
+            r = int(np.searchsorted(q_off, t, side="right") - 1)
+            i = t - q_off[r]
+            vis = (b.k_lens[r] - b.q_lens[r] + i + 1) if (b.causal and b.mode == "prefill") else \
+                b.k_lens[r]
+            flops += 4.0 * wl.head_dim * min(vis, b.k_lens[r])
+        t0 = time.perf_counter()
+        o, l = oracle.attention([b.q_lens[r] for r in reqs], seg_s, seg_l, qc, kp, vp, wl.scale,
+                                b.causal and b.mode == "prefill", rows=(ltok, heads.numpy()))
+        secs += time.perf_counter() - t0
+        results.append((bi, toks, heads, o, l))
+        desc.append(f"{n} random (token, head) rows of the {b.mode} batch")
+    return flops, secs, "; ".join(desc), results
+
+
+# ----------------------------------------------------------------------------- main arms
+def run_reference(args):
+    """The oracle as it stands, timed on the host cores, on bounded samples of the workload."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    wl = synth.make_workload(args.config, device="cuda" if torch.cuda.is_available() else "cpu")
+    rows = [args.ref_rows] * len(wl.batches)
+    for _ in range(args.warmup if args.warmup <= 1 else 1):
+        oracle_sample(wl, wl.batches, [max(1, r // 8) for r in rows], rng_seed=99)
+    fl, sec = 0.0, 0.0
+    sample_desc = ""
+    for s in range(args.steps):
+        f, t, sample_desc, _ = oracle_sample(wl, wl.batches, rows, rng_seed=s)
+        fl += f
+        sec += t
+    value = fl / sec / 1e12
+    cores = cpu_cores()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * sec / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": workload_name(wl), "seed": wl.config - 1},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                             "sample": f"per step: {sample_desc}"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (no CPU fallback)")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+    # weak scaling: every rank runs its own batch of the same shape (seed offset by rank)
+    wl = synth.make_workload(args.config, device=str(device), seed=args.config - 1 + 1000 * rank)
+    path = Path(wl, device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        for leg in path.legs:
+            path.run_leg(leg)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert sa.seg_attn_take_device_error() == 0
+
+    # per-leg events inside the timed region, on the launching (current) stream
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(path.legs) + 1)]
+          for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local).start() if rank == 0 else None
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = time.time()
+    start.record(stream)
+    for s in range(args.steps):
+        ev[s][0].record(stream)
+        for i, leg in enumerate(path.legs):
+            path.run_leg(leg)
+            ev[s][i + 1].record(stream)
+    end.record(stream)
+    torch.cuda.synchronize()
+    t1 = time.time()
+    if dist:
+        dist.barrier()
+    clocks = sampler.stop(t0, t1) if sampler else None
+    ms = start.elapsed_time(end)
+    leg_ms = [sum(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(args.steps)) / args.steps
+              for i in range(len(path.legs))]
+    if dist:
+        t = torch.tensor([ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    assert sa.seg_attn_take_device_error() == 0
+
+    peaks, peak_kind = load_peaks()
+    flops_step = 0.0
+    legs = {}
+    dominant = None
+    for leg, lm in zip(path.legs, leg_ms):
+        b = leg["batch"]
+        if leg["mode"] == sa.MODE_PREFILL:
+            f = prefill_flops(b, wl)
+            tf = f / (lm * 1e-3) / 1e12
+            legs["prefill"] = {"ms": lm, "tflops": tf, "flops": f,
+                               "frac_sustained": tf / peaks["bf16_tflops_sustained"],
+                               "frac_burst": tf / peaks["bf16_tflops"]}
+            flops_step += f
+            cand = ("tensor", lm, f)
+        else:
+            f = decode_flops(b, wl)
+            by = decode_bytes(b, wl, leg["tab"].desc.table_bytes)
+            gbs = by / (lm * 1e-3) / 1e9
+            legs["decode"] = {"ms": lm, "gbs": gbs, "bytes": by, "tflops": f / (lm * 1e-3) / 1e12,
+                              "frac_hbm": gbs / peaks["hbm_gbs"],
+                              "launches": leg["launches"]}
+            flops_step += f
+            cand = ("hbm", lm, by)
+        if dominant is None or cand[1] > dominant[1]:
+            dominant = cand
+    value = world * flops_step / (ms * 1e-3 / args.steps) / 1e12
+
+    if dominant[0] == "tensor":
+        achieved = dominant[2] / (dominant[1] * 1e-3) / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        traffic = profiled_traffic("prefill_sm100", f"cfg{wl.config}")
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": traffic, "kernel": "prefill_kernel<128>",
+                "peak_kind": f"{peak_kind} sustained bf16 (cuBLAS 8192^3 loop)"}
+    else:
+        achieved = dominant[2] / (dominant[1] * 1e-3) / 1e9
+        peak = peaks["hbm_gbs"]
+        traffic = profiled_traffic("decode_sm100", f"cfg{wl.config}")
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "traffic": traffic,
+                "kernel": "decode_chunk_kernel<128> + decode_merge_kernel<128>",
+                "peak_kind": f"{peak_kind} copy bandwidth"}
+
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": workload_name(wl), "seed": wl.config - 1,
+                       "q_heads": wl.q_heads, "kv_heads": wl.kv_heads, "head_dim": wl.head_dim,
+                       "num_slots": wl.num_slots,
+                       "l2": ("inputs larger than L2 (pools %.1f GB), no flush" %
+                              (2 * wl.k_pool.numel() * 2 / 1e9))
+                       if 2 * wl.k_pool.numel() * 2 > L2_BYTES else "inputs fit in L2",
+                       "parallelism": f"dp{world} (independent batches per GPU)"},
+            "legs": legs, "roofline": roof,
+            "gpu_launches": path.launches_per_step() * args.steps,
+            "clocks": clocks}
+
+    if rank == 0 and not args.no_e2e:
+        line["e2e"] = run_e2e(path, args, world)
+    if rank == 0 and not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"], line["parity_sample"] = run_cpu_baseline(path, args)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def run_e2e(path, args, world):
+    """Same step through the public C-ABI calls with host buffers: every step copies its inputs
+    (queries, both pools, tables) from pinned host memory and reads the outputs back."""
+    wl = path.wl
+    dev = path.device
+    h_k = torch.empty(wl.k_pool.shape, dtype=wl.k_pool.dtype, pin_memory=True)
+    h_v = torch.empty(wl.v_pool.shape, dtype=wl.v_pool.dtype, pin_memory=True)
+    h_k.copy_(wl.k_pool)
+    h_v.copy_(wl.v_pool)
+    h_q = [torch.empty(l["batch"].q.shape, dtype=torch.bfloat16, pin_memory=True).copy_(l["batch"].q)
+           for l in path.legs]
+    h_out = [torch.empty(l["out"].shape, dtype=torch.bfloat16, pin_memory=True) for l in path.legs]
+    h_lse = [torch.empty(l["lse"].shape, dtype=torch.float32, pin_memory=True) for l in path.legs]
+    stream = torch.cuda.current_stream(dev)
+    h2d = h_k.numel() * 2 + h_v.numel() * 2 + sum(q.numel() * 2 for q in h_q) + \
+        sum(l["tab"].desc.table_bytes for l in path.legs)
+    d2h = sum(o.numel() * 2 for o in h_out) + sum(l.numel() * 4 for l in h_lse)
+
+    def step():
+        wl.k_pool.copy_(h_k, non_blocking=True)
+        wl.v_pool.copy_(h_v, non_blocking=True)
+        for leg, hq in zip(path.legs, h_q):
+            leg["batch"].q.copy_(hq, non_blocking=True)
+            leg["tab"].device.copy_(leg["tab"].host, non_blocking=True)
+        for leg in path.legs:
+            path.run_leg(leg)
+        for leg, ho, hl in zip(path.legs, h_out, h_lse):
+            ho.copy_(leg["out"], non_blocking=True)
+            hl.copy_(leg["lse"], non_blocking=True)
+
+    n = max(1, min(args.steps, args.e2e_steps))
+    step()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(n):
+        step()
+    e.record(stream)
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / n
+    flops = sum(prefill_flops(l["batch"], wl) if l["mode"] == sa.MODE_PREFILL else
+                decode_flops(l["batch"], wl) for l in path.legs)
+    return {"value": world * flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": ms,
+            "steps": n}
+
+
+def run_cpu_baseline(path, args):
+    """The oracle on a bounded sample of the same workload (rank 0, N = 1), plus a parity
+    spot check of the bench's own GPU outputs on the sampled rows."""
+    wl = path.wl
+    rows = [args.cpu_rows] * len(wl.batches)
+    fl, sec, desc, results = oracle_sample(wl, wl.batches, rows, rng_seed=1234)
+    worst = {"max_abs": 0.0, "mean_abs": 0.0, "lse_rel": 0.0}
+    for bi, toks, heads, o, l in results:
+        leg = path.legs[bi]
+        go = leg["out"][toks.to(path.device), heads.to(path.device)].double().cpu()
+        gl = leg["lse"][toks.to(path.device), heads.to(path.device)].double().cpu()
+        err = (go - o).abs()
+        worst["max_abs"] = max(worst["max_abs"], float(err.max()))
+        worst["mean_abs"] = max(worst["mean_abs"], float(err.mean()))
+        worst["lse_rel"] = max(worst["lse_rel"],
+                               float(((gl - l).abs() / l.abs().clamp(min=1)).max()))
+    base = {"value": fl / sec / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+            "sample": desc, "seconds": sec}
+    return base, worst
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=40)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", type=int, default=5, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--ref-rows", type=int, default=48,
+                    help="oracle rows per batch per step (bounded CPU sample)")
+    ap.add_argument("--cpu-rows", type=int, default=256,
+                    help="oracle rows per batch for the cpu_baseline leg of our arm")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        print("note: fewer than 3 warm-up steps", file=sys.stderr)
+    return run_reference(args) if args.impl == "reference" else run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,185 @@
+/*
+ * seg_attn.h -- C ABI of the B200 (sm_100a) SegmentAttention library.
+ *
+ * SegmentAttention is exact causal / variable-length / grouped-query softmax
+ * attention over a *segmentable* KV cache (Flood README, "Introduction":
+ * the cache is managed in segmentable blocks instead of paged blocks, which
+ * keeps each request's cache contiguous; SegmentAttention is the attention
+ * kernel written for that cache).  Each request's keys and values live in a
+ * shared token-slot pool as a short list of contiguous runs (slot_start, len).
+ * The same library serves chunked prefill (Flood README feature list: a chunk
+ * of new queries attends to the prior context plus itself) and decode (one
+ * query per request over its whole context; README "Kernels > Seg-attn",
+ * batch 128, Q_len 1 rows).
+ *
+ * Math (per request r, query i, query head h):
+ *   g = h / (q_heads / kv_heads)                      (contiguous GQA groups)
+ *   logical key j of r lives in slot  seg_start[s] + (j - off_s), where
+ *   off_s is the sum of the lengths listed before segment s (list order is
+ *   logical order; slot order is irrelevant).
+ *   causal: query i sees keys j <= (k_len - q_len) + i  (bottom-right aligned)
+ *   s_j = scale * <q[i,h,:], K[slot(j), g, :]>
+ *   out[i,h,:] = sum_j softmax(s)_j V[slot(j), g, :]
+ *   lse[i,h]   = ln sum_j exp(s_j)                   (natural log, scale included)
+ *   A query that sees no key gets out = 0 and lse = -inf.
+ * Kernels use the online-softmax state (running max m_i, normaliser l_i) of
+ * FlashAttention, described in the Ascend FlashAttention article, section
+ * "bottleneck 2"; the decode split over key blocks with a per-request
+ * reduction follows the per-block partial attention + per-request reduce of
+ * the FlashAccel article, section "data layout optimisation".
+ *
+ * Conventions for every entry point:
+ *   - The caller owns every buffer.  The library never allocates or frees
+ *     memory and never synchronises the device.
+ *   - Tensors are dense, row-major, 16-byte aligned:
+ *       q, out   bf16 [total_q, q_heads, head_dim]   (requests packed in order)
+ *       k_pool, v_pool  bf16 [num_slots, kv_heads, head_dim]
+ *       lse      fp32 [total_q, q_heads]  (may be NULL)
+ *   - The new tokens' K/V rows are already written into the pool: they are
+ *     the last q_len logical keys of each request's segment list.
+ *   - Supported shapes: head_dim in {64, 128}; q_heads % kv_heads == 0;
+ *     prefill: group size q_heads/kv_heads a power of two <= 128;
+ *     decode:  group size a power of two <= 8.
+ *   - Errors are returned synchronously as a negative seg_attn_status before
+ *     anything is launched; nothing is launched on error.  A launch failure
+ *     is reported as SEG_ATTN_ERR_CUDA.  Device code never traps.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ */
+#ifndef SEG_ATTN_H_
+#define SEG_ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SEG_ATTN_OK = 0,
+  SEG_ATTN_ERR_INVALID_ARG = -1,       /* bad pointer, size, shape or flag */
+  SEG_ATTN_ERR_SEGMENT_OOB = -2,       /* a segment reaches outside [0, num_slots) */
+  SEG_ATTN_ERR_SEGMENT_OVERLAP = -3,   /* two segments of one request share a slot */
+  SEG_ATTN_ERR_QLEN_GT_KLEN = -4,      /* causal request with more queries than keys */
+  SEG_ATTN_ERR_WORKSPACE = -5,         /* workspace missing or smaller than needed */
+  SEG_ATTN_ERR_UNSUPPORTED = -6,       /* valid but outside the supported shapes */
+  SEG_ATTN_ERR_CUDA = -7,              /* a CUDA runtime / driver call failed */
+  SEG_ATTN_ERR_BUFFER_TOO_SMALL = -8   /* host_out smaller than desc->table_bytes */
+} seg_attn_status;
+
+enum { SEG_ATTN_MODE_PREFILL = 0, SEG_ATTN_MODE_DECODE = 1 };
+
+#define SEG_ATTN_TABLE_MAGIC 0x53454741u /* "SEGA" */
+#define SEG_ATTN_TABLE_VERSION 1u
+
+/*
+ * Description of a built segment table.  Filled by seg_attn_build_table; the
+ * caller passes it back unchanged to the compute calls.  Offsets count int32
+ * elements from the start of the table buffer.
+ */
+typedef struct seg_attn_table_desc {
+  uint32_t magic, version;
+  int32_t mode, causal;
+  int32_t batch, q_heads, kv_heads, head_dim;
+  int64_t num_slots;
+  int64_t total_q;         /* sum of q_lens = rows of q / out */
+  int64_t total_k;         /* sum of k_lens */
+  int32_t num_segments;
+  int32_t num_work;        /* prefill: (request, kv head, query-tile pair) items; decode: chunks */
+  int32_t queries_per_tile;/* prefill: 128 / group size */
+  int32_t chunk_len;       /* decode: logical keys per split-K chunk */
+  int32_t max_k_tiles;     /* prefill: largest number of 128-key tiles of one item */
+  int32_t reserved0;
+  int64_t off_q_offsets;   /* [batch+1] packed query offset of each request */
+  int64_t off_k_lens;      /* [batch]   keys of each request */
+  int64_t off_seg_offsets; /* [batch+1] first segment of each request */
+  int64_t off_seg_start;   /* [num_segments] first slot of each segment */
+  int64_t off_seg_kstart;  /* [num_segments] logical index of each segment's first key */
+  int64_t off_seg_len;     /* [num_segments] */
+  int64_t off_work;        /* [num_work][4] work items (16-byte aligned) */
+  int64_t off_req_chunks;  /* decode: [batch+1] first chunk of each request */
+  uint64_t table_bytes;    /* size of the table buffer */
+  uint64_t workspace_bytes;/* device scratch the compute call needs (may be 0) */
+} seg_attn_table_desc;
+
+/*
+ * seg_attn_build_table -- validate per-request segment lists and lay out the
+ * table (CSR segment arrays + the kernel work list) in host memory.
+ *
+ *   batch                 number of requests (>= 0)
+ *   q_lens [batch]        new queries per request (>= 0); NULL in decode mode
+ *                         means 1 each; decode requires every q_len == 1
+ *   seg_counts [batch]    segments per request (>= 0)
+ *   seg_starts, seg_lens  [sum seg_counts] first slot and length (>= 0) of each
+ *                         segment, requests back to back, logical order
+ *   num_slots             pool rows; every segment must lie in [0, num_slots)
+ *   causal                1 = bottom-right causal mask, 0 = none (decode
+ *                         always sees every key of the request)
+ *   mode                  SEG_ATTN_MODE_PREFILL or SEG_ATTN_MODE_DECODE
+ *   q_heads, kv_heads, head_dim   shapes as above
+ *   host_out, host_out_bytes      destination (any alignment >= 16 bytes);
+ *                         pass host_out = NULL to only fill desc (size query)
+ *   desc                  out: table description
+ *
+ * Segments of different requests may share slots (read-only prefix sharing);
+ * segments of one request may not.  Returns SEG_ATTN_OK or a negative status;
+ * on SEG_ATTN_ERR_BUFFER_TOO_SMALL desc->table_bytes holds the needed size.
+ * Host only: touches no device state.  The caller copies table_bytes of
+ * host_out to device memory (16-byte aligned) and passes that copy as
+ * dev_table below.
+ */
+int seg_attn_build_table(int batch, const int32_t* q_lens, const int32_t* seg_counts,
+                         const int32_t* seg_starts, const int32_t* seg_lens, int64_t num_slots,
+                         int causal, int mode, int q_heads, int kv_heads, int head_dim,
+                         void* host_out, size_t host_out_bytes, seg_attn_table_desc* desc);
+
+/* Device workspace (bytes) the compute call for this table needs; 0 if none. */
+size_t seg_attn_workspace_size(const seg_attn_table_desc* desc);
+
+/*
+ * seg_attn_prefill -- chunked-prefill attention (mode PREFILL table).
+ * One persistent-tile sm_100a kernel: K/V tiles of 128 logical keys are
+ * gathered row by row from the pool with TMA, S = QK^T and O += PV run on the
+ * tcgen05 tensor cores with accumulators in tensor memory, the online softmax
+ * runs in registers.  Writes out (and lse if non-NULL) for every row.
+ *   softmax_scale  > 0 and finite (typically 1/sqrt(head_dim))
+ *   workspace      unused for prefill (may be NULL / 0)
+ */
+int seg_attn_prefill(const void* q, const void* k_pool, const void* v_pool, void* out, float* lse,
+                     const void* dev_table, const seg_attn_table_desc* desc, float softmax_scale,
+                     void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * seg_attn_decode -- one query per request over its whole context (mode
+ * DECODE table).  Split-K over chunks of logical keys: one CTA per
+ * (chunk, kv head) streams K/V with 128-bit loads, packs the group's query
+ * heads so each K/V byte is read once per kv head, and keeps the softmax state
+ * in registers; a second kernel merges the per-chunk partials by their
+ * log-sum-exp.  workspace: device memory of at least
+ * seg_attn_workspace_size(desc) bytes, 16-byte aligned (contents are scratch).
+ */
+int seg_attn_decode(const void* q, const void* k_pool, const void* v_pool, void* out, float* lse,
+                    const void* dev_table, const seg_attn_table_desc* desc, float softmax_scale,
+                    void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * seg_attn_take_device_error -- read and clear the library's device error
+ * word.  Kernels never trap; every wait on an mbarrier gives up after one
+ * second, and a CTA that gave up drains its copies, frees its tensor memory,
+ * returns, and sets this word to a non-zero value (its output rows are then
+ * undefined).  Synchronous: copies from the device (implicitly synchronises
+ * the current device).  *value = 0 means no kernel gave up since the last call.
+ */
+int seg_attn_take_device_error(int* value);
+
+/* Static English description of a status code (never NULL). */
+const char* seg_attn_status_string(int status);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int seg_attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SEG_ATTN_H_ */

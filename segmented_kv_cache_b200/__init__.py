@@ -1,0 +1,205 @@
+"""SegmentAttention for B200: Python binding of the C-ABI library ``libsegattn.so``.
+
+Every function here only marshals arguments for the C entry points declared
+in ``include/seg_attn.h`` (same names).  All compute runs in the library's
+sm_100a kernels; there is no fallback path.  PyTorch supplies device memory
+and streams only.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from dataclasses import dataclass
+from typing import Optional, Sequence
+
+import numpy as np
+import torch
+
+from ._build import LIB as LIB_PATH
+
+__all__ = [
+    "SegAttnError", "seg_attn_table_desc", "seg_attn_build_table", "seg_attn_workspace_size",
+    "seg_attn_prefill", "seg_attn_decode", "seg_attn_status_string", "seg_attn_version",
+    "seg_attn_take_device_error", "SegTable", "load_library", "LIB_PATH",
+    "MODE_PREFILL", "MODE_DECODE", "STATUS",
+]
+
+MODE_PREFILL = 0
+MODE_DECODE = 1
+STATUS = {
+    "OK": 0, "INVALID_ARG": -1, "SEGMENT_OOB": -2, "SEGMENT_OVERLAP": -3, "QLEN_GT_KLEN": -4,
+    "WORKSPACE": -5, "UNSUPPORTED": -6, "CUDA": -7, "BUFFER_TOO_SMALL": -8,
+}
+
+
+class seg_attn_table_desc(ctypes.Structure):
+    """Mirror of ``seg_attn_table_desc`` in include/seg_attn.h."""
+    _fields_ = [
+        ("magic", ctypes.c_uint32), ("version", ctypes.c_uint32),
+        ("mode", ctypes.c_int32), ("causal", ctypes.c_int32),
+        ("batch", ctypes.c_int32), ("q_heads", ctypes.c_int32),
+        ("kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+        ("num_slots", ctypes.c_int64), ("total_q", ctypes.c_int64), ("total_k", ctypes.c_int64),
+        ("num_segments", ctypes.c_int32), ("num_work", ctypes.c_int32),
+        ("queries_per_tile", ctypes.c_int32), ("chunk_len", ctypes.c_int32),
+        ("max_k_tiles", ctypes.c_int32), ("reserved0", ctypes.c_int32),
+        ("off_q_offsets", ctypes.c_int64), ("off_k_lens", ctypes.c_int64),
+        ("off_seg_offsets", ctypes.c_int64), ("off_seg_start", ctypes.c_int64),
+        ("off_seg_kstart", ctypes.c_int64), ("off_seg_len", ctypes.c_int64),
+        ("off_work", ctypes.c_int64), ("off_req_chunks", ctypes.c_int64),
+        ("table_bytes", ctypes.c_uint64), ("workspace_bytes", ctypes.c_uint64),
+    ]
+
+
+class SegAttnError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        self.code = code
+        super().__init__(f"{fn}: {seg_attn_status_string(code)} (status {code})")
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def load_library(path: Optional[str] = None) -> ctypes.CDLL:
+    """Load libsegattn.so (built in-tree by ``__graft_entry__.build()``); fail loudly if absent."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        path = path or LIB_PATH
+        if not os.path.exists(path):
+            raise ImportError(f"CUDA library not built: {path} is missing "
+                              "(run python -c 'import __graft_entry__; __graft_entry__.build()')")
+        lib = ctypes.CDLL(path)
+        P, I, I64, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+        D = ctypes.POINTER(seg_attn_table_desc)
+        lib.seg_attn_build_table.argtypes = [I, P, P, P, P, I64, I, I, I, I, I, P, SZ, D]
+        lib.seg_attn_build_table.restype = I
+        lib.seg_attn_workspace_size.argtypes = [D]
+        lib.seg_attn_workspace_size.restype = SZ
+        for fn in (lib.seg_attn_prefill, lib.seg_attn_decode):
+            fn.argtypes = [P, P, P, P, P, P, D, ctypes.c_float, P, SZ, P]
+            fn.restype = I
+        lib.seg_attn_status_string.argtypes = [I]
+        lib.seg_attn_status_string.restype = ctypes.c_char_p
+        lib.seg_attn_version.argtypes = []
+        lib.seg_attn_version.restype = I
+        lib.seg_attn_take_device_error.argtypes = [ctypes.POINTER(ctypes.c_int)]
+        lib.seg_attn_take_device_error.restype = I
+        _lib = lib
+        return lib
+
+
+def seg_attn_status_string(code: int) -> str:
+    return load_library().seg_attn_status_string(int(code)).decode()
+
+
+def seg_attn_version() -> int:
+    return load_library().seg_attn_version()
+
+
+def _i32(x) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(x, dtype=np.int32).reshape(-1))
+
+
+def _np_ptr(a: Optional[np.ndarray]):
+    return ctypes.c_void_p(a.ctypes.data) if a is not None and a.size else ctypes.c_void_p(0)
+
+
+def seg_attn_build_table(batch: int, q_lens: Optional[Sequence[int]], seg_counts: Sequence[int],
+                         seg_starts: Sequence[int], seg_lens: Sequence[int], num_slots: int,
+                         causal: bool, mode: int, q_heads: int, kv_heads: int, head_dim: int,
+                         pin: bool = False):
+    """Returns (host table as an int32 torch tensor, seg_attn_table_desc).  Raises SegAttnError."""
+    lib = load_library()
+    ql = _i32(q_lens) if q_lens is not None else None
+    sc, ss, sl = _i32(seg_counts), _i32(seg_starts), _i32(seg_lens)
+    desc = seg_attn_table_desc()
+    args = [int(batch), _np_ptr(ql), _np_ptr(sc), _np_ptr(ss), _np_ptr(sl), int(num_slots),
+            int(bool(causal)), int(mode), int(q_heads), int(kv_heads), int(head_dim)]
+    rc = lib.seg_attn_build_table(*args, ctypes.c_void_p(0), 0, ctypes.byref(desc))
+    if rc != 0:
+        raise SegAttnError("seg_attn_build_table", rc)
+    n = max(1, (desc.table_bytes + 3) // 4)
+    host = torch.zeros(n, dtype=torch.int32, pin_memory=pin)
+    rc = lib.seg_attn_build_table(*args, ctypes.c_void_p(host.data_ptr()), int(desc.table_bytes),
+                                  ctypes.byref(desc))
+    if rc != 0:
+        raise SegAttnError("seg_attn_build_table", rc)
+    return host, desc
+
+
+def seg_attn_workspace_size(desc: seg_attn_table_desc) -> int:
+    return int(load_library().seg_attn_workspace_size(ctypes.byref(desc)))
+
+
+def _dptr(t: Optional[torch.Tensor]):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _stream_ptr(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _compute(fn_name, q, k_pool, v_pool, out, lse, dev_table, desc, softmax_scale, workspace,
+             stream):
+    lib = load_library()
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    rc = getattr(lib, fn_name)(_dptr(q), _dptr(k_pool), _dptr(v_pool), _dptr(out), _dptr(lse),
+                               _dptr(dev_table), ctypes.byref(desc), float(softmax_scale),
+                               _dptr(workspace), int(ws_bytes), _stream_ptr(stream))
+    if rc != 0:
+        raise SegAttnError(fn_name, rc)
+
+
+def seg_attn_prefill(q, k_pool, v_pool, out, lse, dev_table, desc, softmax_scale,
+                     workspace=None, stream=None) -> None:
+    """Launch chunked-prefill attention on ``stream`` (default: torch's current stream)."""
+    _compute("seg_attn_prefill", q, k_pool, v_pool, out, lse, dev_table, desc, softmax_scale,
+             workspace, stream)
+
+
+def seg_attn_decode(q, k_pool, v_pool, out, lse, dev_table, desc, softmax_scale,
+                    workspace=None, stream=None) -> None:
+    """Launch split-K decode attention on ``stream`` (default: torch's current stream)."""
+    _compute("seg_attn_decode", q, k_pool, v_pool, out, lse, dev_table, desc, softmax_scale,
+             workspace, stream)
+
+
+def seg_attn_take_device_error() -> int:
+    v = ctypes.c_int(0)
+    rc = load_library().seg_attn_take_device_error(ctypes.byref(v))
+    if rc != 0:
+        raise SegAttnError("seg_attn_take_device_error", rc)
+    return v.value
+
+
+@dataclass
+class SegTable:
+    """A built table: host copy, description, device copy and workspace size."""
+    host: torch.Tensor
+    desc: seg_attn_table_desc
+    device: Optional[torch.Tensor] = None
+
+    @classmethod
+    def build(cls, q_lens, seg_starts, seg_lens, num_slots, causal, mode, q_heads, kv_heads,
+              head_dim, pin=False):
+        """Per-request lists in, flattened for seg_attn_build_table."""
+        counts = [len(s) for s in seg_starts]
+        starts = [x for s in seg_starts for x in s]
+        lens = [x for s in seg_lens for x in s]
+        host, desc = seg_attn_build_table(len(counts), q_lens, counts, starts, lens, num_slots,
+                                          causal, mode, q_heads, kv_heads, head_dim, pin=pin)
+        return cls(host=host, desc=desc)
+
+    def to(self, device, non_blocking=False) -> "SegTable":
+        self.device = self.host.to(device, non_blocking=non_blocking)
+        return self
+
+    @property
+    def workspace_bytes(self) -> int:
+        return seg_attn_workspace_size(self.desc)

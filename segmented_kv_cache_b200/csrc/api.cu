@@ -1,0 +1,87 @@
+// C-ABI compute entry points: argument checks, then kernel launches on the
+// caller's stream.  Nothing here allocates, frees or synchronises.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "seg_attn.h"
+#include "seg_attn_internal.h"
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+int check_common(const void* q, const void* k_pool, const void* v_pool, const void* out,
+                 const float* lse, const void* dev_table, const seg_attn_table_desc* desc,
+                 float scale, int mode) {
+  if (!desc || desc->magic != SEG_ATTN_TABLE_MAGIC || desc->version != SEG_ATTN_TABLE_VERSION)
+    return SEG_ATTN_ERR_INVALID_ARG;
+  if (desc->mode != mode) return SEG_ATTN_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !isfinite(scale)) return SEG_ATTN_ERR_INVALID_ARG;
+  if (desc->total_q > 0) {
+    if (!q || !out || !aligned16(q) || !aligned16(out)) return SEG_ATTN_ERR_INVALID_ARG;
+    if (lse && (reinterpret_cast<uintptr_t>(lse) & 3)) return SEG_ATTN_ERR_INVALID_ARG;
+  }
+  if (desc->total_k > 0 && (!k_pool || !v_pool || !aligned16(k_pool) || !aligned16(v_pool)))
+    return SEG_ATTN_ERR_INVALID_ARG;
+  if (desc->num_work > 0 && (!dev_table || !aligned16(dev_table)))
+    return SEG_ATTN_ERR_INVALID_ARG;
+  return SEG_ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" int seg_attn_prefill(const void* q, const void* k_pool, const void* v_pool, void* out,
+                                float* lse, const void* dev_table, const seg_attn_table_desc* desc,
+                                float softmax_scale, void* workspace, size_t workspace_bytes,
+                                void* stream) {
+  (void)workspace;
+  (void)workspace_bytes;
+  int rc = check_common(q, k_pool, v_pool, out, lse, dev_table, desc, softmax_scale,
+                        SEG_ATTN_MODE_PREFILL);
+  if (rc != SEG_ATTN_OK) return rc;
+  if (desc->num_work == 0) return SEG_ATTN_OK;
+  segattn::PrefillLaunch a;
+  a.q = q;
+  a.k_pool = k_pool;
+  a.v_pool = v_pool;
+  a.out = out;
+  a.lse = lse;
+  a.tab = segattn::make_view(dev_table, *desc);
+  a.desc = desc;
+  a.scale = softmax_scale;
+  return segattn::launch_prefill(a, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int seg_attn_decode(const void* q, const void* k_pool, const void* v_pool, void* out,
+                               float* lse, const void* dev_table, const seg_attn_table_desc* desc,
+                               float softmax_scale, void* workspace, size_t workspace_bytes,
+                               void* stream) {
+  int rc = check_common(q, k_pool, v_pool, out, lse, dev_table, desc, softmax_scale,
+                        SEG_ATTN_MODE_DECODE);
+  if (rc != SEG_ATTN_OK) return rc;
+  if (desc->workspace_bytes > 0 &&
+      (!workspace || workspace_bytes < desc->workspace_bytes || !aligned16(workspace)))
+    return SEG_ATTN_ERR_WORKSPACE;
+  if (desc->num_work == 0) return SEG_ATTN_OK;
+  segattn::DecodeLaunch a;
+  a.q = q;
+  a.k_pool = k_pool;
+  a.v_pool = v_pool;
+  a.out = out;
+  a.lse = lse;
+  a.tab = segattn::make_view(dev_table, *desc);
+  a.desc = desc;
+  a.scale = softmax_scale;
+  a.part_o = static_cast<float*>(workspace);
+  a.part_lse = desc->workspace_bytes > 0
+                   ? reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                              segattn::decode_part_o_bytes(*desc))
+                   : nullptr;
+  return segattn::launch_decode(a, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int seg_attn_take_device_error(int* value) {
+  if (!value) return SEG_ATTN_ERR_INVALID_ARG;
+  return segattn::take_device_error(value);
+}

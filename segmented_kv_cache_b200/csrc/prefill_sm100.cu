@@ -1,0 +1,486 @@
+// Chunked-prefill SegmentAttention for sm_100a (tcgen05 + TMEM + TMA).
+//
+// Work item = (request, kv head g, two query tiles).  A query tile is 128
+// rows of (query, head) pairs: 128/G consecutive queries x the G query heads
+// that share kv head g, so every K/V byte fetched serves all G heads, and a
+// small chunk (few new queries per request) still fills the 128 rows.  The
+// two tiles share each K/V tile, which halves L2->SM traffic per flop.
+//
+// K/V tiles are 128 consecutive *logical* keys.  Segments (Flood README,
+// "Introduction": contiguous runs in a shared slot pool) make every row's
+// slot known up front, so the producer warp gathers the tile row by row with
+// TMA gather4 (four pool rows per instruction) straight into the 128-byte
+// swizzled layout the tensor cores read; keys past the end of the request
+// are clamped to its last key and masked.
+//
+// Warp roles (10 warps):
+//   warp 0       TMA producer: Q tiles once, then a 2-stage K ring and a
+//                2-stage V ring.
+//   warp 1       TMEM allocator; lane 0 issues every tcgen05.mma:
+//                  S_t = Q_t K^T   (SS, 128x128xD, fp32 in TMEM)
+//                  O_t += P_t V    (TS: P from TMEM as bf16, V MN-major)
+//                in ping-pong order so one tile's softmax overlaps the other
+//                tile's MMAs.
+//   warps 2-5    softmax for query tile 0, warps 6-9 for tile 1: one thread
+//                per row (its TMEM lane); online softmax (running max m and
+//                normaliser l, as in the Ascend FlashAttention article,
+//                "bottleneck 2") in registers, P written back to TMEM over S,
+//                O rescaled in TMEM only when the max grows by more than 2^8
+//                (the final O / l uses the same reference max, so the result
+//                is unchanged), epilogue O / l -> bf16 and lse.
+// TMEM columns: O0 [0,128) O1 [128,256) S0/P0 [256,384) S1/P1 [384,512).
+// Every mbarrier wait is bounded (1 s); a timeout stops all roles of the CTA,
+// drains in-flight copies and MMAs, frees TMEM and flags a device error.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+#include <math.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "ptx_sm100.cuh"
+#include "seg_attn_internal.h"
+
+namespace segattn {
+
+__device__ int g_device_error;  // non-zero once a bounded wait gave up
+
+namespace {
+
+constexpr int kThreads = 320;
+constexpr uint64_t kWaitLimitNs = 1000000000ull;
+constexpr float kRescaleLog2 = 8.0f;
+constexpr uint32_t kHalfBytes = 128 * 128;  // 128 rows x 64 bf16 (one swizzle-128B panel)
+
+struct PrefillParams {
+  __nv_bfloat16* out;
+  float* lse;
+  TableView tab;
+  float scale_log2;
+  int q_heads, kv_heads, group, qpt, causal;
+};
+
+// Q (2 tiles) + K ring (2) + V ring (2) + barriers + alignment slack.  The
+// d = 64 variant asks for more than half the SM's shared memory as well, so
+// one CTA owns an SM and its 512 tensor-memory columns.
+template <int D>
+constexpr size_t prefill_smem_bytes() {
+  constexpr size_t need = 6 * (D / 64) * (size_t)kHalfBytes + 256 + 1024;
+  return need < 120 * 1024 ? 120 * 1024 : need;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
+  using namespace ptx;
+  constexpr int HALVES = D / 64;
+  constexpr uint32_t TILE = HALVES * kHalfBytes;
+  constexpr int KSTEPS = D / 16;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~static_cast<uintptr_t>(1023));
+  uint8_t* sQ = sm;
+  uint8_t* sK = sm + 2 * TILE;
+  uint8_t* sV = sm + 4 * TILE;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + 6 * TILE);
+  uint64_t* q_full = bars + 0;
+  uint64_t* k_full = bars + 1;   // [2]
+  uint64_t* k_empty = bars + 3;  // [2]
+  uint64_t* v_full = bars + 5;   // [2]
+  uint64_t* v_empty = bars + 7;  // [2]
+  uint64_t* s_full = bars + 9;   // [2] per query tile
+  uint64_t* p_full = bars + 11;  // [2]
+  uint64_t* o_full = bars + 13;  // [2]
+  uint64_t* mma_done = bars + 15;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int4 item = p.tab.work[blockIdx.x];
+  const int req = item.x, g = item.y, q0 = item.z, n_tiles = item.w;
+  const int tok0 = __ldg(p.tab.q_offsets + req);
+  const int q_len = __ldg(p.tab.q_offsets + req + 1) - tok0;
+  const int k_len = __ldg(p.tab.k_lens + req);
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(k_full + s, 1);
+      mbar_init(k_empty + s, 1);
+      mbar_init(v_full + s, 1);
+      mbar_init(v_empty + s, 1);
+      mbar_init(s_full + s, 1);
+      mbar_init(p_full + s, 128);
+      mbar_init(o_full + s, 1);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tm_q);
+    prefetch_tensormap(&tm_k);
+    prefetch_tensormap(&tm_v);
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    int k_issued = 0, v_issued = 0;
+    if (n_tiles > 0) {
+      if (lane == 0) {
+        mbar_expect_tx(q_full, 2 * TILE);
+        for (int t = 0; t < 2; ++t)
+          for (int h = 0; h < HALVES; ++h)
+            tma_load_3d(sQ + t * TILE + h * kHalfBytes, &tm_q, q_full, 64 * h, g * p.group,
+                        tok0 + q0 + t * p.qpt);
+      }
+      int seg = __ldg(p.tab.seg_offsets + req);
+      const int seg_end = __ldg(p.tab.seg_offsets + req + 1);
+      for (int i = 0; i < n_tiles; ++i) {
+        const int st = i & 1;
+        const uint32_t ph = (i >> 1) & 1;
+        int rows[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int j = min(i * kTileKeys + 4 * lane + e, k_len - 1);
+          while (seg + 1 < seg_end && __ldg(p.tab.seg_kstart + seg + 1) <= j) ++seg;
+          const int slot = __ldg(p.tab.seg_start + seg) + (j - __ldg(p.tab.seg_kstart + seg));
+          rows[e] = slot * p.kv_heads + g;
+        }
+        if (!__all_sync(0xffffffffu, mbar_wait(k_empty + st, ph ^ 1, abort_flag, kWaitLimitNs))) break;
+        if (lane == 0) mbar_expect_tx(k_full + st, TILE);
+        __syncwarp();
+#pragma unroll
+        for (int h = 0; h < HALVES; ++h)
+          tma_gather4(sK + st * TILE + h * kHalfBytes + lane * 512, &tm_k, k_full + st, 64 * h,
+                      rows[0], rows[1], rows[2], rows[3]);
+        ++k_issued;
+        if (!__all_sync(0xffffffffu, mbar_wait(v_empty + st, ph ^ 1, abort_flag, kWaitLimitNs))) break;
+        if (lane == 0) mbar_expect_tx(v_full + st, TILE);
+        __syncwarp();
+#pragma unroll
+        for (int h = 0; h < HALVES; ++h)
+          tma_gather4(sV + st * TILE + h * kHalfBytes + lane * 512, &tm_v, v_full + st, 64 * h,
+                      rows[0], rows[1], rows[2], rows[3]);
+        ++v_issued;
+      }
+      // never leave the CTA with copies in flight
+      for (int s = 0; s < 2; ++s) {
+        if (k_issued > s) {
+          const int last = s + 2 * ((k_issued - 1 - s) / 2);
+          mbar_wait(k_full + s, (last >> 1) & 1, nullptr, kWaitLimitNs);
+        }
+        if (v_issued > s) {
+          const int last = s + 2 * ((v_issued - 1 - s) / 2);
+          mbar_wait(v_full + s, (last >> 1) & 1, nullptr, kWaitLimitNs);
+        }
+      }
+      if (lane == 0) mbar_wait(q_full, 0, nullptr, kWaitLimitNs);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && n_tiles > 0) {
+      const uint32_t idesc_qk = idesc_bf16_f32(128, 128, false);
+      const uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
+      const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
+      const uint32_t tS0 = tmem + 256, tO0 = tmem;
+      auto issue_qk = [&](int t, int st) {
+#pragma unroll
+        for (int k = 0; k < KSTEPS; ++k) {
+          const uint32_t off = (k >> 2) * kHalfBytes + (k & 3) * 32;
+          mma_ss(tS0 + 128 * t, sdesc_sw128(q_addr + t * TILE + off, 16, 1024),
+                 sdesc_sw128(k_addr + st * TILE + off, 16, 1024), idesc_qk, k > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int t, int st, bool acc) {
+#pragma unroll
+        for (int k = 0; k < kTileKeys / 16; ++k)
+          mma_ts(tO0 + 128 * t, tS0 + 128 * t + 8 * k,
+                 sdesc_sw128(v_addr + st * TILE + k * 2048, kHalfBytes, 1024), idesc_pv,
+                 (acc || k > 0) ? 1u : 0u);
+      };
+      bool ok = mbar_wait(q_full, 0, abort_flag, kWaitLimitNs) &&
+                mbar_wait(k_full + 0, 0, abort_flag, kWaitLimitNs);
+      if (ok) {
+        tc_fence_after();
+        issue_qk(0, 0);
+        mma_commit(s_full + 0);
+        issue_qk(1, 0);
+        mma_commit(s_full + 1);
+        mma_commit(k_empty + 0);
+      }
+      for (int i = 0; ok && i < n_tiles; ++i) {
+        const int st = i & 1;
+        const uint32_t ph = (i >> 1) & 1;
+        const bool more = i + 1 < n_tiles;
+        const int st1 = (i + 1) & 1;
+        const uint32_t ph1 = ((i + 1) >> 1) & 1;
+        if (!(ok = mbar_wait(v_full + st, ph, abort_flag, kWaitLimitNs))) break;
+        if (!(ok = mbar_wait(p_full + 0, i & 1, abort_flag, kWaitLimitNs))) break;
+        tc_fence_after();
+        issue_pv(0, st, i > 0);
+        mma_commit(o_full + 0);
+        if (more) {
+          if (!(ok = mbar_wait(k_full + st1, ph1, abort_flag, kWaitLimitNs))) break;
+          tc_fence_after();
+          issue_qk(0, st1);
+          mma_commit(s_full + 0);
+        }
+        if (!(ok = mbar_wait(p_full + 1, i & 1, abort_flag, kWaitLimitNs))) break;
+        tc_fence_after();
+        issue_pv(1, st, i > 0);
+        mma_commit(o_full + 1);
+        mma_commit(v_empty + st);
+        if (more) {
+          issue_qk(1, st1);
+          mma_commit(s_full + 1);
+          mma_commit(k_empty + st1);
+        }
+      }
+      // all MMAs finished before tensor memory is released
+      mma_commit(mma_done);
+      mbar_wait(mma_done, 0, nullptr, kWaitLimitNs);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax + epilogue
+    const int t = (warp - 2) >> 2;
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const int qi = q0 + t * p.qpt + row / p.group;
+    const int head = g * p.group + row % p.group;
+    const bool row_valid = qi < q_len;
+    const int vis = p.causal ? min(k_len, k_len - q_len + qi + 1) : k_len;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    const uint32_t tS = lane_base + 256 + 128 * t;
+    const uint32_t tO = lane_base + 128 * t;
+    const float sl2 = p.scale_log2;
+    float m_ref = -INFINITY;  // raw score units
+    float l = 0.f;
+    bool ok = true;
+    for (int i = 0; i < n_tiles; ++i) {
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(s_full + t, i & 1, abort_flag, kWaitLimitNs))))
+        break;
+      tc_fence_after();
+      const int kb = i * kTileKeys;
+      const bool masked = kb + kTileKeys > vis;
+      // pass 1: row max (two 64-column halves)
+      float mx = -INFINITY;
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t a[32], b[32];
+        tmem_ld32(tS + 64 * hh, a);
+        tmem_ld32(tS + 64 * hh + 32, b);
+        tmem_wait_ld(a);
+        tmem_wait_ld(b);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          float x = __uint_as_float(a[e]), y = __uint_as_float(b[e]);
+          if (masked) {
+            if (kb + 64 * hh + e >= vis) x = -INFINITY;
+            if (kb + 64 * hh + 32 + e >= vis) y = -INFINITY;
+          }
+          mx = fmaxf(mx, fmaxf(x, y));
+        }
+      }
+      const float m_new = fmaxf(m_ref, mx);
+      float alpha = 1.f;
+      bool rescale = false;
+      if (m_ref == -INFINITY) {
+        m_ref = m_new;  // nothing accumulated yet for this row (or only zeros)
+      } else if ((m_new - m_ref) * sl2 > kRescaleLog2) {
+        alpha = ex2((m_ref - m_new) * sl2);
+        m_ref = m_new;
+        rescale = true;
+      }
+      l *= alpha;
+      const float base = m_ref == -INFINITY ? 0.f : m_ref * sl2;
+      // pass 2: P = 2^(s*scale*log2e - base) as bf16 pairs into the first 64 S columns;
+      // chunk c+1 is loaded while chunk c is exponentiated (P chunk c only overwrites
+      // S columns that were already read).
+      auto make_p = [&](const uint32_t (&cur)[32], int c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          float x = __uint_as_float(cur[2 * e]), y = __uint_as_float(cur[2 * e + 1]);
+          if (masked) {
+            if (kb + 32 * c + 2 * e >= vis) x = -INFINITY;
+            if (kb + 32 * c + 2 * e + 1 >= vis) y = -INFINITY;
+          }
+          const float pa = ex2(fmaf(x, sl2, -base)), pb = ex2(fmaf(y, sl2, -base));
+          l += pa + pb;
+          pk[e] = pack_bf16(pa, pb);
+        }
+        tmem_st16(tS + 16 * c, pk);
+      };
+      {
+        uint32_t a[32], b[32];
+        tmem_ld32(tS, a);
+        tmem_wait_ld(a);
+        tmem_ld32(tS + 32, b);
+        make_p(a, 0);
+        tmem_wait_ld(b);
+        tmem_ld32(tS + 64, a);
+        make_p(b, 1);
+        tmem_wait_ld(a);
+        tmem_ld32(tS + 96, b);
+        make_p(a, 2);
+        tmem_wait_ld(b);
+        make_p(b, 3);
+      }
+      if (__any_sync(0xffffffffu, rescale)) {
+        // O_t holds PV of the previous tile (S_t of this tile completed after it); rescale in place
+        if (!(ok = __all_sync(0xffffffffu,
+                              mbar_wait(o_full + t, (i - 1) & 1, abort_flag, kWaitLimitNs))))
+          break;
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + 32 * c, o);
+          tmem_wait_ld(o);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st32(tO + 32 * c, o);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(p_full + t);
+    }
+    if (ok && n_tiles > 0)
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait(o_full + t, (n_tiles - 1) & 1, abort_flag, kWaitLimitNs));
+    if (ok) {
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      __nv_bfloat16* orow = p.out + ((int64_t)(tok0 + qi) * p.q_heads + head) * D;
+      if (n_tiles > 0) tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        if (n_tiles > 0) {
+          tmem_ld32(tO + 32 * c, o);
+          tmem_wait_ld(o);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = 0u;
+        }
+        if (row_valid) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 8) {
+            uint4 v;
+            v.x = pack_bf16(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv);
+            v.y = pack_bf16(__uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
+            v.z = pack_bf16(__uint_as_float(o[e + 4]) * inv, __uint_as_float(o[e + 5]) * inv);
+            v.w = pack_bf16(__uint_as_float(o[e + 6]) * inv, __uint_as_float(o[e + 7]) * inv);
+            *reinterpret_cast<uint4*>(orow + 32 * c + e) = v;
+          }
+        }
+      }
+      if (row_valid && p.lse)
+        p.lse[(int64_t)(tok0 + qi) * p.q_heads + head] =
+            l > 0.f ? (m_ref * sl2 + log2f(l)) * 0.69314718055994531f : -INFINITY;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+  if (threadIdx.x == 0 && *abort_flag) atomicOr(&g_device_error, 1);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+bool encode(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims,
+            const cuuint64_t* strides, const cuuint32_t* box) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint32_t elem[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides,
+            box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D>
+int launch_prefill_d(const PrefillLaunch& a, cudaStream_t stream) {
+  const seg_attn_table_desc& d = *a.desc;
+  const int group = d.q_heads / d.kv_heads;
+  CUtensorMap tq, tk, tv;
+  {
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)d.q_heads, (cuuint64_t)d.total_q};
+    const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)d.q_heads * D * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)group, (cuuint32_t)d.queries_per_tile};
+    if (!encode(&tq, a.q, 3, dims, strides, box)) return SEG_ATTN_ERR_CUDA;
+  }
+  {
+    const int64_t rows = d.num_slots * d.kv_heads;
+    const bool empty = rows == 0 || d.total_k == 0;
+    const cuuint64_t dims[2] = {(cuuint64_t)D, empty ? 1ull : (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+    const cuuint32_t box[2] = {64, 1};
+    // with no keys no tile is ever loaded; the query buffer stands in as a valid address
+    if (!encode(&tk, empty ? a.q : a.k_pool, 2, dims, strides, box)) return SEG_ATTN_ERR_CUDA;
+    if (!encode(&tv, empty ? a.q : a.v_pool, 2, dims, strides, box)) return SEG_ATTN_ERR_CUDA;
+  }
+  PrefillParams p;
+  p.out = static_cast<__nv_bfloat16*>(a.out);
+  p.lse = a.lse;
+  p.tab = a.tab;
+  p.scale_log2 = (float)((double)a.scale * 1.4426950408889634);
+  p.q_heads = d.q_heads;
+  p.kv_heads = d.kv_heads;
+  p.group = group;
+  p.qpt = d.queries_per_tile;
+  p.causal = d.causal;
+  constexpr size_t smem = prefill_smem_bytes<D>();
+  if (cudaFuncSetAttribute(prefill_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return SEG_ATTN_ERR_CUDA;
+  prefill_kernel<D><<<d.num_work, kThreads, smem, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? SEG_ATTN_OK : SEG_ATTN_ERR_CUDA;
+}
+
+}  // namespace
+
+int launch_prefill(const PrefillLaunch& a, cudaStream_t stream) {
+  return a.desc->head_dim == 128 ? launch_prefill_d<128>(a, stream)
+                                 : launch_prefill_d<64>(a, stream);
+}
+
+int take_device_error(int* value) {
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int)) != cudaSuccess) return SEG_ATTN_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess) return SEG_ATTN_ERR_CUDA;
+  *value = v;
+  return SEG_ATTN_OK;
+}
+
+}  // namespace segattn

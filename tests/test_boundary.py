@@ -1,0 +1,172 @@
+"""The C ABI without a GPU: the library loads, exports what include/*.h declares,
+and the host-side table builder / argument checks behave as documented."""
+import ctypes
+import glob
+import os
+import re
+
+import numpy as np
+import pytest
+import torch
+
+import segmented_kv_cache_b200 as sa
+from segmented_kv_cache_b200 import _build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+S = sa.STATUS
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built_library():
+    _build.build()
+    return sa.load_library()
+
+
+def declared_functions():
+    names = []
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names += re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b(seg_attn_\w+)\s*\(", text, re.M)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(built_library):
+    names = declared_functions()
+    assert {"seg_attn_build_table", "seg_attn_prefill", "seg_attn_decode",
+            "seg_attn_workspace_size", "seg_attn_status_string"} <= set(names)
+    for n in names:
+        assert hasattr(built_library, n), n
+
+
+def test_status_strings_and_version():
+    for name, code in S.items():
+        assert sa.seg_attn_status_string(code)
+    assert sa.seg_attn_status_string(12345) == "unknown status"
+    assert sa.seg_attn_version() >= 100
+
+
+def build(q_lens, segs, num_slots=100, causal=True, mode=sa.MODE_PREFILL, hq=8, hkv=2, d=128):
+    starts = [[s for s, _ in r] for r in segs]
+    lens = [[l for _, l in r] for r in segs]
+    return sa.SegTable.build(q_lens, starts, lens, num_slots, causal, mode, hq, hkv, d)
+
+
+def code_of(fn):
+    with pytest.raises(sa.SegAttnError) as e:
+        fn()
+    return e.value.code
+
+
+def test_validation_errors():
+    assert code_of(lambda: build([2], [[(95, 10)]])) == S["SEGMENT_OOB"]
+    assert code_of(lambda: build([2], [[(-1, 3)]])) == S["SEGMENT_OOB"]
+    assert code_of(lambda: build([2], [[(10, 5), (12, 4)]])) == S["SEGMENT_OVERLAP"]
+    assert code_of(lambda: build([5], [[(10, 4)]])) == S["QLEN_GT_KLEN"]
+    # non-causal prefill may have more queries than keys
+    build([5], [[(10, 4)]], causal=False)
+    assert code_of(lambda: build([2], [[(10, -1)]])) == S["INVALID_ARG"]
+    assert code_of(lambda: build([-1], [[(10, 4)]])) == S["INVALID_ARG"]
+    assert code_of(lambda: build([1], [[(10, 4)]], hq=6, hkv=4)) == S["INVALID_ARG"]
+    assert code_of(lambda: build([1], [[(10, 4)]], d=96)) == S["UNSUPPORTED"]
+    assert code_of(lambda: build([1], [[(10, 4)]], hq=6, hkv=2)) == S["UNSUPPORTED"]  # G=3
+    assert code_of(lambda: build([1], [[(10, 4)]], hq=32, hkv=2, mode=sa.MODE_DECODE)) == S["UNSUPPORTED"]
+    assert code_of(lambda: build([2], [[(10, 4)]], mode=sa.MODE_DECODE)) == S["INVALID_ARG"]
+    # the same slots in two requests are legal (shared read-only prefix)
+    build([1, 1], [[(10, 4)], [(10, 4)]])
+    # int32 pool row index limit
+    assert code_of(lambda: build([1], [[(0, 4)]], num_slots=2**30, hkv=2)) == S["UNSUPPORTED"]
+
+
+def test_size_query_and_small_buffer():
+    lib = sa.load_library()
+    desc = sa.seg_attn_table_desc()
+    q = np.array([3], np.int32)
+    c = np.array([1], np.int32)
+    st = np.array([4], np.int32)
+    ln = np.array([7], np.int32)
+    P = lambda a: ctypes.c_void_p(a.ctypes.data)
+    rc = lib.seg_attn_build_table(1, P(q), P(c), P(st), P(ln), 20, 1, 0, 8, 2, 128, None, 0,
+                                  ctypes.byref(desc))
+    assert rc == 0 and desc.table_bytes > 0 and desc.magic == 0x53454741
+    buf = np.zeros(desc.table_bytes // 4 - 1, np.int32)
+    rc = lib.seg_attn_build_table(1, P(q), P(c), P(st), P(ln), 20, 1, 0, 8, 2, 128, P(buf),
+                                  buf.nbytes, ctypes.byref(desc))
+    assert rc == S["BUFFER_TOO_SMALL"]
+    assert lib.seg_attn_build_table(1, P(q), P(c), P(st), P(ln), 20, 1, 0, 8, 2, 128, None, 0,
+                                    None) == S["INVALID_ARG"]
+
+
+def view(tab, off, n):
+    return tab.host[off: off + n].tolist()
+
+
+def test_prefill_table_contents():
+    tab = build([3, 0, 40], [[(50, 2), (10, 5)], [(0, 3)], [(20, 20), (60, 30)]], num_slots=100,
+                hq=8, hkv=2)
+    d = tab.desc
+    assert d.batch == 3 and d.total_q == 43 and d.total_k == 60 and d.num_segments == 5
+    assert view(tab, d.off_q_offsets, 4) == [0, 3, 3, 43]
+    assert view(tab, d.off_k_lens, 3) == [7, 3, 50]
+    assert view(tab, d.off_seg_offsets, 4) == [0, 2, 3, 5]
+    assert view(tab, d.off_seg_start, 5) == [50, 10, 0, 20, 60]
+    assert view(tab, d.off_seg_kstart, 5) == [0, 2, 0, 0, 20]
+    assert view(tab, d.off_seg_len, 5) == [2, 5, 3, 20, 30]
+    assert d.off_work % 4 == 0 and d.queries_per_tile == 32  # 128 rows / group 4
+    work = np.array(view(tab, d.off_work, 4 * d.num_work)).reshape(-1, 4)
+    # request 0: one pair x 2 kv heads; request 2: 40 queries -> 1 pair (64 per pair) x 2 heads
+    assert len(work) == 4 and sorted(set(work[:, 0])) == [0, 2]
+    assert list(work[:, 3]) == sorted(work[:, 3], reverse=True)  # longest first
+    # causal tile count: last query of request 2 sees all 50 keys -> 1 tile of 128
+    assert all(w[3] == 1 for w in work)
+
+
+def test_decode_chunks_cover_each_request():
+    k = [5000, 1, 0, 2049]
+    segs = [[(0, 5000)], [(6000, 1)], [], [(7000, 1000), (9000, 1049)]]
+    tab = build([1] * 4, segs, num_slots=20000, mode=sa.MODE_DECODE, hq=8, hkv=1)
+    d = tab.desc
+    L = d.chunk_len
+    assert L >= 256 and d.workspace_bytes > 0
+    work = np.array(view(tab, d.off_work, 4 * d.num_work)).reshape(-1, 4)
+    rc = view(tab, d.off_req_chunks, 5)
+    for r in range(4):
+        w = work[rc[r]: rc[r + 1]]
+        assert (w[:, 0] == r).all()
+        assert w[0, 1] == 0 and w[-1, 2] == k[r]
+        assert (w[1:, 1] == w[:-1, 2]).all()
+        assert (w[:, 3] == len(w)).all()
+        assert ((w[:, 2] - w[:, 1]) <= L).all()
+
+
+def test_compute_calls_reject_bad_arguments_before_any_launch():
+    # all of these fail host-side checks; no CUDA call is made
+    tab = build([2], [[(10, 5)]])
+    fake = torch.zeros(16, dtype=torch.uint8)
+    p = lambda: ctypes.c_void_p(fake.data_ptr())
+    lib = sa.load_library()
+    desc = tab.desc
+    call = lambda fn, scale, dsc=desc, q=None, ws=None, wsb=0: getattr(lib, fn)(
+        q if q is not None else p(), p(), p(), p(), None, p(), ctypes.byref(dsc), scale,
+        ws, wsb, None)
+    assert call("seg_attn_prefill", 0.0) == S["INVALID_ARG"]
+    assert call("seg_attn_prefill", float("nan")) == S["INVALID_ARG"]
+    assert call("seg_attn_decode", 0.1) == S["INVALID_ARG"]  # table built for prefill
+    assert call("seg_attn_prefill", 0.1, q=ctypes.c_void_p(fake.data_ptr() + 2)) == S["INVALID_ARG"]
+    bad = sa.seg_attn_table_desc.from_buffer_copy(desc)
+    bad.magic = 0
+    assert call("seg_attn_prefill", 0.1, dsc=bad) == S["INVALID_ARG"]
+    dtab = build([1, 1], [[(0, 3000)], [(4000, 10)]], num_slots=5000, mode=sa.MODE_DECODE, hq=8,
+                 hkv=1)
+    assert dtab.desc.workspace_bytes > 0
+    assert call("seg_attn_decode", 0.1, dsc=dtab.desc) == S["WORKSPACE"]
+    assert call("seg_attn_decode", 0.1, dsc=dtab.desc, ws=p(), wsb=16) == S["WORKSPACE"]
+
+
+def test_empty_batch_is_a_noop():
+    tab = build([], [], num_slots=0)
+    assert tab.desc.num_work == 0 and tab.desc.total_q == 0
+    lib = sa.load_library()
+    rc = lib.seg_attn_prefill(None, None, None, None, None, None, ctypes.byref(tab.desc), 0.1,
+                              None, 0, None)
+    assert rc == 0

@@ -1,0 +1,130 @@
+"""GPU parity of seg_attn_decode (split-K + log-sum-exp merge) against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import segmented_kv_cache_b200 as sa
+from segmented_kv_cache_b200 import synth
+
+from helpers import compact_requests, compare, random_case, run_batch, run_cuda
+
+pytestmark = pytest.mark.gpu
+
+
+def _dev(case):
+    return {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in case.items()}
+
+
+def _check_case(case, what):
+    c = _dev(case)
+    out, lse, tab = run_cuda(c["q"], c["k_pool"], c["v_pool"], None, c["seg_starts"],
+                             c["seg_lens"], c["num_slots"], True, sa.MODE_DECODE, c["scale"])
+    torch.cuda.synchronize()
+    ref_o, ref_l = oracle.attention(case["q_lens"], case["seg_starts"], case["seg_lens"],
+                                    case["q"], case["k_pool"], case["v_pool"], case["scale"], True)
+    return compare(out, lse, ref_o, ref_l, what), tab
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("hq,hkv", [(8, 1), (16, 4), (4, 2), (8, 8)])
+def test_decode_random(d, hq, hkv):
+    case = random_case(100 + d + hq + hkv, batch=5, hq=hq, hkv=hkv, d=d, causal=True, max_k=3000,
+                       nseg_max=6, q_mode="decode")
+    _check_case(case, f"decode d{d} {hq}/{hkv}")
+
+
+def test_decode_multichunk_and_single_chunk_requests():
+    # long requests split into many chunks, short ones use the single-chunk path
+    case = random_case(7, batch=6, hq=64, hkv=8, d=128, causal=True, max_k=9000, nseg_max=8,
+                       q_mode="decode")
+    case["seg_starts"][1], case["seg_lens"][1] = case["seg_starts"][1][:1], [1]
+    summary, tab = _check_case(case, "decode mixed")
+    rc = tab.host[tab.desc.off_req_chunks: tab.desc.off_req_chunks + 7].tolist()
+    n = np.diff(rc)
+    assert n.max() > 1 and n.min() == 1
+
+
+def test_decode_zero_length_request():
+    case = random_case(8, batch=3, hq=8, hkv=1, d=128, causal=True, max_k=700, q_mode="decode")
+    case["seg_starts"][1], case["seg_lens"][1] = [], []
+    c = _dev(case)
+    out, lse, _ = run_cuda(c["q"], c["k_pool"], c["v_pool"], None, c["seg_starts"], c["seg_lens"],
+                           c["num_slots"], True, sa.MODE_DECODE, c["scale"])
+    torch.cuda.synchronize()
+    assert torch.all(out[1] == 0) and torch.all(torch.isneginf(lse[1]))
+    ref_o, ref_l = oracle.attention(case["q_lens"], case["seg_starts"], case["seg_lens"],
+                                    case["q"], case["k_pool"], case["v_pool"], case["scale"], True)
+    compare(out, lse, ref_o, ref_l, "decode k=0")
+
+
+def test_decode_ragged_chunk_tails_and_tiny_segments():
+    # segments of length 1..3 force the per-key slot lookup on every block
+    case = random_case(9, batch=4, hq=8, hkv=2, d=128, causal=True, max_k=1500, nseg_max=1,
+                       q_mode="decode")
+    g = torch.Generator().manual_seed(3)
+    pool_k, pool_v = case["k_pool"], case["v_pool"]
+    new_s, new_l = [], []
+    for ss, ll in zip(case["seg_starts"], case["seg_lens"]):
+        s2, l2 = [], []
+        for s, l in zip(ss, ll):
+            pos = s
+            while pos < s + l:
+                step = min(int(torch.randint(1, 4, (1,), generator=g)), s + l - pos)
+                s2.append(pos)
+                l2.append(step)
+                pos += step
+        new_s.append(s2)
+        new_l.append(l2)
+    case["seg_starts"], case["seg_lens"] = new_s, new_l
+    _check_case(case, "decode tiny segments")
+
+
+def test_decode_split_choice_does_not_change_result():
+    # the same request as one chunk (short) and as part of a multi-chunk batch
+    case = random_case(10, batch=1, hq=8, hkv=1, d=128, causal=True, max_k=2000, q_mode="decode")
+    c = _dev(case)
+    out1, lse1, t1 = run_cuda(c["q"], c["k_pool"], c["v_pool"], None, c["seg_starts"],
+                              c["seg_lens"], c["num_slots"], True, sa.MODE_DECODE, c["scale"])
+    rep = 40
+    out2, lse2, t2 = run_cuda(c["q"].repeat(rep, 1, 1), c["k_pool"], c["v_pool"], None,
+                              c["seg_starts"] * rep, c["seg_lens"] * rep, c["num_slots"], True,
+                              sa.MODE_DECODE, c["scale"])
+    torch.cuda.synchronize()
+    assert t1.desc.chunk_len != t2.desc.chunk_len
+    assert (out2.float() - out1.float()).abs().max() <= 2 ** -7
+    assert (lse2 - lse1).abs().max() <= 1e-5
+
+
+@pytest.mark.parametrize("cfg", [4])
+def test_config4_sampled_requests(cfg):
+    wl = synth.make_workload(cfg, device="cuda")
+    b = wl.batches[0]
+    out, lse, _ = run_batch(wl, b)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out.float()).all()
+    g = torch.Generator().manual_seed(11)
+    k = np.array(b.k_lens)
+    reqs = sorted(set([int(k.argmax()), int(k.argmin())] +
+                      torch.randint(0, b.batch, (4,), generator=g).tolist()))
+    sub = compact_requests(wl, b, reqs)
+    ref_o, ref_l = oracle.attention(sub["q_lens"], sub["seg_starts"], sub["seg_lens"], sub["q"],
+                                    sub["k_pool"], sub["v_pool"], wl.scale, True)
+    rows = sub["q_rows"].cuda()
+    compare(out[rows], lse[rows], ref_o, ref_l, "config 4")
+
+
+def test_config5_decode_sampled():
+    wl = synth.make_workload(5, device="cuda")
+    b = wl.batches[0]
+    out, lse, _ = run_batch(wl, b)
+    torch.cuda.synchronize()
+    sub = compact_requests(wl, b, [0, 5])
+    ref_o, ref_l = oracle.attention(sub["q_lens"], sub["seg_starts"], sub["seg_lens"], sub["q"],
+                                    sub["k_pool"], sub["v_pool"], wl.scale, True)
+    rows = sub["q_rows"].cuda()
+    compare(out[rows], lse[rows], ref_o, ref_l, "config 5 decode")
+
+
+def test_no_device_error_recorded():
+    assert sa.seg_attn_take_device_error() == 0

@@ -1,0 +1,151 @@
+"""GPU parity of seg_attn_prefill (tcgen05 / TMEM / TMA gather) against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import segmented_kv_cache_b200 as sa
+from segmented_kv_cache_b200 import synth
+
+from helpers import compact_requests, compare, random_case, run_batch, run_cuda
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(case, causal=None):
+    causal = case["causal"] if causal is None else causal
+    dev = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in case.items()}
+    out, lse, tab = run_cuda(dev["q"], dev["k_pool"], dev["v_pool"], case["q_lens"],
+                             case["seg_starts"], case["seg_lens"], case["num_slots"], causal,
+                             sa.MODE_PREFILL, case["scale"])
+    torch.cuda.synchronize()
+    return out, lse, tab
+
+
+def _check(case, what):
+    out, lse, tab = _run(case)
+    ref_o, ref_l = oracle.attention(case["q_lens"], case["seg_starts"], case["seg_lens"],
+                                    case["q"], case["k_pool"], case["v_pool"], case["scale"],
+                                    case["causal"])
+    return compare(out, lse, ref_o, ref_l, what)
+
+
+def test_config1_tiny():
+    wl = synth.make_workload(1)
+    b = wl.batches[0]
+    case = dict(q=b.q, k_pool=wl.k_pool, v_pool=wl.v_pool, q_lens=b.q_lens,
+                seg_starts=b.seg_starts, seg_lens=b.seg_lens, num_slots=wl.num_slots,
+                scale=wl.scale, causal=b.causal)
+    _check(case, "config 1")
+
+
+def test_config2_pages_shaped_full():
+    wl = synth.make_workload(2)
+    b = wl.batches[0]
+    case = dict(q=b.q, k_pool=wl.k_pool, v_pool=wl.v_pool, q_lens=b.q_lens,
+                seg_starts=b.seg_starts, seg_lens=b.seg_lens, num_slots=wl.num_slots,
+                scale=wl.scale, causal=b.causal)
+    _check(case, "config 2")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("hq,hkv", [(8, 1), (8, 2), (4, 4), (32, 2)])
+@pytest.mark.parametrize("causal", [True, False])
+def test_prefill_random(d, hq, hkv, causal):
+    case = random_case(1000 + d + 7 * hq + hkv + causal, batch=4, hq=hq, hkv=hkv, d=d,
+                       causal=causal, max_k=700, nseg_max=5, q_mode="chunk")
+    _check(case, f"prefill d{d} {hq}/{hkv} causal={causal}")
+
+
+def test_prefill_full_causal_many_tiles():
+    # q = k (no prior context): diagonal masking on every tile of both query tiles
+    case = random_case(21, batch=3, hq=16, hkv=2, d=128, causal=True, max_k=900, nseg_max=3,
+                       q_mode="full")
+    _check(case, "full causal")
+
+
+def test_prefill_tiny_segments_gather():
+    # 1..3-slot segments: every gathered row comes from a different run
+    case = random_case(22, batch=2, hq=8, hkv=1, d=128, causal=True, max_k=400, nseg_max=1)
+    g = torch.Generator().manual_seed(4)
+    new_s, new_l = [], []
+    for ss, ll in zip(case["seg_starts"], case["seg_lens"]):
+        s2, l2 = [], []
+        for s, l in zip(ss, ll):
+            pos = s
+            while pos < s + l:
+                step = min(int(torch.randint(1, 4, (1,), generator=g)), s + l - pos)
+                s2.append(pos)
+                l2.append(step)
+                pos += step
+        new_s.append(s2)
+        new_l.append(l2)
+    case["seg_starts"], case["seg_lens"] = new_s, new_l
+    _check(case, "tiny segments")
+
+
+def test_prefill_zero_keys_noncausal_and_zero_queries():
+    case = random_case(23, batch=3, hq=8, hkv=2, d=128, causal=False, max_k=300)
+    case["q_lens"] = [3, 0, 2]
+    case["q"] = case["q"][:5] if case["q"].shape[0] >= 5 else torch.randn(5, 8, 128).to(torch.bfloat16)
+    case["seg_starts"][2], case["seg_lens"][2] = [], []
+    out, lse, _ = _run(case)
+    assert torch.all(out[3:] == 0) and torch.all(torch.isneginf(lse[3:]))
+    ref_o, ref_l = oracle.attention(case["q_lens"], case["seg_starts"], case["seg_lens"],
+                                    case["q"], case["k_pool"], case["v_pool"], case["scale"], False)
+    compare(out, lse, ref_o, ref_l, "zero keys")
+
+
+def test_prefill_large_scores_trigger_rescale():
+    # scaled-up queries make the running max jump by more than 2^8 across tiles
+    case = random_case(24, batch=2, hq=8, hkv=1, d=128, causal=True, max_k=800, q_mode="full")
+    case["scale"] = 0.5
+    _check(case, "rescale")
+
+
+def test_decode_row_equals_last_prefill_row():
+    case = random_case(25, batch=2, hq=8, hkv=1, d=128, causal=True, max_k=600, q_mode="full")
+    out, lse, _ = _run(case)
+    last = np.cumsum(case["q_lens"]) - 1
+    dev = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in case.items()}
+    out_d, lse_d, _ = run_cuda(dev["q"][torch.tensor(last).cuda()], dev["k_pool"], dev["v_pool"],
+                               None, case["seg_starts"], case["seg_lens"], case["num_slots"], True,
+                               sa.MODE_DECODE, case["scale"])
+    torch.cuda.synchronize()
+    assert (out_d.float() - out[last].float()).abs().max() <= 2 ** -7
+    assert (lse_d - lse[last]).abs().max() <= 1e-4
+
+
+def test_config3_sampled_requests():
+    wl = synth.make_workload(3, device="cuda")
+    b = wl.batches[0]
+    out, lse, _ = run_batch(wl, b)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out.float()).all()
+    reqs = [r for r in range(b.batch) if b.q_lens[r] > 0][:3]
+    sub = compact_requests(wl, b, reqs)
+    ref_o, ref_l = oracle.attention(sub["q_lens"], sub["seg_starts"], sub["seg_lens"], sub["q"],
+                                    sub["k_pool"], sub["v_pool"], wl.scale, True)
+    rows = sub["q_rows"].cuda()
+    compare(out[rows], lse[rows], ref_o, ref_l, "config 3")
+
+
+def test_config5_prefill_sampled_rows():
+    wl = synth.make_workload(5, device="cuda")
+    b = wl.batches[1]
+    out, lse, _ = run_batch(wl, b)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out.float()).all()
+    sub = compact_requests(wl, b, [0])
+    g = torch.Generator().manual_seed(5)
+    toks = torch.cat([torch.tensor([0, 2047]), torch.randint(0, 2048, (14,), generator=g)])
+    heads = torch.randint(0, wl.q_heads, (toks.numel(),), generator=g)
+    ref_o, ref_l = oracle.attention(sub["q_lens"], sub["seg_starts"], sub["seg_lens"], sub["q"],
+                                    sub["k_pool"], sub["v_pool"], wl.scale, True,
+                                    rows=(toks.numpy(), heads.numpy()))
+    compare(out[toks.cuda(), heads.cuda()], lse[toks.cuda(), heads.cuda()], ref_o, ref_l,
+            "config 5 prefill")
+
+
+def test_no_device_error_recorded():
+    assert sa.seg_attn_take_device_error() == 0

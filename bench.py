@@ -251,7 +251,8 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    wl = synth.make_workload(args.config, device="cuda" if torch.cuda.is_available() else "cpu")
+    wl = synth.make_workload(args.config, device="cuda" if torch.cuda.is_available() else "cpu",
+                             context_scale=args.context_scale)
     rows = [args.ref_rows] * len(wl.batches)
     for _ in range(args.warmup if args.warmup <= 1 else 1):
         oracle_sample(wl, wl.batches, [max(1, r // 8) for r in rows], rng_seed=99)
@@ -291,7 +292,8 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=device)
     # weak scaling: every rank runs its own batch of the same shape (seed offset by rank)
-    wl = synth.make_workload(args.config, device=str(device), seed=args.config - 1 + 1000 * rank)
+    wl = synth.make_workload(args.config, device=str(device), seed=args.config - 1 + 1000 * rank,
+                             context_scale=args.context_scale)
     path = Path(wl, device)
     stream = torch.cuda.current_stream(device)
 
@@ -381,7 +383,9 @@ def run_ours(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": workload_name(wl), "seed": wl.config - 1,
+            "config": {"workload": workload_name(wl) + ("" if args.context_scale == 1.0 else
+                                                       f" (context x{args.context_scale})"),
+                       "seed": wl.config - 1,
                        "q_heads": wl.q_heads, "kv_heads": wl.kv_heads, "head_dim": wl.head_dim,
                        "num_slots": wl.num_slots,
                        "l2": ("inputs larger than L2 (pools %.1f GB), no flush" %
@@ -484,6 +488,8 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=256,
                     help="oracle rows per batch for the cpu_baseline leg of our arm")
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--context-scale", type=float, default=1.0,
+                    help="shorten the long-context mix (profiling captures only; 1.0 = as specified)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

@@ -133,8 +133,11 @@ def _pool_values(num_slots, kv_heads, head_dim, live, gen, device, std):
     return pool
 
 
-def _structure(cfg: int, gen: torch.Generator):
-    """Lengths, segment counts and cut points of each config (no values)."""
+def _structure(cfg: int, gen: torch.Generator, context_scale: float = 1.0):
+    """Lengths, segment counts and cut points of each config (no values).
+
+    ``context_scale`` shortens the long-context mix (config 5) for profiling
+    runs that must stay small; every other config ignores it."""
     if cfg == 1:
         q_lens = [16, 33]
         seg_lens = [[8, 8], [17, 16]]
@@ -161,8 +164,9 @@ def _structure(cfg: int, gen: torch.Generator):
         return dict(q_heads=64, kv_heads=8, head_dim=128, num_slots=slots,
                     batches=[("decode", [1] * B, seg_lens, True)], qk_std=1.0)
     if cfg == 5:
-        k_dec = [131072] * 8
-        k_pre = [131072 + 2048]
+        ctx = max(1024, int(131072 * context_scale))
+        k_dec = [ctx] * 8
+        k_pre = [ctx + 2048]
         nsegs = torch.randint(4, 17, (9,), generator=gen).tolist()
         lens_all = [split_uniform_cuts(k, n, gen) for k, n in zip(k_dec + k_pre, nsegs)]
         slots = math.ceil(1.1 * (sum(k_dec) + sum(k_pre)))
@@ -173,11 +177,11 @@ def _structure(cfg: int, gen: torch.Generator):
 
 
 def make_workload(cfg: int, device: str = "cpu", values: bool = True,
-                  seed: Optional[int] = None) -> Workload:
+                  seed: Optional[int] = None, context_scale: float = 1.0) -> Workload:
     """Build config ``cfg`` (1..5).  Seed defaults to cfg - 1."""
     seed = cfg - 1 if seed is None else seed
     gen = torch.Generator(device="cpu").manual_seed(seed)
-    st = _structure(cfg, gen)
+    st = _structure(cfg, gen, context_scale)
     batches = []
     all_lens = []
     for mode, q_lens, seg_lens, causal in st["batches"]:

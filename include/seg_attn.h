@@ -172,6 +172,30 @@ int seg_attn_decode(const void* q, const void* k_pool, const void* v_pool, void*
  */
 int seg_attn_take_device_error(int* value);
 
+/*
+ * seg_attn_decode_noalloc -- seg_attn_decode for callers that cannot allocate
+ * device memory (no counterpart on the source pages; this is a library
+ * convenience).  Typical callers: a plugin inside another runtime that owns
+ * all device memory and offers no allocator, or a serving loop that must not
+ * call cudaMalloc after start-up because it can synchronise the device.
+ *
+ * Same arguments and results as seg_attn_decode, minus the workspace: the
+ * split-K scratch is a fixed 64 MiB device array inside the library, which
+ * every GPU that loads the library keeps until the process exits.
+ *   - Returns SEG_ATTN_ERR_WORKSPACE, launching nothing, when the table needs
+ *     more than 64 MiB of scratch (seg_attn_workspace_size(desc) > 64 MiB).
+ *   - All calls share the array and it keeps the last call's contents; no
+ *     part of it needs to start at zero.  Calls that overlap on the GPU (other
+ *     streams or host threads) race on it: order them, e.g. on one stream.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before starting any stream capture.
+ *   - Calls no cudaMalloc, cudaFree or other allocating routine.
+ */
+int seg_attn_decode_noalloc(const void* q, const void* k_pool, const void* v_pool, void* out,
+                            float* lse, const void* dev_table, const seg_attn_table_desc* desc,
+                            float softmax_scale, void* stream);
+
 /* Static English description of a status code (never NULL). */
 const char* seg_attn_status_string(int status);
 

@@ -51,6 +51,12 @@ namespace {
 constexpr int kThreads = 320;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
 constexpr float kRescaleLog2 = 8.0f;
+// Of every 16 pairs of scores, this many are exponentiated with the FMA-pipe
+// polynomial instead of the SFU, to balance the two pipes.
+#ifndef SEG_ATTN_EXP2_POLY_PAIRS
+#define SEG_ATTN_EXP2_POLY_PAIRS 0
+#endif
+constexpr int kPolyPairs = SEG_ATTN_EXP2_POLY_PAIRS;
 constexpr uint32_t kHalfBytes = 128 * 128;  // 128 rows x 64 bf16 (one swizzle-128B panel)
 
 struct PrefillParams {
@@ -270,14 +276,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m_ref = -INFINITY;  // raw score units
     float l = 0.f;
     bool ok = true;
-    for (int i = 0; i < n_tiles; ++i) {
-      if (!(ok = __all_sync(0xffffffffu, mbar_wait(s_full + t, i & 1, abort_flag, kWaitLimitNs))))
-        break;
-      tc_fence_after();
+    // Causal / tail mask of tile i, applied in place in tensor memory (-inf in
+    // the columns this row must not see).  Only tiles where some row of the warp
+    // needs it pay for it; the softmax itself never compares per element.
+    auto mask_tile = [&](int i) {
       const int kb = i * kTileKeys;
-      const bool masked = kb + kTileKeys > vis;
-      // pass 1: row max (two 64-column halves)
-      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t a[32];
+        tmem_ld32(tS + 32 * c, a);
+        tmem_wait_ld(a);
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          if (kb + 32 * c + e >= vis) a[e] = 0xff800000u;  // -inf
+        tmem_st32(tS + 32 * c, a);
+      }
+      tmem_wait_st();
+    };
+    // One tile of the online softmax (S already masked where needed).
+    auto softmax_tile = [&](int i) -> bool {
+      auto f = [](uint32_t bits) { return __uint_as_float(bits); };
+      // pass 1: row max (two 64-column halves, four independent chains)
+      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         uint32_t a[32], b[32];
@@ -286,16 +306,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld(a);
         tmem_wait_ld(b);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          float x = __uint_as_float(a[e]), y = __uint_as_float(b[e]);
-          if (masked) {
-            if (kb + 64 * hh + e >= vis) x = -INFINITY;
-            if (kb + 64 * hh + 32 + e >= vis) y = -INFINITY;
-          }
-          mx = fmaxf(mx, fmaxf(x, y));
+        for (int e = 0; e < 32; e += 2) {
+          const int k = (e >> 1) & 1;
+          mx[k] = fmaxf(mx[k], fmaxf(f(a[e]), f(a[e + 1])));
+          mx[2 + k] = fmaxf(mx[2 + k], fmaxf(f(b[e]), f(b[e + 1])));
         }
       }
-      const float m_new = fmaxf(m_ref, mx);
+      const float row_max = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+      const float m_new = fmaxf(m_ref, row_max);
       float alpha = 1.f;
       bool rescale = false;
       if (m_ref == -INFINITY) {
@@ -305,22 +323,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         m_ref = m_new;
         rescale = true;
       }
-      l *= alpha;
       const float base = m_ref == -INFINITY ? 0.f : m_ref * sl2;
       // pass 2: P = 2^(s*scale*log2e - base) as bf16 pairs into the first 64 S columns;
       // chunk c+1 is loaded while chunk c is exponentiated (P chunk c only overwrites
       // S columns that were already read).
-      auto make_p = [&](const uint32_t (&cur)[32], int c) {
+      float ls[2] = {0.f, 0.f};
+      auto make_p = [&](const uint32_t (&cur)[32], int c) {  // S chunk c -> P columns [16c, 16c+16)
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          float x = __uint_as_float(cur[2 * e]), y = __uint_as_float(cur[2 * e + 1]);
-          if (masked) {
-            if (kb + 32 * c + 2 * e >= vis) x = -INFINITY;
-            if (kb + 32 * c + 2 * e + 1 >= vis) y = -INFINITY;
-          }
-          const float pa = ex2(fmaf(x, sl2, -base)), pb = ex2(fmaf(y, sl2, -base));
-          l += pa + pb;
+          const float xa = fmaf(f(cur[2 * e]), sl2, -base);
+          const float xb = fmaf(f(cur[2 * e + 1]), sl2, -base);
+          const bool poly = kPolyPairs > 0 && (e % 16) * kPolyPairs / 16 != ((e % 16) + 1) * kPolyPairs / 16;
+          const float pa = poly ? exp2_poly(xa) : ex2(xa);
+          const float pb = poly ? exp2_poly(xb) : ex2(xb);
+          ls[0] += pa;
+          ls[1] += pb;
           pk[e] = pack_bf16(pa, pb);
         }
         tmem_st16(tS + 16 * c, pk);
@@ -340,11 +358,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld(b);
         make_p(b, 3);
       }
+      l = l * alpha + (ls[0] + ls[1]);
       if (__any_sync(0xffffffffu, rescale)) {
         // O_t holds PV of the previous tile (S_t of this tile completed after it); rescale in place
-        if (!(ok = __all_sync(0xffffffffu,
-                              mbar_wait(o_full + t, (i - 1) & 1, abort_flag, kWaitLimitNs))))
-          break;
+        if (!__all_sync(0xffffffffu, mbar_wait(o_full + t, (i - 1) & 1, abort_flag, kWaitLimitNs)))
+          return false;
         tc_fence_after();
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
@@ -356,6 +374,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_st32(tO + 32 * c, o);
         }
       }
+      return true;
+    };
+    for (int i = 0; i < n_tiles; ++i) {
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(s_full + t, i & 1, abort_flag, kWaitLimitNs))))
+        break;
+      tc_fence_after();
+      const bool masked = __any_sync(0xffffffffu, (i + 1) * kTileKeys > vis);
+      if (masked) mask_tile(i);
+      ok = softmax_tile(i);
+      if (!ok) break;
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(p_full + t);

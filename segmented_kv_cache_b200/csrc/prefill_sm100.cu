@@ -11,7 +11,10 @@
 // slot known up front, so the producer warp gathers the tile row by row with
 // TMA gather4 (four pool rows per instruction) straight into the 128-byte
 // swizzled layout the tensor cores read; keys past the end of the request
-// are clamped to its last key and masked.
+// are clamped to its last key and masked.  A tile whose 128 keys are 128
+// consecutive pool slots (the common case: segments are long) is instead
+// loaded as two tiled boxes, which the TMA engine moves far faster than 64
+// four-row gathers.
 //
 // Warp roles (10 warps):
 //   warp 0       TMA producer: Q tiles once, then a 2-stage K ring and a
@@ -84,7 +87,8 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_k3,
+                   const __grid_constant__ CUtensorMap tm_v3, const PrefillParams p) {
   using namespace ptx;
   constexpr int HALVES = D / 64;
   constexpr uint32_t TILE = HALVES * kHalfBytes;
@@ -134,6 +138,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tensormap(&tm_q);
     prefetch_tensormap(&tm_k);
     prefetch_tensormap(&tm_v);
+    prefetch_tensormap(&tm_k3);
+    prefetch_tensormap(&tm_v3);
   }
   if (warp == 1) tmem_alloc(tmem_slot, 512);
   tc_fence_before();
@@ -157,29 +163,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; i < n_tiles; ++i) {
         const int st = i & 1;
         const uint32_t ph = (i >> 1) & 1;
-        int rows[4];
+        int rows[4], slot_first = 0;
+        bool run = true;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int j = min(i * kTileKeys + 4 * lane + e, k_len - 1);
           while (seg + 1 < seg_end && __ldg(p.tab.seg_kstart + seg + 1) <= j) ++seg;
           const int slot = __ldg(p.tab.seg_start + seg) + (j - __ldg(p.tab.seg_kstart + seg));
           rows[e] = slot * p.kv_heads + g;
+          if (e == 0) slot_first = slot;
         }
-        if (!__all_sync(0xffffffffu, mbar_wait(k_empty + st, ph ^ 1, abort_flag, kWaitLimitNs))) break;
-        if (lane == 0) mbar_expect_tx(k_full + st, TILE);
-        __syncwarp();
+        // Most tiles are 128 consecutive pool slots (segments are long): one tiled
+        // box per 64-column half.  Tiles that straddle a segment boundary or the end
+        // of the request are gathered row by row.
+        const int slot0 = __shfl_sync(0xffffffffu, slot_first, 0);
 #pragma unroll
-        for (int h = 0; h < HALVES; ++h)
-          tma_gather4(sK + st * TILE + h * kHalfBytes + lane * 512, &tm_k, k_full + st, 64 * h,
-                      rows[0], rows[1], rows[2], rows[3]);
+        for (int e = 0; e < 4; ++e) run &= rows[e] == (slot0 + 4 * lane + e) * p.kv_heads + g;
+        const bool contiguous = __all_sync(0xffffffffu, run);
+        auto load_tile = [&](uint8_t* dst, const CUtensorMap* tiled, const CUtensorMap* rowmap,
+                             uint64_t* bar) {
+          if (lane == 0) mbar_expect_tx(bar, TILE);
+          __syncwarp();
+          if (contiguous) {
+            if (lane == 0)
+              for (int h = 0; h < HALVES; ++h)
+                tma_load_3d(dst + h * kHalfBytes, tiled, bar, 64 * h, g, slot0);
+          } else {
+#pragma unroll
+            for (int h = 0; h < HALVES; ++h)
+              tma_gather4(dst + h * kHalfBytes + lane * 512, rowmap, bar, 64 * h, rows[0], rows[1],
+                          rows[2], rows[3]);
+          }
+        };
+        if (!__all_sync(0xffffffffu, mbar_wait(k_empty + st, ph ^ 1, abort_flag, kWaitLimitNs))) break;
+        load_tile(sK + st * TILE, &tm_k3, &tm_k, k_full + st);
         ++k_issued;
         if (!__all_sync(0xffffffffu, mbar_wait(v_empty + st, ph ^ 1, abort_flag, kWaitLimitNs))) break;
-        if (lane == 0) mbar_expect_tx(v_full + st, TILE);
-        __syncwarp();
-#pragma unroll
-        for (int h = 0; h < HALVES; ++h)
-          tma_gather4(sV + st * TILE + h * kHalfBytes + lane * 512, &tm_v, v_full + st, 64 * h,
-                      rows[0], rows[1], rows[2], rows[3]);
+        load_tile(sV + st * TILE, &tm_v3, &tm_v, v_full + st);
         ++v_issued;
       }
       // never leave the CTA with copies in flight
@@ -460,7 +480,7 @@ template <int D>
 int launch_prefill_d(const PrefillLaunch& a, cudaStream_t stream) {
   const seg_attn_table_desc& d = *a.desc;
   const int group = d.q_heads / d.kv_heads;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, tk3, tv3;
   {
     const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)d.q_heads, (cuuint64_t)d.total_q};
     const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)d.q_heads * D * 2};
@@ -476,6 +496,13 @@ int launch_prefill_d(const PrefillLaunch& a, cudaStream_t stream) {
     // with no keys no tile is ever loaded; the query buffer stands in as a valid address
     if (!encode(&tk, empty ? a.q : a.k_pool, 2, dims, strides, box)) return SEG_ATTN_ERR_CUDA;
     if (!encode(&tv, empty ? a.q : a.v_pool, 2, dims, strides, box)) return SEG_ATTN_ERR_CUDA;
+    // the same pools as [slots][kv heads][d]: 128 consecutive slots of one head per box
+    const cuuint64_t dims3[3] = {(cuuint64_t)D, (cuuint64_t)d.kv_heads,
+                                 empty ? 1ull : (cuuint64_t)d.num_slots};
+    const cuuint64_t strides3[2] = {(cuuint64_t)D * 2, (cuuint64_t)d.kv_heads * D * 2};
+    const cuuint32_t box3[3] = {64, 1, (cuuint32_t)kTileKeys};
+    if (!encode(&tk3, empty ? a.q : a.k_pool, 3, dims3, strides3, box3)) return SEG_ATTN_ERR_CUDA;
+    if (!encode(&tv3, empty ? a.q : a.v_pool, 3, dims3, strides3, box3)) return SEG_ATTN_ERR_CUDA;
   }
   PrefillParams p;
   p.out = static_cast<__nv_bfloat16*>(a.out);
@@ -491,7 +518,7 @@ int launch_prefill_d(const PrefillLaunch& a, cudaStream_t stream) {
   if (cudaFuncSetAttribute(prefill_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
     return SEG_ATTN_ERR_CUDA;
-  prefill_kernel<D><<<d.num_work, kThreads, smem, stream>>>(tq, tk, tv, p);
+  prefill_kernel<D><<<d.num_work, kThreads, smem, stream>>>(tq, tk, tv, tk3, tv3, p);
   return cudaGetLastError() == cudaSuccess ? SEG_ATTN_OK : SEG_ATTN_ERR_CUDA;
 }
 

@@ -54,12 +54,6 @@ namespace {
 constexpr int kThreads = 320;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
 constexpr float kRescaleLog2 = 8.0f;
-// Of every 16 pairs of scores, this many are exponentiated with the FMA-pipe
-// polynomial instead of the SFU, to balance the two pipes.
-#ifndef SEG_ATTN_EXP2_POLY_PAIRS
-#define SEG_ATTN_EXP2_POLY_PAIRS 0
-#endif
-constexpr int kPolyPairs = SEG_ATTN_EXP2_POLY_PAIRS;
 constexpr uint32_t kHalfBytes = 128 * 128;  // 128 rows x 64 bf16 (one swizzle-128B panel)
 
 struct PrefillParams {
@@ -195,10 +189,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                           rows[2], rows[3]);
           }
         };
-        if (!__all_sync(0xffffffffu, mbar_wait(k_empty + st, ph ^ 1, abort_flag, kWaitLimitNs))) break;
+        if (!__all_sync(0xffffffffu, mbar_wait(k_empty + st, ph ^ 1, abort_flag, kWaitLimitNs, true))) break;
         load_tile(sK + st * TILE, &tm_k3, &tm_k, k_full + st);
         ++k_issued;
-        if (!__all_sync(0xffffffffu, mbar_wait(v_empty + st, ph ^ 1, abort_flag, kWaitLimitNs))) break;
+        if (!__all_sync(0xffffffffu, mbar_wait(v_empty + st, ph ^ 1, abort_flag, kWaitLimitNs, true))) break;
         load_tile(sV + st * TILE, &tm_v3, &tm_v, v_full + st);
         ++v_issued;
       }
@@ -316,22 +310,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     // One tile of the online softmax (S already masked where needed).
     auto softmax_tile = [&](int i) -> bool {
       auto f = [](uint32_t bits) { return __uint_as_float(bits); };
-      // pass 1: row max (two 64-column halves, four independent chains)
+      // the whole S row in registers: one round trip to tensor memory
+      uint32_t sv[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, sv[c]);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_wait_ld(sv[c]);
       float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        uint32_t a[32], b[32];
-        tmem_ld32(tS + 64 * hh, a);
-        tmem_ld32(tS + 64 * hh + 32, b);
-        tmem_wait_ld(a);
-        tmem_wait_ld(b);
+      for (int c = 0; c < 4; ++c)
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const int k = (e >> 1) & 1;
-          mx[k] = fmaxf(mx[k], fmaxf(f(a[e]), f(a[e + 1])));
-          mx[2 + k] = fmaxf(mx[2 + k], fmaxf(f(b[e]), f(b[e + 1])));
-        }
-      }
+        for (int e = 0; e < 32; e += 2) mx[c] = fmaxf(mx[c], fmaxf(f(sv[c][e]), f(sv[c][e + 1])));
       const float row_max = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
       const float m_new = fmaxf(m_ref, row_max);
       float alpha = 1.f;
@@ -344,39 +333,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         rescale = true;
       }
       const float base = m_ref == -INFINITY ? 0.f : m_ref * sl2;
-      // pass 2: P = 2^(s*scale*log2e - base) as bf16 pairs into the first 64 S columns;
-      // chunk c+1 is loaded while chunk c is exponentiated (P chunk c only overwrites
-      // S columns that were already read).
+      // P = 2^(s*scale*log2e - base) as bf16 pairs over the first 64 S columns
       float ls[2] = {0.f, 0.f};
-      auto make_p = [&](const uint32_t (&cur)[32], int c) {  // S chunk c -> P columns [16c, 16c+16)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const float xa = fmaf(f(cur[2 * e]), sl2, -base);
-          const float xb = fmaf(f(cur[2 * e + 1]), sl2, -base);
-          const bool poly = kPolyPairs > 0 && (e % 16) * kPolyPairs / 16 != ((e % 16) + 1) * kPolyPairs / 16;
-          const float pa = poly ? exp2_poly(xa) : ex2(xa);
-          const float pb = poly ? exp2_poly(xb) : ex2(xb);
+          const float pa = ex2(fmaf(f(sv[c][2 * e]), sl2, -base));
+          const float pb = ex2(fmaf(f(sv[c][2 * e + 1]), sl2, -base));
           ls[0] += pa;
           ls[1] += pb;
           pk[e] = pack_bf16(pa, pb);
         }
         tmem_st16(tS + 16 * c, pk);
-      };
-      {
-        uint32_t a[32], b[32];
-        tmem_ld32(tS, a);
-        tmem_wait_ld(a);
-        tmem_ld32(tS + 32, b);
-        make_p(a, 0);
-        tmem_wait_ld(b);
-        tmem_ld32(tS + 64, a);
-        make_p(b, 1);
-        tmem_wait_ld(a);
-        tmem_ld32(tS + 96, b);
-        make_p(a, 2);
-        tmem_wait_ld(b);
-        make_p(b, 3);
       }
       l = l * alpha + (ls[0] + ls[1]);
       if (__any_sync(0xffffffffu, rescale)) {

@@ -64,13 +64,15 @@ __device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t bar, uint32_t par
 // Wait for the phase of `bar` with the given parity.  Gives up (returns
 // false) when *abort becomes non-zero or after limit_ns; a give-up caused by
 // the time limit sets *abort so every other role of the CTA stops too.
+// `suspend` lets the hardware park the thread between polls (for waits off the
+// critical path, such as the producer's wait for a free ring slot).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          uint64_t limit_ns) {
+                                          uint64_t limit_ns, bool suspend = false) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait_suspend(a, parity, 200000u)) return true;
+    if (suspend ? mbar_try_wait_suspend(a, parity, 200000u) : mbar_try_wait(a, parity)) return true;
     if ((it & 15) == 0) {
       if (abort && *abort) return false;
       if (globaltimer_ns() - t0 > limit_ns) {
@@ -225,21 +227,6 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16
       "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
       "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
       : "memory");
-}
-
-// 2^x on the FMA pipe, for softmax exponents x <= 8 (inputs below -126,
-// including -inf, give a value below 2^-125 instead of 0).  Cody-Waite style
-// range reduction x = n + f with n = round(x), f in [-1/2, 1/2]: adding
-// 1.5 * 2^23 rounds x to an integer in the low mantissa bits; 2^f comes from a
-// degree-3 polynomial fitted here by a Remez exchange for minimum relative
-// error on [-1/2, 1/2] (max relative error 7.5e-5, well under the bf16 rounding
-// of P); 2^n is applied by adding n to the exponent field.
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -126.0f);
-  const float t = x + 12582912.0f;
-  const float f = x - (t - 12582912.0f);
-  const float p = fmaf(fmaf(fmaf(0.0551716685f, f, 0.2426111251f), f, 0.6932609677f), f, 0.9999280572f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
 __device__ __forceinline__ float ex2(float x) {

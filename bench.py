@@ -174,7 +174,8 @@ class Path:
             lse = torch.empty(b.q.shape[0], wl.q_heads, dtype=torch.float32, device=device)
             ws = (torch.empty(tab.workspace_bytes, dtype=torch.uint8, device=device)
                   if tab.workspace_bytes else None)
-            launches = 1 + (1 if (mode == sa.MODE_DECODE and tab.workspace_bytes) else 0)
+            # second launch: decode merge, or prefill merge of split items
+            launches = 1 + (1 if tab.workspace_bytes else 0)
             self.legs.append(dict(batch=b, mode=mode, tab=tab, out=out, lse=lse, ws=ws,
                                   launches=launches))
 

@@ -70,7 +70,7 @@ typedef enum {
 enum { SEG_ATTN_MODE_PREFILL = 0, SEG_ATTN_MODE_DECODE = 1 };
 
 #define SEG_ATTN_TABLE_MAGIC 0x53454741u /* "SEGA" */
-#define SEG_ATTN_TABLE_VERSION 1u
+#define SEG_ATTN_TABLE_VERSION 2u
 
 /*
  * Description of a built segment table.  Filled by seg_attn_build_table; the
@@ -85,10 +85,13 @@ typedef struct seg_attn_table_desc {
   int64_t total_q;         /* sum of q_lens = rows of q / out */
   int64_t total_k;         /* sum of k_lens */
   int32_t num_segments;
-  int32_t num_work;        /* prefill: (request, kv head, query-tile pair) items; decode: chunks */
+  int32_t num_work;        /* prefill: (request, kv head, query-tile pair, key range) items;
+                              decode: chunks */
   int32_t queries_per_tile;/* prefill: 128 / group size */
   int32_t chunk_len;       /* decode: logical keys per split-K chunk */
   int32_t max_k_tiles;     /* prefill: largest number of 128-key tiles of one item */
+  int32_t num_merge;       /* prefill: items whose key range was split over several CTAs */
+  int32_t num_parts;       /* prefill: partial-result slots of those items */
   int32_t reserved0;
   int64_t off_q_offsets;   /* [batch+1] packed query offset of each request */
   int64_t off_k_lens;      /* [batch]   keys of each request */
@@ -96,8 +99,10 @@ typedef struct seg_attn_table_desc {
   int64_t off_seg_start;   /* [num_segments] first slot of each segment */
   int64_t off_seg_kstart;  /* [num_segments] logical index of each segment's first key */
   int64_t off_seg_len;     /* [num_segments] */
-  int64_t off_work;        /* [num_work][4] work items (16-byte aligned) */
+  int64_t off_work;        /* work items, 16-byte aligned: decode [num_work][4],
+                              prefill [num_work][8] */
   int64_t off_req_chunks;  /* decode: [batch+1] first chunk of each request */
+  int64_t off_merge;       /* prefill: [num_merge][8] split items and their partial slots */
   uint64_t table_bytes;    /* size of the table buffer */
   uint64_t workspace_bytes;/* device scratch the compute call needs (may be 0) */
 } seg_attn_table_desc;
@@ -143,7 +148,11 @@ size_t seg_attn_workspace_size(const seg_attn_table_desc* desc);
  * tcgen05 tensor cores with accumulators in tensor memory, the online softmax
  * runs in registers.  Writes out (and lse if non-NULL) for every row.
  *   softmax_scale  > 0 and finite (typically 1/sqrt(head_dim))
- *   workspace      unused for prefill (may be NULL / 0)
+ *   workspace      device memory of at least seg_attn_workspace_size(desc)
+ *                  bytes, 16-byte aligned, when that size is non-zero: the
+ *                  planner splits the key range of long items over several
+ *                  CTAs when that balances the grid, and their fp32 partials
+ *                  are merged by a second kernel (contents are scratch)
  */
 int seg_attn_prefill(const void* q, const void* k_pool, const void* v_pool, void* out, float* lse,
                      const void* dev_table, const seg_attn_table_desc* desc, float softmax_scale,

@@ -43,11 +43,13 @@ class seg_attn_table_desc(ctypes.Structure):
         ("num_slots", ctypes.c_int64), ("total_q", ctypes.c_int64), ("total_k", ctypes.c_int64),
         ("num_segments", ctypes.c_int32), ("num_work", ctypes.c_int32),
         ("queries_per_tile", ctypes.c_int32), ("chunk_len", ctypes.c_int32),
-        ("max_k_tiles", ctypes.c_int32), ("reserved0", ctypes.c_int32),
+        ("max_k_tiles", ctypes.c_int32), ("num_merge", ctypes.c_int32),
+        ("num_parts", ctypes.c_int32), ("reserved0", ctypes.c_int32),
         ("off_q_offsets", ctypes.c_int64), ("off_k_lens", ctypes.c_int64),
         ("off_seg_offsets", ctypes.c_int64), ("off_seg_start", ctypes.c_int64),
         ("off_seg_kstart", ctypes.c_int64), ("off_seg_len", ctypes.c_int64),
         ("off_work", ctypes.c_int64), ("off_req_chunks", ctypes.c_int64),
+        ("off_merge", ctypes.c_int64),
         ("table_bytes", ctypes.c_uint64), ("workspace_bytes", ctypes.c_uint64),
     ]
 

@@ -35,11 +35,12 @@ extern "C" int seg_attn_prefill(const void* q, const void* k_pool, const void* v
                                 float* lse, const void* dev_table, const seg_attn_table_desc* desc,
                                 float softmax_scale, void* workspace, size_t workspace_bytes,
                                 void* stream) {
-  (void)workspace;
-  (void)workspace_bytes;
   int rc = check_common(q, k_pool, v_pool, out, lse, dev_table, desc, softmax_scale,
                         SEG_ATTN_MODE_PREFILL);
   if (rc != SEG_ATTN_OK) return rc;
+  if (desc->workspace_bytes > 0 &&
+      (!workspace || workspace_bytes < desc->workspace_bytes || !aligned16(workspace)))
+    return SEG_ATTN_ERR_WORKSPACE;
   if (desc->num_work == 0) return SEG_ATTN_OK;
   segattn::PrefillLaunch a;
   a.q = q;
@@ -50,6 +51,12 @@ extern "C" int seg_attn_prefill(const void* q, const void* k_pool, const void* v
   a.tab = segattn::make_view(dev_table, *desc);
   a.desc = desc;
   a.scale = softmax_scale;
+  a.part_o = static_cast<float*>(workspace);
+  a.part_lse = desc->workspace_bytes > 0
+                   ? reinterpret_cast<float*>(
+                         static_cast<char*>(workspace) +
+                         segattn::prefill_part_o_bytes(desc->num_parts, desc->head_dim))
+                   : nullptr;
   return segattn::launch_prefill(a, static_cast<cudaStream_t>(stream));
 }
 

@@ -62,6 +62,8 @@ struct PrefillParams {
   TableView tab;
   float scale_log2;
   int q_heads, kv_heads, group, qpt, causal;
+  float* part_o;    // split items: [slot][kItemRows][D], O / l of the piece
+  float* part_lse;  // split items: [slot][kItemRows], log2 of the piece's sum of exp
 };
 
 // Q (2 tiles) + K ring (2) + V ring (2) + barriers + alignment slack.  The
@@ -107,8 +109,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int4 item = p.tab.work[blockIdx.x];
-  const int req = item.x, g = item.y, q0 = item.z, n_tiles = item.w;
+  // piece: keys tiles [kt0, kt1) of item (request, kv head g, query tiles from q0);
+  // slot >= 0 when the item is split and this piece writes a partial result
+  const int4 w0 = p.tab.work[2 * blockIdx.x], w1 = p.tab.work[2 * blockIdx.x + 1];
+  const int req = w0.x, g = w0.y, q0 = w0.z, kt0 = w0.w, slot = w1.y;
+  const int n_tiles = w1.x - kt0;
   const int tok0 = __ldg(p.tab.q_offsets + req);
   const int q_len = __ldg(p.tab.q_offsets + req + 1) - tok0;
   const int k_len = __ldg(p.tab.k_lens + req);
@@ -161,7 +166,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool run = true;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int j = min(i * kTileKeys + 4 * lane + e, k_len - 1);
+          const int j = min((kt0 + i) * kTileKeys + 4 * lane + e, k_len - 1);
           while (seg + 1 < seg_end && __ldg(p.tab.seg_kstart + seg + 1) <= j) ++seg;
           const int slot = __ldg(p.tab.seg_start + seg) + (j - __ldg(p.tab.seg_kstart + seg));
           rows[e] = slot * p.kv_heads + g;
@@ -294,7 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the columns this row must not see).  Only tiles where some row of the warp
     // needs it pay for it; the softmax itself never compares per element.
     auto mask_tile = [&](int i) {
-      const int kb = i * kTileKeys;
+      const int kb = (kt0 + i) * kTileKeys;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t a[32];
@@ -370,7 +375,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!(ok = __all_sync(0xffffffffu, mbar_wait(s_full + t, i & 1, abort_flag, kWaitLimitNs))))
         break;
       tc_fence_after();
-      const bool masked = __any_sync(0xffffffffu, (i + 1) * kTileKeys > vis);
+      const bool masked = __any_sync(0xffffffffu, (kt0 + i + 1) * kTileKeys > vis);
       if (masked) mask_tile(i);
       ok = softmax_tile(i);
       if (!ok) break;
@@ -381,7 +386,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok && n_tiles > 0)
       ok = __all_sync(0xffffffffu,
                       mbar_wait(o_full + t, (n_tiles - 1) & 1, abort_flag, kWaitLimitNs));
-    if (ok) {
+    if (ok && slot >= 0) {
+      // piece of a split item: O / l and log2(sum of exp) of this key range, every row
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const int64_t prow = (int64_t)slot * kItemRows + t * kTileRows + row;
+      float* po = p.part_o + prow * D;
+      if (n_tiles > 0) tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        if (n_tiles > 0) {
+          tmem_ld32(tO + 32 * c, o);
+          tmem_wait_ld(o);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = 0u;
+        }
+#pragma unroll
+        for (int e = 0; e < 32; e += 4)
+          *reinterpret_cast<float4*>(po + 32 * c + e) =
+              make_float4(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv,
+                          __uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
+      }
+      p.part_lse[prow] = l > 0.f ? m_ref * sl2 + log2f(l) : -INFINITY;
+    } else if (ok) {
       const float inv = l > 0.f ? 1.f / l : 0.f;
       __nv_bfloat16* orow = p.out + ((int64_t)(tok0 + qi) * p.q_heads + head) * D;
       if (n_tiles > 0) tc_fence_after();
@@ -420,6 +448,51 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_dealloc(tmem, 512);
   }
   if (threadIdx.x == 0 && *abort_flag) atomicOr(&g_device_error, 1);
+}
+
+// Combine the pieces of each split item: weights 2^(lse_j - max) on the pieces'
+// normalised outputs.  One warp per row, each lane D/32 consecutive columns.
+template <int D>
+__global__ void __launch_bounds__(256) prefill_merge_kernel(const PrefillParams p) {
+  constexpr int PER = D / 32;
+  const int4 m0 = p.tab.merge[2 * blockIdx.x], m1 = p.tab.merge[2 * blockIdx.x + 1];
+  const int req = m0.x, g = m0.y, q0 = m0.z, slot0 = m0.w, parts = m1.x;
+  const int tok0 = __ldg(p.tab.q_offsets + req);
+  const int q_len = __ldg(p.tab.q_offsets + req + 1) - tok0;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int row = blockIdx.y * 8 + warp; row < kItemRows; row += 8 * gridDim.y) {
+    const int t = row / kTileRows, r = row % kTileRows;
+    const int qi = q0 + t * p.qpt + r / p.group;
+    if (qi >= q_len) continue;
+    const int head = g * p.group + r % p.group;
+    float M = -INFINITY;
+    for (int j = 0; j < parts; ++j)
+      M = fmaxf(M, p.part_lse[(int64_t)(slot0 + j) * kItemRows + row]);
+    const float Mb = M == -INFINITY ? 0.f : M;
+    float acc[PER], L = 0.f;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) acc[e] = 0.f;
+    for (int j = 0; j < parts; ++j) {
+      const int64_t prow = (int64_t)(slot0 + j) * kItemRows + row;
+      const float w = ptx::ex2(p.part_lse[prow] - Mb);
+      L += w;
+      const float* po = p.part_o + prow * D + lane * PER;
+#pragma unroll
+      for (int e = 0; e < PER; e += 2) {
+        const float2 x = *reinterpret_cast<const float2*>(po + e);
+        acc[e] += w * x.x;
+        acc[e + 1] += w * x.y;
+      }
+    }
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    __nv_bfloat16* orow = p.out + ((int64_t)(tok0 + qi) * p.q_heads + head) * D + lane * PER;
+#pragma unroll
+    for (int e = 0; e < PER; e += 2)
+      *reinterpret_cast<uint32_t*>(orow + e) = pack_bf16(acc[e] * inv, acc[e + 1] * inv);
+    if (p.lse && lane == 0)
+      p.lse[(int64_t)(tok0 + qi) * p.q_heads + head] =
+          L > 0.f ? (Mb + log2f(L)) * 0.69314718055994531f : -INFINITY;
+  }
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -484,12 +557,19 @@ int launch_prefill_d(const PrefillLaunch& a, cudaStream_t stream) {
   p.group = group;
   p.qpt = d.queries_per_tile;
   p.causal = d.causal;
+  p.part_o = a.part_o;
+  p.part_lse = a.part_lse;
   constexpr size_t smem = prefill_smem_bytes<D>();
   if (cudaFuncSetAttribute(prefill_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
     return SEG_ATTN_ERR_CUDA;
   prefill_kernel<D><<<d.num_work, kThreads, smem, stream>>>(tq, tk, tv, tk3, tv3, p);
-  return cudaGetLastError() == cudaSuccess ? SEG_ATTN_OK : SEG_ATTN_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return SEG_ATTN_ERR_CUDA;
+  if (d.num_merge > 0) {
+    prefill_merge_kernel<D><<<dim3(d.num_merge, 4), 256, 0, stream>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return SEG_ATTN_ERR_CUDA;
+  }
+  return SEG_ATTN_OK;
 }
 
 }  // namespace

@@ -5,8 +5,11 @@
 // as a few contiguous slot runs.  The builder flattens the per-request lists
 // into CSR arrays, records each segment's logical start so the kernels can
 // translate logical key j -> slot in O(1) per run, and plans the work:
-//   prefill: one item per (request, kv head, pair of 128-row query tiles),
-//            longest first so the long causal items start in the first wave;
+//   prefill: one item per (request, kv head, pair of 128-row query tiles);
+//            long items are cut into pieces along their K tiles when that
+//            shortens the longest-first schedule on the 148 SMs (the pieces'
+//            partial results are merged by a second kernel), then the pieces
+//            are ordered longest first;
 //   decode:  split-K chunks of logical keys (per-block partial attention with
 //            a per-request reduction, FlashAccel article, "data layout
 //            optimisation"), sized so the grid covers the 148 SMs many times.
@@ -14,8 +17,11 @@
 #include <string.h>
 
 #include <algorithm>
+#include <array>
+#include <functional>
 #include <limits>
 #include <numeric>
+#include <queue>
 #include <vector>
 
 #include "seg_attn.h"
@@ -104,25 +110,81 @@ extern "C" int seg_attn_build_table(int batch, const int32_t* q_lens, const int3
   if (total_q > kI32Max) return SEG_ATTN_ERR_UNSUPPORTED;
 
   // ---- work plan
-  std::vector<int4> work;
+  std::vector<int4> work;                      // decode chunks
+  std::vector<std::array<int32_t, 8>> pwork;   // prefill pieces
+  std::vector<std::array<int32_t, 8>> pmerge;  // prefill items split over several pieces
   std::vector<int32_t> req_chunks;
-  int32_t queries_per_tile = 0, chunk_len = 0, max_k_tiles = 0;
+  int32_t queries_per_tile = 0, chunk_len = 0, max_k_tiles = 0, part_slots = 0;
   if (mode == SEG_ATTN_MODE_PREFILL) {
     queries_per_tile = segattn::kTileRows / group;
     const int32_t span = queries_per_tile * segattn::kTilesPerItem;
+    struct Item { int32_t r, g, q0, tiles; };
+    std::vector<Item> items;
     for (int r = 0; r < batch; ++r) {
       const int64_t prior = (int64_t)kl[r] - ql[r];
       for (int32_t q0 = 0; q0 < ql[r]; q0 += span) {
         const int64_t q_end = std::min<int64_t>(ql[r], (int64_t)q0 + span);
         const int64_t visible = causal ? std::min<int64_t>(kl[r], prior + q_end) : kl[r];
         const int32_t tiles = (int32_t)((visible + segattn::kTileKeys - 1) / segattn::kTileKeys);
-        for (int g = 0; g < kv_heads; ++g) work.push_back(make_int4(r, g, q0, tiles));
+        for (int g = 0; g < kv_heads; ++g) items.push_back({r, g, q0, tiles});
         max_k_tiles = std::max(max_k_tiles, tiles);
       }
     }
-    // longest first; stable keeps (request, query tile, head) order among equals
-    std::stable_sort(work.begin(), work.end(),
-                     [](const int4& a, const int4& b) { return a.w > b.w; });
+    // Each CTA runs one piece (a contiguous range of an item's K tiles).  Pick how
+    // far to split long items by simulating the longest-first assignment of pieces
+    // to the SMs (what the block scheduler does with a grid in that order) and
+    // keeping the factor with the shortest makespan; ties keep fewer splits.
+    auto pieces_of = [](int32_t tiles, int f) {
+      if (f <= 1 || tiles < 2 * segattn::kMinPieceTiles) return 1;
+      return std::min(f, tiles / segattn::kMinPieceTiles);
+    };
+    auto makespan = [&](int f) {
+      std::vector<int64_t> cost;
+      for (const Item& it : items) {
+        const int p = pieces_of(it.tiles, f);
+        for (int j = 0; j < p; ++j)
+          cost.push_back((int64_t)it.tiles * (j + 1) / p - (int64_t)it.tiles * j / p +
+                         segattn::kPieceOverheadTiles);
+      }
+      std::sort(cost.begin(), cost.end(), std::greater<int64_t>());
+      std::priority_queue<int64_t, std::vector<int64_t>, std::greater<int64_t>> sm;
+      for (int i = 0; i < segattn::kSmCount; ++i) sm.push(0);
+      int64_t span_max = 0;
+      for (int64_t c : cost) {
+        const int64_t t = sm.top() + c;
+        sm.pop();
+        sm.push(t);
+        span_max = std::max(span_max, t);
+      }
+      return span_max;
+    };
+    int best_f = 1;
+    int64_t best = makespan(1);
+    for (int f = 2; f <= segattn::kMaxSplit; ++f) {
+      const int64_t m = makespan(f);
+      if (m * 100 < best * 98) {
+        best = m;
+        best_f = f;
+      }
+    }
+    for (const Item& it : items) {
+      const int p = pieces_of(it.tiles, best_f);
+      const int32_t slot0 = p > 1 ? part_slots : -1;
+      if (p > 1) {
+        pmerge.push_back({it.r, it.g, it.q0, slot0, p, 0, 0, 0});
+        part_slots += p;
+      }
+      for (int j = 0; j < p; ++j) {
+        const int32_t kt0 = (int32_t)((int64_t)it.tiles * j / p);
+        const int32_t kt1 = (int32_t)((int64_t)it.tiles * (j + 1) / p);
+        pwork.push_back({it.r, it.g, it.q0, kt0, kt1, p > 1 ? slot0 + j : -1, 0, 0});
+      }
+    }
+    // longest first; stable keeps (request, query tile, head, piece) order among equals
+    std::stable_sort(pwork.begin(), pwork.end(),
+                     [](const std::array<int32_t, 8>& a, const std::array<int32_t, 8>& b) {
+                       return a[4] - a[3] > b[4] - b[3];
+                     });
   } else {
     int64_t L = 2048;
     auto ctas = [&](int64_t len) {
@@ -144,7 +206,8 @@ extern "C" int seg_attn_build_table(int batch, const int32_t* q_lens, const int3
       req_chunks[r + 1] = req_chunks[r] + n;
     }
   }
-  if (work.size() > (size_t)kI32Max) return SEG_ATTN_ERR_UNSUPPORTED;
+  const size_t n_work = mode == SEG_ATTN_MODE_PREFILL ? pwork.size() : work.size();
+  if (n_work > (size_t)kI32Max) return SEG_ATTN_ERR_UNSUPPORTED;
 
   // ---- layout
   Layout lay;
@@ -154,8 +217,9 @@ extern "C" int seg_attn_build_table(int batch, const int32_t* q_lens, const int3
   desc->off_seg_start = lay.take(nseg);
   desc->off_seg_kstart = lay.take(nseg);
   desc->off_seg_len = lay.take(nseg);
-  desc->off_work = lay.take(4 * (int64_t)work.size());
+  desc->off_work = lay.take((mode == SEG_ATTN_MODE_PREFILL ? 8 : 4) * (int64_t)n_work);
   desc->off_req_chunks = lay.take(mode == SEG_ATTN_MODE_DECODE ? batch + 1 : 0);
+  desc->off_merge = lay.take(8 * (int64_t)pmerge.size());
 
   desc->magic = SEG_ATTN_TABLE_MAGIC;
   desc->version = SEG_ATTN_TABLE_VERSION;
@@ -169,12 +233,17 @@ extern "C" int seg_attn_build_table(int batch, const int32_t* q_lens, const int3
   desc->total_q = total_q;
   desc->total_k = total_k;
   desc->num_segments = (int32_t)nseg;
-  desc->num_work = (int32_t)work.size();
+  desc->num_work = (int32_t)n_work;
+  desc->num_merge = (int32_t)pmerge.size();
+  desc->num_parts = part_slots;
   desc->queries_per_tile = queries_per_tile;
   desc->chunk_len = chunk_len;
   desc->max_k_tiles = max_k_tiles;
   desc->table_bytes = (uint64_t)lay.n * sizeof(int32_t);
   desc->workspace_bytes = 0;
+  if (mode == SEG_ATTN_MODE_PREFILL && part_slots > 0)
+    desc->workspace_bytes = segattn::prefill_part_o_bytes(part_slots, head_dim) +
+                            align_up((size_t)part_slots * segattn::kItemRows * sizeof(float), 256);
   if (mode == SEG_ATTN_MODE_DECODE) {
     bool multi = false;
     for (int r = 0; r < batch; ++r) multi |= (req_chunks[r + 1] - req_chunks[r]) > 1;
@@ -211,7 +280,14 @@ extern "C" int seg_attn_build_table(int batch, const int32_t* q_lens, const int3
     }
     s0 += seg_counts[r];
   }
-  if (!work.empty()) memcpy(t + desc->off_work, work.data(), work.size() * sizeof(int4));
+  if (mode == SEG_ATTN_MODE_PREFILL) {
+    for (size_t i = 0; i < pwork.size(); ++i)
+      memcpy(t + desc->off_work + 8 * i, pwork[i].data(), 8 * sizeof(int32_t));
+    for (size_t i = 0; i < pmerge.size(); ++i)
+      memcpy(t + desc->off_merge + 8 * i, pmerge[i].data(), 8 * sizeof(int32_t));
+  } else if (!work.empty()) {
+    memcpy(t + desc->off_work, work.data(), work.size() * sizeof(int4));
+  }
   if (mode == SEG_ATTN_MODE_DECODE)
     memcpy(t + desc->off_req_chunks, req_chunks.data(), req_chunks.size() * sizeof(int32_t));
   return SEG_ATTN_OK;

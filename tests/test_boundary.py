@@ -113,12 +113,11 @@ def test_prefill_table_contents():
     assert view(tab, d.off_seg_kstart, 5) == [0, 2, 0, 0, 20]
     assert view(tab, d.off_seg_len, 5) == [2, 5, 3, 20, 30]
     assert d.off_work % 4 == 0 and d.queries_per_tile == 32  # 128 rows / group 4
-    work = np.array(view(tab, d.off_work, 4 * d.num_work)).reshape(-1, 4)
+    work = np.array(view(tab, d.off_work, 8 * d.num_work)).reshape(-1, 8)
     # request 0: one pair x 2 kv heads; request 2: 40 queries -> 1 pair (64 per pair) x 2 heads
     assert len(work) == 4 and sorted(set(work[:, 0])) == [0, 2]
-    assert list(work[:, 3]) == sorted(work[:, 3], reverse=True)  # longest first
-    # causal tile count: last query of request 2 sees all 50 keys -> 1 tile of 128
-    assert all(w[3] == 1 for w in work)
+    # causal tile count: last query of request 2 sees all 50 keys -> tiles [0, 1), unsplit
+    assert all(w[3] == 0 and w[4] == 1 and w[5] == -1 for w in work)
 
 
 def test_decode_chunks_cover_each_request():
@@ -170,3 +169,37 @@ def test_empty_batch_is_a_noop():
     rc = lib.seg_attn_prefill(None, None, None, None, None, None, ctypes.byref(tab.desc), 0.1,
                               None, 0, None)
     assert rc == 0
+
+
+def test_prefill_split_plan_covers_every_item_once():
+    # one long request, few query tiles: the planner cuts items along their keys
+    tab = build([64], [[(0, 20000)]], num_slots=20000, hq=16, hkv=2)
+    d = tab.desc
+    assert d.num_merge > 0 and d.num_parts > d.num_merge and d.workspace_bytes > 0
+    work = np.array(view(tab, d.off_work, 8 * d.num_work)).reshape(-1, 8)
+    merge = np.array(view(tab, d.off_merge, 8 * d.num_merge)).reshape(-1, 8)
+    seen_slots = set()
+    for r, g, q0, slot0, parts, *_ in merge:
+        visible = min(20000, 20000 - 64 + min(64, q0 + 32))  # 16 queries per tile, 2 tiles
+        tiles = (visible + 127) // 128
+        pieces = work[(work[:, 0] == r) & (work[:, 1] == g) & (work[:, 2] == q0)]
+        assert len(pieces) == parts
+        pieces = pieces[np.argsort(pieces[:, 3])]
+        assert pieces[0, 3] == 0 and pieces[-1, 4] == tiles
+        assert (pieces[1:, 3] == pieces[:-1, 4]).all()
+        assert sorted(pieces[:, 5]) == list(range(slot0, slot0 + parts))
+        seen_slots |= set(pieces[:, 5].tolist())
+    assert seen_slots == set(range(d.num_parts))
+    # longest pieces first
+    lens = work[:, 4] - work[:, 3]
+    assert list(lens) == sorted(lens, reverse=True)
+    rows = 256
+    assert d.workspace_bytes >= d.num_parts * rows * (d.head_dim + 1) * 4
+
+
+def test_prefill_without_split_needs_no_workspace():
+    tab = build([40, 3], [[(20, 20), (60, 30)], [(0, 7)]], num_slots=100, hq=8, hkv=2)
+    d = tab.desc
+    assert d.num_merge == 0 and d.num_parts == 0 and d.workspace_bytes == 0
+    work = np.array(view(tab, d.off_work, 8 * d.num_work)).reshape(-1, 8)
+    assert (work[:, 5] == -1).all() and (work[:, 3] == 0).all()

@@ -96,6 +96,30 @@ def test_prefill_zero_keys_noncausal_and_zero_queries():
     compare(out, lse, ref_o, ref_l, "zero keys")
 
 
+@pytest.mark.parametrize("causal", [True, False])
+def test_prefill_split_items_merge(causal):
+    # few query tiles over a long context: the planner splits items along their keys,
+    # the pieces' partials are merged by the second kernel
+    g = torch.Generator().manual_seed(31)
+    k_len, q_len, hq, hkv, d = 20000, 64, 16, 2, 128
+    seg_lens = synth.split_uniform_cuts(k_len, 5, g)
+    S = k_len + 300
+    starts = synth.place_segments(seg_lens, S, g)
+    k = torch.full((S, hkv, d), float("nan")).to(torch.bfloat16)
+    v = k.clone()
+    for s0, l in zip(starts, seg_lens):
+        k[s0:s0 + l] = torch.randn(l, hkv, d, generator=g).to(torch.bfloat16)
+        v[s0:s0 + l] = torch.randn(l, hkv, d, generator=g).to(torch.bfloat16)
+    case = dict(q=torch.randn(q_len, hq, d, generator=g).to(torch.bfloat16), k_pool=k, v_pool=v,
+                q_lens=[q_len], seg_starts=[starts], seg_lens=[seg_lens], num_slots=S,
+                scale=d ** -0.5, causal=causal)
+    out, lse, tab = _run(case)
+    assert tab.desc.num_merge > 0
+    ref_o, ref_l = oracle.attention(case["q_lens"], case["seg_starts"], case["seg_lens"],
+                                    case["q"], k, v, case["scale"], causal)
+    compare(out, lse, ref_o, ref_l, "split items")
+
+
 def test_prefill_large_scores_trigger_rescale():
     # scaled-up queries make the running max jump by more than 2^8 across tiles
     case = random_case(24, batch=2, hq=8, hkv=1, d=128, causal=True, max_k=800, q_mode="full")

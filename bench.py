@@ -149,6 +149,25 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def rank_seed(config, rank):
+    """Weak scaling: every rank draws its own batch of the same shape."""
+    return config - 1 + 1000 * rank
+
+
+def max_over_ranks(value, dist=None, device="cpu"):
+    """Max of a per-rank timing over all ranks (the job ends with the slowest rank)."""
+    if dist is None:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, units_per_rank_step, ms_total, steps):
+    """Whole-job rate: units processed by all ranks / the slowest rank's time."""
+    return world * units_per_rank_step / (ms_total * 1e-3 / steps)
+
+
 def cpu_cores():
     try:
         return len(os.sched_getaffinity(0))
@@ -293,7 +312,7 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=device)
     # weak scaling: every rank runs its own batch of the same shape (seed offset by rank)
-    wl = synth.make_workload(args.config, device=str(device), seed=args.config - 1 + 1000 * rank,
+    wl = synth.make_workload(args.config, device=str(device), seed=rank_seed(args.config, rank),
                              context_scale=args.context_scale)
     path = Path(wl, device)
     stream = torch.cuda.current_stream(device)
@@ -331,10 +350,7 @@ def run_ours(args):
     ms = start.elapsed_time(end)
     leg_ms = [sum(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(args.steps)) / args.steps
               for i in range(len(path.legs))]
-    if dist:
-        t = torch.tensor([ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, dist, device)
     assert sa.seg_attn_take_device_error() == 0
 
     peaks, peak_kind = load_peaks()
@@ -362,7 +378,7 @@ def run_ours(args):
             cand = ("hbm", lm, by)
         if dominant is None or cand[1] > dominant[1]:
             dominant = cand
-    value = world * flops_step / (ms * 1e-3 / args.steps) / 1e12
+    value = job_throughput(world, flops_step, ms, args.steps) / 1e12
 
     if dominant[0] == "tensor":
         achieved = dominant[2] / (dominant[1] * 1e-3) / 1e12

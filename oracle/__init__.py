@@ -21,24 +21,27 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "seg_attn_oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
 _lock = threading.Lock()
-_lib = None
+_libs = {}
 
 
-def build(force: bool = False) -> str:
-    """Compile the oracle into ``oracle/liboracle.so`` (gcc, OpenMP, IEEE double)."""
-    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
-        tmp = _LIB + f".tmp{os.getpid()}"
+def build(force: bool = False, mutant: int = 0) -> str:
+    """Compile the oracle into ``oracle/liboracle.so`` (gcc, OpenMP, IEEE double).
+
+    ``mutant`` > 0 builds a copy with one planted mistake (see the C source),
+    used only by the tests that check the pins catch such mistakes."""
+    path = _LIB if mutant == 0 else os.path.join(_HERE, f"liboracle_mut{mutant}.so")
+    if force or not os.path.exists(path) or os.path.getmtime(path) < os.path.getmtime(_SRC):
+        tmp = path + f".tmp{os.getpid()}"
         subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
-                               "-o", tmp, _SRC, "-lm"])
-        os.replace(tmp, _LIB)
-    return _LIB
+                               f"-DORACLE_MUTANT={mutant}", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, path)
+    return path
 
 
-def _load():
-    global _lib
+def _load(mutant: int = 0):
     with _lock:
-        if _lib is None:
-            lib = ctypes.CDLL(build())
+        if mutant not in _libs:
+            lib = ctypes.CDLL(build(mutant=mutant))
             P = ctypes.c_void_p
             lib.oracle_rows.argtypes = [ctypes.c_int, P, P, P, P, P, P, P, ctypes.c_int,
                                         ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int,
@@ -48,8 +51,8 @@ def _load():
                                              ctypes.c_int, ctypes.c_int, ctypes.c_double,
                                              ctypes.c_int, P, P]
             lib.oracle_attention.restype = ctypes.c_int
-            _lib = lib
-    return _lib
+            _libs[mutant] = lib
+    return _libs[mutant]
 
 
 def _i32(x):
@@ -65,7 +68,8 @@ def _ptr(a: np.ndarray):
     return a.ctypes.data_as(ctypes.c_void_p) if a.size else ctypes.c_void_p(0)
 
 
-def attention(q_lens, seg_starts, seg_lens, q, k_pool, v_pool, scale, causal, rows=None):
+def attention(q_lens, seg_starts, seg_lens, q, k_pool, v_pool, scale, causal, rows=None,
+              mutant=0):
     """Oracle outputs for one batch.
 
     ``seg_starts`` / ``seg_lens`` are per-request lists (logical order).
@@ -74,7 +78,7 @@ def attention(q_lens, seg_starts, seg_lens, q, k_pool, v_pool, scale, causal, ro
     only those rows are computed and out is [n, d], lse [n].
     Otherwise out is [sum q_lens, Hq, d] and lse [sum q_lens, Hq].  float64.
     """
-    lib = _load()
+    lib = _load(mutant)
     counts = _i32([len(s) for s in seg_starts])
     starts = _i32([x for s in seg_starts for x in s])
     lens = _i32([x for s in seg_lens for x in s])

@@ -24,7 +24,17 @@
  *
  * Inputs are bf16 bit patterns widened exactly to double.  Parity: pinned by
  * the CPU tests (brute force on a contiguous copy, closed forms, invariances).
+ *
+ * ORACLE_MUTANT (compile-time, default 0) plants one deliberate mistake so the
+ * tests can show that the pins catch it; the shipped oracle is built with 0.
+ *   1 score without the scale        2 top-left causal alignment
+ *   3 kv head h % Hkv instead of h / G   4 segments walked in slot order
+ *   5 lse without the max            6 output not divided by l
+ *   7 V replaced by K in the weighted sum
  */
+#ifndef ORACLE_MUTANT
+#define ORACLE_MUTANT 0
+#endif
 #include <math.h>
 #include <stdint.h>
 #include <stdlib.h>
@@ -43,8 +53,20 @@ static int64_t *request_slots(int count, const int32_t *starts, const int32_t *l
     for (int s = 0; s < count; ++s) k_len += lens[s];
     int64_t *slots = (int64_t *)malloc(sizeof(int64_t) * (size_t)(k_len > 0 ? k_len : 1));
     int64_t j = 0;
+#if ORACLE_MUTANT == 4
+    /* planted mistake: segments taken in slot order instead of list order */
+    int *order = (int *)malloc(sizeof(int) * (size_t)(count > 0 ? count : 1));
+    for (int s = 0; s < count; ++s) order[s] = s;
+    for (int a = 0; a < count; ++a)
+        for (int b = a + 1; b < count; ++b)
+            if (starts[order[b]] < starts[order[a]]) { int tmp = order[a]; order[a] = order[b]; order[b] = tmp; }
+    for (int s = 0; s < count; ++s)
+        for (int32_t t = 0; t < lens[order[s]]; ++t) slots[j++] = (int64_t)starts[order[s]] + t;
+    free(order);
+#else
     for (int s = 0; s < count; ++s)
         for (int32_t t = 0; t < lens[s]; ++t) slots[j++] = (int64_t)starts[s] + t;
+#endif
     *k_len_out = k_len;
     return slots;
 }
@@ -64,19 +86,33 @@ static void one_row(const uint16_t *qrow, const uint16_t *k_pool, const uint16_t
         const uint16_t *krow = k_pool + ((size_t)slots[j] * kv_heads + g) * d;
         double acc = 0.0;
         for (int t = 0; t < d; ++t) acc += bf16_to_double(qrow[t]) * bf16_to_double(krow[t]);
+#if ORACLE_MUTANT == 1
+        s_buf[j] = acc;
+#else
         s_buf[j] = scale * acc;
+#endif
         if (s_buf[j] > m) m = s_buf[j];
     }
     double l = 0.0;
     for (int t = 0; t < d; ++t) out[t] = 0.0;
     for (int64_t j = 0; j < n; ++j) {
         const double p = exp(s_buf[j] - m);
+#if ORACLE_MUTANT == 7
+        const uint16_t *vrow = k_pool + ((size_t)slots[j] * kv_heads + g) * d;
+#else
         const uint16_t *vrow = v_pool + ((size_t)slots[j] * kv_heads + g) * d;
+#endif
         l += p;
         for (int t = 0; t < d; ++t) out[t] += p * bf16_to_double(vrow[t]);
     }
+#if ORACLE_MUTANT != 6
     for (int t = 0; t < d; ++t) out[t] /= l;
+#endif
+#if ORACLE_MUTANT == 5
+    *lse = log(l);
+#else
     *lse = m + log(l);
+#endif
 }
 
 /*
@@ -126,11 +162,19 @@ int oracle_rows(int batch, const int32_t *q_lens, const int32_t *seg_counts,
                 int r = 0; /* request owning this token */
                 while (q_off[r + 1] <= tok) ++r;
                 const int64_t qi = tok - q_off[r];
+#if ORACLE_MUTANT == 2
+                const int64_t visible = causal ? qi + 1 : k_lens[r];
+#else
                 const int64_t visible =
                     causal ? (k_lens[r] - q_lens[r]) + qi + 1 : k_lens[r];
+#endif
                 const int h = row_head[i];
                 one_row(q + ((size_t)tok * q_heads + h) * head_dim, k_pool, v_pool, slots[r],
+#if ORACLE_MUTANT == 3
+                        k_lens[r], visible, h % kv_heads, kv_heads, head_dim, scale,
+#else
                         k_lens[r], visible, h / group, kv_heads, head_dim, scale,
+#endif
                         out + (size_t)i * head_dim, lse + i, s_buf);
             }
             free(s_buf);

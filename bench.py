@@ -493,6 +493,41 @@ def run_cpu_baseline(path, args):
     return base, worst
 
 
+def run_kv_append(args):
+    """Bandwidth of seg_attn_kv_append: 262144 new tokens (64/8 heads, d 128) scattered to
+    slots handed out by the segment allocator for 256 sequences; prints its own JSON line."""
+    device = torch.device("cuda", 0)
+    hkv, d, n_seq, per_seq = 8, 128, 256, 1024
+    S = int(1.1 * n_seq * per_seq)
+    pool = sa.SegPool(S)
+    g = torch.Generator(device=device).manual_seed(0)
+    slots = torch.cat([torch.from_numpy(pool.append(s, per_seq)) for s in range(n_seq)]).to(device)
+    n = slots.numel()
+    k_pool = torch.empty(S, hkv, d, dtype=torch.bfloat16, device=device)
+    v_pool = torch.empty_like(k_pool)
+    k_new = torch.randn(n, hkv, d, generator=g, device=device).to(torch.bfloat16)
+    v_new = torch.randn(n, hkv, d, generator=g, device=device).to(torch.bfloat16)
+    for _ in range(args.warmup):
+        sa.seg_attn_kv_append(k_new, v_new, slots, k_pool, v_pool)
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(args.steps):
+        sa.seg_attn_kv_append(k_new, v_new, slots, k_pool, v_pool)
+    e.record()
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / args.steps
+    by = 2 * 2 * n * hkv * d * 2 + 4 * n  # K and V read + written, plus the slot array
+    peaks, kind = load_peaks()
+    ok = torch.equal(k_pool[slots.long()].view(torch.int16), k_new.view(torch.int16))
+    print(json.dumps({"metric": "kv append HBM GB/s", "value": by / (ms * 1e-3) / 1e9,
+                      "unit": "GB/s", "ms_per_step": ms, "steps": args.steps,
+                      "frac_hbm": by / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], "bytes": by,
+                      "tokens": n, "bit_exact": bool(ok),
+                      "device_error": sa.seg_attn_take_device_error()}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -505,6 +540,8 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=256,
                     help="oracle rows per batch for the cpu_baseline leg of our arm")
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--kv-append", action="store_true",
+                    help="measure the KV-append kernel instead of the attention step")
     ap.add_argument("--context-scale", type=float, default=1.0,
                     help="shorten the long-context mix (profiling captures only; 1.0 = as specified)")
     ap.add_argument("--no-e2e", action="store_true")
@@ -512,6 +549,8 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("note: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.kv_append:
+        return run_kv_append(args)
     return run_reference(args) if args.impl == "reference" else run_ours(args)
 
 

@@ -64,7 +64,8 @@ typedef enum {
   SEG_ATTN_ERR_WORKSPACE = -5,         /* workspace missing or smaller than needed */
   SEG_ATTN_ERR_UNSUPPORTED = -6,       /* valid but outside the supported shapes */
   SEG_ATTN_ERR_CUDA = -7,              /* a CUDA runtime / driver call failed */
-  SEG_ATTN_ERR_BUFFER_TOO_SMALL = -8   /* host_out smaller than desc->table_bytes */
+  SEG_ATTN_ERR_BUFFER_TOO_SMALL = -8,  /* output buffer smaller than needed */
+  SEG_ATTN_ERR_NO_SPACE = -9           /* the slot pool has too few free slots */
 } seg_attn_status;
 
 enum { SEG_ATTN_MODE_PREFILL = 0, SEG_ATTN_MODE_DECODE = 1 };
@@ -175,8 +176,8 @@ int seg_attn_decode(const void* q, const void* k_pool, const void* v_pool, void*
  * seg_attn_take_device_error -- read and clear the library's device error
  * word.  Kernels never trap; every wait on an mbarrier gives up after one
  * second, and a CTA that gave up drains its copies, frees its tensor memory,
- * returns, and sets this word to a non-zero value (its output rows are then
- * undefined).  Synchronous: copies from the device (implicitly synchronises
+ * returns, and sets bit 0 of this word (its output rows are then undefined);
+ * seg_attn_kv_append sets bit 1 for a slot out of range.  Synchronous: copies from the device (implicitly synchronises
  * the current device).  *value = 0 means no kernel gave up since the last call.
  */
 int seg_attn_take_device_error(int* value);
@@ -204,6 +205,66 @@ int seg_attn_take_device_error(int* value);
 int seg_attn_decode_noalloc(const void* q, const void* k_pool, const void* v_pool, void* out,
                             float* lse, const void* dev_table, const seg_attn_table_desc* desc,
                             float softmax_scale, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Segment allocator (host) and KV append (device).
+ *
+ * The cache manager behind the tables: each sequence (request) owns a short
+ * list of contiguous slot runs of the pool, as in Flood's segmentable KV cache
+ * (Flood README, "Introduction": segmentable blocks instead of paged blocks,
+ * for contiguity).  Appending n tokens to a sequence first grows its last run
+ * in place when the slots right after it are free; the rest goes to the
+ * smallest free run that holds all of it (ties: lowest start), or, when no
+ * free run is large enough, to the largest free runs in turn (ties: highest
+ * start) -- so a sequence keeps as few segments as possible.  Releasing a
+ * sequence returns its runs to the free list, merged with free neighbours.
+ * The pool object is host memory only; it is not thread-safe.
+ * ---------------------------------------------------------------------- */
+typedef struct seg_attn_pool seg_attn_pool;
+
+typedef struct seg_attn_pool_stats {
+  int64_t num_slots, free_slots;
+  int64_t free_runs, largest_free_run;
+  int64_t sequences, segments;
+} seg_attn_pool_stats;
+
+/* New pool of num_slots slots (0 <= num_slots <= INT32_MAX), all free. */
+int seg_attn_pool_create(int64_t num_slots, seg_attn_pool** out);
+int seg_attn_pool_destroy(seg_attn_pool* pool);
+
+/*
+ * Append n_tokens slots to sequence `seq` (created on first use).  On success
+ * new_slots[i] (if non-NULL, [n_tokens]) is the slot of the i-th new token,
+ * in logical order.  SEG_ATTN_ERR_NO_SPACE (pool unchanged) when fewer than
+ * n_tokens slots are free.
+ */
+int seg_attn_pool_append(seg_attn_pool* pool, int64_t seq, int64_t n_tokens, int32_t* new_slots);
+
+/* Return every slot of `seq` to the pool and forget the sequence. */
+int seg_attn_pool_release(seg_attn_pool* pool, int64_t seq);
+
+/*
+ * Segment list of `seq` in logical order -- the (start, length) input of
+ * seg_attn_build_table.  *count is always set; SEG_ATTN_ERR_BUFFER_TOO_SMALL
+ * when it exceeds capacity.
+ */
+int seg_attn_pool_segments(const seg_attn_pool* pool, int64_t seq, int32_t* starts, int32_t* lens,
+                           int capacity, int* count);
+
+int seg_attn_pool_get_stats(const seg_attn_pool* pool, seg_attn_pool_stats* out);
+
+/*
+ * seg_attn_kv_append -- write the K/V rows of new tokens into their pool slots.
+ *   k_new, v_new   bf16 [n_tokens, kv_heads, head_dim] (device, 16-byte aligned)
+ *   slots          int32 [n_tokens] device array, slot of each token
+ *   k_pool, v_pool bf16 [num_slots, kv_heads, head_dim] (device)
+ * A slot outside [0, num_slots) is skipped and recorded in the device error
+ * word (bit 2, see seg_attn_take_device_error); nothing is written out of
+ * bounds.  kv_heads * head_dim * 2 must be a multiple of 16 bytes.
+ */
+int seg_attn_kv_append(const void* k_new, const void* v_new, const int32_t* slots,
+                       int64_t n_tokens, int kv_heads, int head_dim, void* k_pool, void* v_pool,
+                       int64_t num_slots, void* stream);
 
 /* Static English description of a status code (never NULL). */
 const char* seg_attn_status_string(int status);

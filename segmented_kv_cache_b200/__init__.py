@@ -22,14 +22,14 @@ __all__ = [
     "SegAttnError", "seg_attn_table_desc", "seg_attn_build_table", "seg_attn_workspace_size",
     "seg_attn_prefill", "seg_attn_decode", "seg_attn_status_string", "seg_attn_version",
     "seg_attn_take_device_error", "SegTable", "load_library", "LIB_PATH",
-    "MODE_PREFILL", "MODE_DECODE", "STATUS",
+    "MODE_PREFILL", "MODE_DECODE", "STATUS", "SegPool", "seg_attn_kv_append",
 ]
 
 MODE_PREFILL = 0
 MODE_DECODE = 1
 STATUS = {
     "OK": 0, "INVALID_ARG": -1, "SEGMENT_OOB": -2, "SEGMENT_OVERLAP": -3, "QLEN_GT_KLEN": -4,
-    "WORKSPACE": -5, "UNSUPPORTED": -6, "CUDA": -7, "BUFFER_TOO_SMALL": -8,
+    "WORKSPACE": -5, "UNSUPPORTED": -6, "CUDA": -7, "BUFFER_TOO_SMALL": -8, "NO_SPACE": -9,
 }
 
 
@@ -52,6 +52,13 @@ class seg_attn_table_desc(ctypes.Structure):
         ("off_merge", ctypes.c_int64),
         ("table_bytes", ctypes.c_uint64), ("workspace_bytes", ctypes.c_uint64),
     ]
+
+
+class seg_attn_pool_stats(ctypes.Structure):
+    """Mirror of ``seg_attn_pool_stats`` in include/seg_attn.h."""
+    _fields_ = [("num_slots", ctypes.c_int64), ("free_slots", ctypes.c_int64),
+                ("free_runs", ctypes.c_int64), ("largest_free_run", ctypes.c_int64),
+                ("sequences", ctypes.c_int64), ("segments", ctypes.c_int64)]
 
 
 class SegAttnError(RuntimeError):
@@ -90,6 +97,19 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         lib.seg_attn_version.restype = I
         lib.seg_attn_take_device_error.argtypes = [ctypes.POINTER(ctypes.c_int)]
         lib.seg_attn_take_device_error.restype = I
+        PP = ctypes.POINTER(ctypes.c_void_p)
+        lib.seg_attn_pool_create.argtypes = [I64, PP]
+        lib.seg_attn_pool_destroy.argtypes = [P]
+        lib.seg_attn_pool_append.argtypes = [P, I64, I64, P]
+        lib.seg_attn_pool_release.argtypes = [P, I64]
+        lib.seg_attn_pool_segments.argtypes = [P, I64, P, P, I, ctypes.POINTER(I)]
+        lib.seg_attn_pool_get_stats.argtypes = [P, ctypes.POINTER(seg_attn_pool_stats)]
+        for fn in (lib.seg_attn_pool_create, lib.seg_attn_pool_destroy, lib.seg_attn_pool_append,
+                   lib.seg_attn_pool_release, lib.seg_attn_pool_segments,
+                   lib.seg_attn_pool_get_stats):
+            fn.restype = I
+        lib.seg_attn_kv_append.argtypes = [P, P, P, I64, I, I, P, P, I64, P]
+        lib.seg_attn_kv_append.restype = I
         _lib = lib
         return lib
 
@@ -205,3 +225,70 @@ class SegTable:
     @property
     def workspace_bytes(self) -> int:
         return seg_attn_workspace_size(self.desc)
+
+
+class SegPool:
+    """Host segment allocator of a slot pool (wraps the seg_attn_pool_* calls)."""
+
+    def __init__(self, num_slots: int):
+        self._lib = load_library()
+        self._h = ctypes.c_void_p()
+        rc = self._lib.seg_attn_pool_create(int(num_slots), ctypes.byref(self._h))
+        if rc != 0:
+            raise SegAttnError("seg_attn_pool_create", rc)
+
+    def close(self):
+        if self._h:
+            self._lib.seg_attn_pool_destroy(self._h)
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def append(self, seq: int, n_tokens: int) -> np.ndarray:
+        """Slots (int32, logical order) of n_tokens new tokens of sequence ``seq``."""
+        out = np.zeros(max(1, int(n_tokens)), dtype=np.int32)
+        rc = self._lib.seg_attn_pool_append(self._h, int(seq), int(n_tokens),
+                                            ctypes.c_void_p(out.ctypes.data))
+        if rc != 0:
+            raise SegAttnError("seg_attn_pool_append", rc)
+        return out[:n_tokens]
+
+    def release(self, seq: int) -> None:
+        rc = self._lib.seg_attn_pool_release(self._h, int(seq))
+        if rc != 0:
+            raise SegAttnError("seg_attn_pool_release", rc)
+
+    def segments(self, seq: int):
+        """(starts, lens) lists of ``seq`` in logical order."""
+        count = ctypes.c_int(0)
+        self._lib.seg_attn_pool_segments(self._h, int(seq), None, None, 0, ctypes.byref(count))
+        n = count.value
+        st = np.zeros(max(1, n), dtype=np.int32)
+        ln = np.zeros(max(1, n), dtype=np.int32)
+        rc = self._lib.seg_attn_pool_segments(self._h, int(seq), ctypes.c_void_p(st.ctypes.data),
+                                              ctypes.c_void_p(ln.ctypes.data), n,
+                                              ctypes.byref(count))
+        if rc != 0:
+            raise SegAttnError("seg_attn_pool_segments", rc)
+        return st[:n].tolist(), ln[:n].tolist()
+
+    def stats(self) -> dict:
+        st = seg_attn_pool_stats()
+        rc = self._lib.seg_attn_pool_get_stats(self._h, ctypes.byref(st))
+        if rc != 0:
+            raise SegAttnError("seg_attn_pool_get_stats", rc)
+        return {name: getattr(st, name) for name, _ in st._fields_}
+
+
+def seg_attn_kv_append(k_new, v_new, slots, k_pool, v_pool, stream=None) -> None:
+    """Write k_new / v_new [n, Hkv, d] (device bf16) into the pools at ``slots`` (device int32)."""
+    lib = load_library()
+    rc = lib.seg_attn_kv_append(_dptr(k_new), _dptr(v_new), _dptr(slots), int(slots.numel()),
+                                int(k_pool.shape[1]), int(k_pool.shape[2]), _dptr(k_pool),
+                                _dptr(v_pool), int(k_pool.shape[0]), _stream_ptr(stream))
+    if rc != 0:
+        raise SegAttnError("seg_attn_kv_append", rc)

@@ -90,5 +90,11 @@ extern "C" int seg_attn_decode(const void* q, const void* k_pool, const void* v_
 
 extern "C" int seg_attn_take_device_error(int* value) {
   if (!value) return SEG_ATTN_ERR_INVALID_ARG;
-  return segattn::take_device_error(value);
+  int wait_err = 0, append_err = 0;
+  int rc = segattn::take_device_error(&wait_err);
+  if (rc != SEG_ATTN_OK) return rc;
+  rc = segattn::take_append_error(&append_err);
+  if (rc != SEG_ATTN_OK) return rc;
+  *value = (wait_err ? 1 : 0) | (append_err ? 2 : 0);
+  return SEG_ATTN_OK;
 }

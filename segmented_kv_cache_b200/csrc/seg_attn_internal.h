@@ -75,8 +75,10 @@ struct DecodeLaunch {
 int launch_prefill(const PrefillLaunch& a, cudaStream_t stream);
 int launch_decode(const DecodeLaunch& a, cudaStream_t stream);
 
-// Reads and clears the device error word (set when a bounded wait gave up).
+// Read and clear the device error words: a bounded wait that gave up (prefill)
+// and a KV-append slot out of range.
 int take_device_error(int* value);
+int take_append_error(int* value);
 
 // Workspace split of the decode call.
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }

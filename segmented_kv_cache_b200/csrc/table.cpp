@@ -308,7 +308,8 @@ extern "C" const char* seg_attn_status_string(int status) {
     case SEG_ATTN_ERR_WORKSPACE: return "workspace missing or too small";
     case SEG_ATTN_ERR_UNSUPPORTED: return "unsupported shape";
     case SEG_ATTN_ERR_CUDA: return "CUDA error";
-    case SEG_ATTN_ERR_BUFFER_TOO_SMALL: return "table buffer too small";
+    case SEG_ATTN_ERR_BUFFER_TOO_SMALL: return "output buffer too small";
+    case SEG_ATTN_ERR_NO_SPACE: return "not enough free slots in the pool";
     default: return "unknown status";
   }
 }

@@ -51,6 +51,13 @@ def _load(mutant: int = 0):
                                              ctypes.c_int, ctypes.c_int, ctypes.c_double,
                                              ctypes.c_int, P, P]
             lib.oracle_attention.restype = ctypes.c_int
+            lib.oracle_rows_fp8.argtypes = [ctypes.c_int, P, P, P, P, P, P, P, P, P,
+                                            ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                            ctypes.c_double, ctypes.c_int, ctypes.c_int64, P, P, P,
+                                            P]
+            lib.oracle_rows_fp8.restype = ctypes.c_int
+            lib.oracle_e4m3_decode.argtypes = [P, ctypes.c_int64, P]
+            lib.oracle_e4m3_decode.restype = None
             _libs[mutant] = lib
     return _libs[mutant]
 
@@ -111,3 +118,51 @@ def batch_attention(wl, batch, rows=None):
     """Convenience wrapper over a synthetic workload's batch."""
     return attention(batch.q_lens, batch.seg_starts, batch.seg_lens, batch.q, wl.k_pool,
                      wl.v_pool, wl.scale, batch.causal, rows=rows)
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """float64 values of E4M3 codes (uint8 array), from the format definition."""
+    c = np.ascontiguousarray(np.asarray(codes, dtype=np.uint8).reshape(-1))
+    out = np.zeros(c.size, dtype=np.float64)
+    _load().oracle_e4m3_decode(_ptr(c), c.size, _ptr(out))
+    return out
+
+
+def _codes(t: torch.Tensor) -> np.ndarray:
+    assert t.dtype in (torch.uint8, torch.float8_e4m3fn)
+    return t.detach().cpu().contiguous().view(torch.uint8).numpy()
+
+
+def attention_fp8(q_lens, seg_starts, seg_lens, q, k_pool, v_pool, k_scale, v_scale, scale,
+                  causal, rows=None):
+    """Oracle for an FP8 (E4M3) KV cache: pools of E4M3 codes with per-kv-head scales
+    (``k_scale``/``v_scale``, length Hkv); queries bf16.  Same outputs as ``attention``."""
+    lib = _load()
+    counts = _i32([len(s) for s in seg_starts])
+    starts = _i32([x for s in seg_starts for x in s])
+    lens = _i32([x for s in seg_lens for x in s])
+    ql = _i32(q_lens)
+    qb, kb, vb = _bits(q), _codes(k_pool), _codes(v_pool)
+    ks = np.ascontiguousarray(np.asarray(k_scale, dtype=np.float64).reshape(-1))
+    vs = np.ascontiguousarray(np.asarray(v_scale, dtype=np.float64).reshape(-1))
+    hq, d = q.shape[1], q.shape[2]
+    hkv = k_pool.shape[1]
+    if rows is None:
+        total = int(ql.sum())
+        tok = np.repeat(np.arange(total, dtype=np.int64), hq)
+        head = np.tile(np.arange(hq, dtype=np.int32), total)
+    else:
+        tok = np.ascontiguousarray(np.asarray(rows[0], dtype=np.int64))
+        head = np.ascontiguousarray(np.asarray(rows[1], dtype=np.int32))
+    out = np.zeros((tok.size, d), dtype=np.float64)
+    lse = np.zeros((tok.size,), dtype=np.float64)
+    rc = lib.oracle_rows_fp8(len(q_lens), _ptr(ql), _ptr(counts), _ptr(starts), _ptr(lens),
+                             _ptr(qb), _ptr(kb), _ptr(vb), _ptr(ks), _ptr(vs), hq, hkv, d,
+                             float(scale), int(bool(causal)), tok.size, _ptr(tok), _ptr(head),
+                             _ptr(out), _ptr(lse))
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments")
+    o, l = torch.from_numpy(out), torch.from_numpy(lse)
+    if rows is None:
+        o, l = o.view(-1, hq, d), l.view(-1, hq)
+    return o, l

@@ -266,6 +266,31 @@ int seg_attn_kv_append(const void* k_new, const void* v_new, const int32_t* slot
                        int64_t n_tokens, int kv_heads, int head_dim, void* k_pool, void* v_pool,
                        int64_t num_slots, void* stream);
 
+/*
+ * seg_attn_decode_fp8 -- seg_attn_decode over an FP8 KV cache (Flood README,
+ * "Roadmap": segment attention especially with FP8 kvcache).
+ *   k_pool, v_pool  uint8 E4M3 codes [num_slots, kv_heads, head_dim] (16-byte
+ *                   aligned); the cached value is code * k_scale[g] (v_scale[g])
+ *   k_scale, v_scale  device fp32 [kv_heads], per-kv-head dequantisation scales
+ * Queries stay bf16 (used as f16 in the products: |q| must stay below 65504);
+ * out / lse / table / workspace exactly as seg_attn_decode.  Half the HBM
+ * bytes of the bf16 cache.
+ */
+int seg_attn_decode_fp8(const void* q, const void* k_pool, const void* v_pool, const float* k_scale,
+                        const float* v_scale, void* out, float* lse, const void* dev_table,
+                        const seg_attn_table_desc* desc, float softmax_scale, void* workspace,
+                        size_t workspace_bytes, void* stream);
+
+/*
+ * seg_attn_kv_append_fp8 -- quantise the bf16 K/V rows of new tokens to E4M3
+ * (code = round-to-nearest-even(x / scale[g]), saturated to +-448) and write
+ * them into their slots of FP8 pools.  Same slot rules as seg_attn_kv_append.
+ */
+int seg_attn_kv_append_fp8(const void* k_new, const void* v_new, const int32_t* slots,
+                           int64_t n_tokens, int kv_heads, int head_dim, const float* k_scale,
+                           const float* v_scale, void* k_pool, void* v_pool, int64_t num_slots,
+                           void* stream);
+
 /* Static English description of a status code (never NULL). */
 const char* seg_attn_status_string(int status);
 

@@ -23,6 +23,7 @@ __all__ = [
     "seg_attn_prefill", "seg_attn_decode", "seg_attn_status_string", "seg_attn_version",
     "seg_attn_take_device_error", "SegTable", "load_library", "LIB_PATH",
     "MODE_PREFILL", "MODE_DECODE", "STATUS", "SegPool", "seg_attn_kv_append",
+    "seg_attn_decode_fp8", "seg_attn_kv_append_fp8",
 ]
 
 MODE_PREFILL = 0
@@ -110,6 +111,10 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
             fn.restype = I
         lib.seg_attn_kv_append.argtypes = [P, P, P, I64, I, I, P, P, I64, P]
         lib.seg_attn_kv_append.restype = I
+        lib.seg_attn_kv_append_fp8.argtypes = [P, P, P, I64, I, I, P, P, P, P, I64, P]
+        lib.seg_attn_kv_append_fp8.restype = I
+        lib.seg_attn_decode_fp8.argtypes = [P, P, P, P, P, P, P, P, D, ctypes.c_float, P, SZ, P]
+        lib.seg_attn_decode_fp8.restype = I
         _lib = lib
         return lib
 
@@ -292,3 +297,29 @@ def seg_attn_kv_append(k_new, v_new, slots, k_pool, v_pool, stream=None) -> None
                                 _dptr(v_pool), int(k_pool.shape[0]), _stream_ptr(stream))
     if rc != 0:
         raise SegAttnError("seg_attn_kv_append", rc)
+
+
+def seg_attn_kv_append_fp8(k_new, v_new, slots, k_scale, v_scale, k_pool, v_pool,
+                           stream=None) -> None:
+    """Quantise k_new / v_new (bf16 [n, Hkv, d]) with per-kv-head scales and write the E4M3
+    codes into uint8 pools [S, Hkv, d] at ``slots``."""
+    lib = load_library()
+    rc = lib.seg_attn_kv_append_fp8(_dptr(k_new), _dptr(v_new), _dptr(slots), int(slots.numel()),
+                                    int(k_pool.shape[1]), int(k_pool.shape[2]), _dptr(k_scale),
+                                    _dptr(v_scale), _dptr(k_pool), _dptr(v_pool),
+                                    int(k_pool.shape[0]), _stream_ptr(stream))
+    if rc != 0:
+        raise SegAttnError("seg_attn_kv_append_fp8", rc)
+
+
+def seg_attn_decode_fp8(q, k_pool, v_pool, k_scale, v_scale, out, lse, dev_table, desc,
+                        softmax_scale, workspace=None, stream=None) -> None:
+    """Decode over E4M3 pools (uint8 [S, Hkv, d]) with per-kv-head fp32 scales."""
+    lib = load_library()
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    rc = lib.seg_attn_decode_fp8(_dptr(q), _dptr(k_pool), _dptr(v_pool), _dptr(k_scale),
+                                 _dptr(v_scale), _dptr(out), _dptr(lse), _dptr(dev_table),
+                                 ctypes.byref(desc), float(softmax_scale), _dptr(workspace),
+                                 int(ws_bytes), _stream_ptr(stream))
+    if rc != 0:
+        raise SegAttnError("seg_attn_decode_fp8", rc)

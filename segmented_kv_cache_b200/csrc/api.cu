@@ -60,13 +60,19 @@ extern "C" int seg_attn_prefill(const void* q, const void* k_pool, const void* v
   return segattn::launch_prefill(a, static_cast<cudaStream_t>(stream));
 }
 
-extern "C" int seg_attn_decode(const void* q, const void* k_pool, const void* v_pool, void* out,
-                               float* lse, const void* dev_table, const seg_attn_table_desc* desc,
-                               float softmax_scale, void* workspace, size_t workspace_bytes,
-                               void* stream) {
+namespace {
+
+int decode_common(const void* q, const void* k_pool, const void* v_pool, const float* k_scale,
+                  const float* v_scale, bool fp8, void* out, float* lse, const void* dev_table,
+                  const seg_attn_table_desc* desc, float softmax_scale, void* workspace,
+                  size_t workspace_bytes, void* stream) {
   int rc = check_common(q, k_pool, v_pool, out, lse, dev_table, desc, softmax_scale,
                         SEG_ATTN_MODE_DECODE);
   if (rc != SEG_ATTN_OK) return rc;
+  if (fp8 && desc->total_k > 0 &&
+      (!k_scale || !v_scale || (reinterpret_cast<uintptr_t>(k_scale) & 3) ||
+       (reinterpret_cast<uintptr_t>(v_scale) & 3)))
+    return SEG_ATTN_ERR_INVALID_ARG;
   if (desc->workspace_bytes > 0 &&
       (!workspace || workspace_bytes < desc->workspace_bytes || !aligned16(workspace)))
     return SEG_ATTN_ERR_WORKSPACE;
@@ -85,7 +91,29 @@ extern "C" int seg_attn_decode(const void* q, const void* k_pool, const void* v_
                    ? reinterpret_cast<float*>(static_cast<char*>(workspace) +
                                               segattn::decode_part_o_bytes(*desc))
                    : nullptr;
+  a.fp8 = fp8;
+  a.k_scale = k_scale;
+  a.v_scale = v_scale;
   return segattn::launch_decode(a, static_cast<cudaStream_t>(stream));
+}
+
+}  // namespace
+
+extern "C" int seg_attn_decode(const void* q, const void* k_pool, const void* v_pool, void* out,
+                               float* lse, const void* dev_table, const seg_attn_table_desc* desc,
+                               float softmax_scale, void* workspace, size_t workspace_bytes,
+                               void* stream) {
+  return decode_common(q, k_pool, v_pool, nullptr, nullptr, false, out, lse, dev_table, desc,
+                       softmax_scale, workspace, workspace_bytes, stream);
+}
+
+extern "C" int seg_attn_decode_fp8(const void* q, const void* k_pool, const void* v_pool,
+                                   const float* k_scale, const float* v_scale, void* out,
+                                   float* lse, const void* dev_table,
+                                   const seg_attn_table_desc* desc, float softmax_scale,
+                                   void* workspace, size_t workspace_bytes, void* stream) {
+  return decode_common(q, k_pool, v_pool, k_scale, v_scale, true, out, lse, dev_table, desc,
+                       softmax_scale, workspace, workspace_bytes, stream);
 }
 
 extern "C" int seg_attn_take_device_error(int* value) {

@@ -69,6 +69,9 @@ struct DecodeLaunch {
   float scale;
   float* part_o;    // [num_work][Hq][D] fp32, normalised per chunk
   float* part_lse;  // [num_work][Hq] fp32, log2 domain
+  bool fp8;              // pools hold E4M3 codes
+  const float* k_scale;  // [Hkv] device, FP8 only
+  const float* v_scale;
 };
 
 // Each returns SEG_ATTN_OK or SEG_ATTN_ERR_CUDA (launch error).

@@ -27,7 +27,7 @@ from typing import List, Optional
 import torch
 
 __all__ = ["Batch", "Workload", "make_workload", "CONFIG_NAMES", "split_uniform_cuts",
-           "place_segments"]
+           "place_segments", "fp8_pools"]
 
 CONFIG_NAMES = {
     1: "tiny causal prefill (2 req, q=k=16/33, 4/1 heads, d64)",
@@ -209,3 +209,17 @@ def make_workload(cfg: int, device: str = "cpu", values: bool = True,
                                  st["qk_std"])
         wl.v_pool = _pool_values(wl.num_slots, wl.kv_heads, wl.head_dim, live, vgen, device, 1.0)
     return wl
+
+
+def fp8_pools(k_pool: torch.Tensor, v_pool: torch.Tensor):
+    """E4M3 copies of bf16 pools for the FP8 KV-cache variant: per-kv-head scales so the
+    largest live magnitude maps to 448, codes from torch's float8_e4m3fn cast (free NaN
+    slots stay NaN codes).  Returns (k8, v8 as uint8 views, k_scale, v_scale fp32)."""
+    def one(pool):
+        amax = torch.nan_to_num(pool.float(), nan=0.0).abs().amax(dim=(0, 2)).clamp(min=1e-30)
+        scale = (amax / 448.0).float()
+        codes = (pool.float() / scale.view(1, -1, 1)).clamp(-448, 448).to(torch.float8_e4m3fn)
+        return codes.view(torch.uint8), scale
+    k8, ks = one(k_pool)
+    v8, vs = one(v_pool)
+    return k8, v8, ks, vs

@@ -1,0 +1,118 @@
+"""FP8 (E4M3) KV cache: quantising append (bit-exact) and decode parity against the
+FP8 oracle path (same tolerances as the bf16 cache)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import segmented_kv_cache_b200 as sa
+from segmented_kv_cache_b200 import synth
+
+from helpers import compact_requests, compare, random_case
+
+pytestmark = pytest.mark.gpu
+
+
+def test_fp8_append_matches_torch_quantisation():
+    g = torch.Generator().manual_seed(1)
+    S, hkv, d, n = 3000, 8, 128, 777
+    k_new = (3 * torch.randn(n, hkv, d, generator=g)).to(torch.bfloat16)
+    v_new = (3 * torch.randn(n, hkv, d, generator=g)).to(torch.bfloat16)
+    k_new[0, 0, :4] = torch.tensor([1e4, -1e4, 1e-7, 0.0]).to(torch.bfloat16)  # saturation, tiny
+    ks = (0.01 + torch.rand(hkv, generator=g)).float()
+    vs = (0.01 + torch.rand(hkv, generator=g)).float()
+    slots = torch.randperm(S, generator=g)[:n].to(torch.int32)
+    k8 = torch.zeros(S, hkv, d, dtype=torch.uint8, device="cuda")
+    v8 = torch.zeros_like(k8)
+    sa.seg_attn_kv_append_fp8(k_new.cuda(), v_new.cuda(), slots.cuda(), ks.cuda(), vs.cuda(), k8, v8)
+    torch.cuda.synchronize()
+    ek = (k_new.float() / ks.view(1, -1, 1)).clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8)
+    ev = (v_new.float() / vs.view(1, -1, 1)).clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8)
+    assert torch.equal(k8.cpu()[slots.long()], ek)
+    assert torch.equal(v8.cpu()[slots.long()], ev)
+    untouched = torch.ones(S, dtype=torch.bool)
+    untouched[slots.long()] = False
+    assert int(k8.cpu()[untouched].sum()) == 0
+    assert sa.seg_attn_take_device_error() == 0
+
+
+def _fp8_case(case):
+    k8, v8, ks, vs = synth.fp8_pools(case["k_pool"], case["v_pool"])
+    return dict(case, k8=k8, v8=v8, ks=ks, vs=vs)
+
+
+def _run_fp8(case):
+    q = case["q"].cuda()
+    hq, d = q.shape[1], q.shape[2]
+    tab = sa.SegTable.build(None, case["seg_starts"], case["seg_lens"], case["num_slots"], True,
+                            sa.MODE_DECODE, hq, case["k8"].shape[1], d).to("cuda")
+    out = torch.full_like(q, float("nan"))
+    lse = torch.full(q.shape[:2], float("nan"), dtype=torch.float32, device="cuda")
+    ws = (torch.empty(tab.workspace_bytes, dtype=torch.uint8, device="cuda")
+          if tab.workspace_bytes else None)
+    sa.seg_attn_decode_fp8(q, case["k8"].cuda(), case["v8"].cuda(), case["ks"].cuda(),
+                           case["vs"].cuda(), out, lse, tab.device, tab.desc, case["scale"], ws)
+    torch.cuda.synchronize()
+    return out, lse, tab
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("hq,hkv", [(8, 1), (16, 4), (4, 2), (8, 8)])
+def test_fp8_decode_random(d, hq, hkv):
+    case = _fp8_case(random_case(300 + d + hq + hkv, batch=5, hq=hq, hkv=hkv, d=d, causal=True,
+                                 max_k=4000, nseg_max=6, q_mode="decode"))
+    out, lse, _ = _run_fp8(case)
+    ref_o, ref_l = oracle.attention_fp8(case["q_lens"], case["seg_starts"], case["seg_lens"],
+                                        case["q"], case["k8"], case["v8"], case["ks"], case["vs"],
+                                        case["scale"], True)
+    compare(out, lse, ref_o, ref_l, f"fp8 decode d{d} {hq}/{hkv}")
+
+
+def test_fp8_decode_multichunk_zero_and_tiny_segments():
+    case = random_case(310, batch=6, hq=64, hkv=8, d=128, causal=True, max_k=9000, nseg_max=8,
+                       q_mode="decode")
+    case["seg_starts"][2], case["seg_lens"][2] = [], []
+    g = torch.Generator().manual_seed(2)
+    s3, l3 = [], []
+    for s0, l0 in zip(case["seg_starts"][3], case["seg_lens"][3]):
+        pos = s0
+        while pos < s0 + l0:
+            step = min(int(torch.randint(1, 4, (1,), generator=g)), s0 + l0 - pos)
+            s3.append(pos)
+            l3.append(step)
+            pos += step
+    case["seg_starts"][3], case["seg_lens"][3] = s3, l3
+    case = _fp8_case(case)
+    out, lse, tab = _run_fp8(case)
+    assert tab.workspace_bytes > 0
+    assert torch.all(out[2] == 0) and torch.all(torch.isneginf(lse[2]))
+    ref_o, ref_l = oracle.attention_fp8(case["q_lens"], case["seg_starts"], case["seg_lens"],
+                                        case["q"], case["k8"], case["v8"], case["ks"], case["vs"],
+                                        case["scale"], True)
+    compare(out, lse, ref_o, ref_l, "fp8 mixed")
+
+
+def test_fp8_config4_sampled_requests():
+    wl = synth.make_workload(4, device="cuda")
+    b = wl.batches[0]
+    k8, v8, ks, vs = synth.fp8_pools(wl.k_pool, wl.v_pool)
+    tab = sa.SegTable.build(None, b.seg_starts, b.seg_lens, wl.num_slots, True, sa.MODE_DECODE,
+                            wl.q_heads, wl.kv_heads, wl.head_dim).to("cuda")
+    out = torch.empty_like(b.q)
+    lse = torch.empty(b.q.shape[:2], dtype=torch.float32, device="cuda")
+    ws = torch.empty(tab.workspace_bytes, dtype=torch.uint8, device="cuda")
+    sa.seg_attn_decode_fp8(b.q, k8, v8, ks, vs, out, lse, tab.device, tab.desc, wl.scale, ws)
+    torch.cuda.synchronize()
+    reqs = [0, 17, 63, 127]
+    wl8 = synth.Workload(config=4, name="", q_heads=wl.q_heads, kv_heads=wl.kv_heads,
+                         head_dim=wl.head_dim, num_slots=wl.num_slots, scale=wl.scale,
+                         batches=[b], k_pool=k8, v_pool=v8)
+    sub = compact_requests(wl8, b, reqs)
+    ref_o, ref_l = oracle.attention_fp8(sub["q_lens"], sub["seg_starts"], sub["seg_lens"],
+                                        sub["q"], sub["k_pool"], sub["v_pool"], ks.cpu(),
+                                        vs.cpu(), wl.scale, True)
+    rows = sub["q_rows"].cuda()
+    compare(out[rows], lse[rows], ref_o, ref_l, "fp8 config 4")
+    assert sa.seg_attn_take_device_error() == 0

@@ -65,8 +65,8 @@ def decode_flops(batch, wl):
     return 4.0 * wl.head_dim * wl.q_heads * float(sum(batch.k_lens))
 
 
-def decode_bytes(batch, wl, table_bytes):
-    kv = 2 * 2 * wl.kv_heads * wl.head_dim * float(sum(batch.k_lens))
+def decode_bytes(batch, wl, table_bytes, kv_bytes=2):
+    kv = 2 * kv_bytes * wl.kv_heads * wl.head_dim * float(sum(batch.k_lens))
     qo = 2 * 2 * batch.batch * wl.q_heads * wl.head_dim
     return kv + qo + 4 * batch.batch * wl.q_heads + table_bytes
 
@@ -179,10 +179,13 @@ def cpu_cores():
 class Path:
     """Device-resident buffers + tables of one workload, and the calls of one step."""
 
-    def __init__(self, wl, device):
+    def __init__(self, wl, device, kv_dtype="bf16"):
         self.wl = wl
         self.device = device
         self.legs = []
+        self.kv_dtype = kv_dtype
+        if kv_dtype == "fp8":  # decode legs read E4M3 copies of the pools
+            self.k8, self.v8, self.ks, self.vs = synth.fp8_pools(wl.k_pool, wl.v_pool)
         for b in wl.batches:
             mode = sa.MODE_PREFILL if b.mode == "prefill" else sa.MODE_DECODE
             tab = sa.SegTable.build(b.q_lens if mode == sa.MODE_PREFILL else None, b.seg_starts,
@@ -199,6 +202,11 @@ class Path:
                                   launches=launches))
 
     def run_leg(self, leg, stream=None):
+        if leg["mode"] == sa.MODE_DECODE and self.kv_dtype == "fp8":
+            sa.seg_attn_decode_fp8(leg["batch"].q, self.k8, self.v8, self.ks, self.vs, leg["out"],
+                                   leg["lse"], leg["tab"].device, leg["tab"].desc, self.wl.scale,
+                                   leg["ws"], stream)
+            return
         fn = sa.seg_attn_prefill if leg["mode"] == sa.MODE_PREFILL else sa.seg_attn_decode
         fn(leg["batch"].q, self.wl.k_pool, self.wl.v_pool, leg["out"], leg["lse"],
            leg["tab"].device, leg["tab"].desc, self.wl.scale, leg["ws"], stream)
@@ -314,7 +322,7 @@ def run_ours(args):
     # weak scaling: every rank runs its own batch of the same shape (seed offset by rank)
     wl = synth.make_workload(args.config, device=str(device), seed=rank_seed(args.config, rank),
                              context_scale=args.context_scale)
-    path = Path(wl, device)
+    path = Path(wl, device, args.kv_dtype)
     stream = torch.cuda.current_stream(device)
 
     def step():
@@ -369,7 +377,8 @@ def run_ours(args):
             cand = ("tensor", lm, f)
         else:
             f = decode_flops(b, wl)
-            by = decode_bytes(b, wl, leg["tab"].desc.table_bytes)
+            by = decode_bytes(b, wl, leg["tab"].desc.table_bytes,
+                              1 if args.kv_dtype == "fp8" else 2)
             gbs = by / (lm * 1e-3) / 1e9
             legs["decode"] = {"ms": lm, "gbs": gbs, "bytes": by, "tflops": f / (lm * 1e-3) / 1e12,
                               "frac_hbm": gbs / peaks["hbm_gbs"],
@@ -540,6 +549,8 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=256,
                     help="oracle rows per batch for the cpu_baseline leg of our arm")
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--kv-dtype", choices=["bf16", "fp8"], default="bf16",
+                    help="cache type of the decode legs (fp8: E4M3 with per-kv-head scales)")
     ap.add_argument("--kv-append", action="store_true",
                     help="measure the KV-append kernel instead of the attention step")
     ap.add_argument("--context-scale", type=float, default=1.0,

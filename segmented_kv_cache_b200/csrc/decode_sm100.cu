@@ -358,10 +358,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_chunk_kernel(const D
 // K fragment layout: a thread's 16-byte chunk of a K row holds four k-steps
 // (4 values each: the (2q, 2q+1) and (2q+8, 2q+9) slots); its V chunk holds
 // D/8 consecutive values of one key, O^T row of m-tile i = (D/8)*r + 2i (+1).
-constexpr int kWarpKeys8 = 64;
+constexpr int kWarpKeys8 = 32;  // keys per warp iteration (3 CTAs per SM fit in registers)
 
 template <int D>
-__global__ void __launch_bounds__(kDecodeThreads, 2) decode_chunk_fp8_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(kDecodeThreads, 3) decode_chunk_fp8_kernel(const DecodeParams p) {
   constexpr int KSTEPS = D / 16;  // k-steps of QK, m-tiles of PV
   constexpr int KCH = D / 64;     // 16-byte K chunks per row per thread
   constexpr int VB = D / 8;       // V bytes per key per thread

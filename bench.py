@@ -13,6 +13,11 @@ TFLOPS).  `value` is the step's attention TFLOP/s: (prefill flops, causal
 per-leg numbers (prefill TFLOP/s, decode GB/s) and their fractions of the
 measured peaks are in `legs`.
 
+Configs 6 and 7 are the shared-prefix workloads (prefix caching): their tables
+are built with SEG_ATTN_SHARE_PREFIX, and the same step without sharing is timed
+beside them (`legs.*.plain_ms`).  Their decode roofline counts each distinct K/V
+slot once (the bytes a shared-prefix job must move).
+
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config C]
 """
 from __future__ import annotations
@@ -69,6 +74,41 @@ def decode_bytes(batch, wl, table_bytes, kv_bytes=2):
     kv = 2 * kv_bytes * wl.kv_heads * wl.head_dim * float(sum(batch.k_lens))
     qo = 2 * 2 * batch.batch * wl.q_heads * wl.head_dim
     return kv + qo + 4 * batch.batch * wl.q_heads + table_bytes
+
+
+def distinct_slots(batch):
+    """Number of distinct pool slots the batch's segment lists name."""
+    runs = sorted((s, s + l) for ss, ll in zip(batch.seg_starts, batch.seg_lens)
+                  for s, l in zip(ss, ll) if l > 0)
+    n, end = 0, -1
+    for a, b in runs:
+        if b > end:
+            n += b - max(a, end)
+            end = b
+    return n
+
+
+def decode_bytes_distinct(batch, wl, table_bytes, kv_bytes=2):
+    """decode_bytes with every distinct K/V slot counted once (shared prefixes)."""
+    kv = 2 * kv_bytes * wl.kv_heads * wl.head_dim * float(distinct_slots(batch))
+    qo = 2 * 2 * batch.batch * wl.q_heads * wl.head_dim
+    return kv + qo + 4 * batch.batch * wl.q_heads + table_bytes
+
+
+def launches_of(desc):
+    """Kernel launches one compute call makes for a built table."""
+    shared = desc.shared == 1
+    n = 0
+    if shared and desc.num_group_work > 0:
+        n += 1  # pass over the shared prefixes
+    if desc.mode == sa.MODE_PREFILL:
+        n += (1 if desc.num_work > 0 else 0) + (1 if desc.num_merge > 0 else 0)
+    else:
+        n += 1 if desc.num_work > 0 else 0
+        n += 1 if (desc.workspace_bytes > 0 and not shared) else 0
+    if shared and desc.num_cascade > 0:
+        n += 1
+    return n
 
 
 def source_digest(path):
@@ -179,7 +219,7 @@ def cpu_cores():
 class Path:
     """Device-resident buffers + tables of one workload, and the calls of one step."""
 
-    def __init__(self, wl, device, kv_dtype="bf16"):
+    def __init__(self, wl, device, kv_dtype="bf16", share=False):
         self.wl = wl
         self.device = device
         self.legs = []
@@ -189,15 +229,15 @@ class Path:
         for b in wl.batches:
             mode = sa.MODE_PREFILL if b.mode == "prefill" else sa.MODE_DECODE
             tab = sa.SegTable.build(b.q_lens if mode == sa.MODE_PREFILL else None, b.seg_starts,
-                                    b.seg_lens, wl.num_slots, b.causal, mode, wl.q_heads,
+                                    b.seg_lens, wl.num_slots, b.causal,
+                                    mode | (sa.SHARE_PREFIX if share else 0), wl.q_heads,
                                     wl.kv_heads, wl.head_dim, pin=True)
             tab.to(device)
             out = torch.empty_like(b.q)
             lse = torch.empty(b.q.shape[0], wl.q_heads, dtype=torch.float32, device=device)
             ws = (torch.empty(tab.workspace_bytes, dtype=torch.uint8, device=device)
                   if tab.workspace_bytes else None)
-            # second launch: decode merge, or prefill merge of split items
-            launches = 1 + (1 if tab.workspace_bytes else 0)
+            launches = launches_of(tab.desc)
             self.legs.append(dict(batch=b, mode=mode, tab=tab, out=out, lse=lse, ws=ws,
                                   launches=launches))
 
@@ -219,7 +259,10 @@ def workload_name(wl):
     return {1: "tiny causal prefill", 2: "pages-shaped prefill q=k=1024",
             3: "chunked prefill varlen (16 req, 2048 new tokens)",
             4: "batched decode 128 req k=1024..32768",
-            5: "long-context mix: decode 8x131072 + prefill 2048 over 131072"}[wl.config]
+            5: "long-context mix: decode 8x131072 + prefill 2048 over 131072",
+            6: "shared-prefix decode: 8 groups x 8 req, prefix 8192..32768 + own 512..4096",
+            7: "shared-prefix chunked prefill: 4 groups x 8 req, prefix 4096..16384, "
+               "chunks 4..32"}[wl.config]
 
 
 # ----------------------------------------------------------------------------- oracle legs
@@ -322,7 +365,11 @@ def run_ours(args):
     # weak scaling: every rank runs its own batch of the same shape (seed offset by rank)
     wl = synth.make_workload(args.config, device=str(device), seed=rank_seed(args.config, rank),
                              context_scale=args.context_scale)
-    path = Path(wl, device, args.kv_dtype)
+    share = args.share_prefix if args.share_prefix is not None else wl.config in (6, 7)
+    if share and args.kv_dtype == "fp8":
+        raise SystemExit("shared-prefix tables run the bf16 tensor-core prefix pass; "
+                         "use --kv-dtype bf16 or --no-share-prefix")
+    path = Path(wl, device, args.kv_dtype, share)
     stream = torch.cuda.current_stream(device)
 
     def step():
@@ -360,6 +407,7 @@ def run_ours(args):
               for i in range(len(path.legs))]
     ms = max_over_ranks(ms, dist, device)
     assert sa.seg_attn_take_device_error() == 0
+    plain_ms = time_plain_legs(wl, device, args) if share else None
 
     peaks, peak_kind = load_peaks()
     flops_step = 0.0
@@ -372,22 +420,34 @@ def run_ours(args):
             tf = f / (lm * 1e-3) / 1e12
             legs["prefill"] = {"ms": lm, "tflops": tf, "flops": f,
                                "frac_sustained": tf / peaks["bf16_tflops_sustained"],
-                               "frac_burst": tf / peaks["bf16_tflops"]}
+                               "frac_burst": tf / peaks["bf16_tflops"],
+                               "launches": leg["launches"]}
             flops_step += f
             cand = ("tensor", lm, f)
         else:
             f = decode_flops(b, wl)
-            by = decode_bytes(b, wl, leg["tab"].desc.table_bytes,
-                              1 if args.kv_dtype == "fp8" else 2)
+            kvb = 1 if args.kv_dtype == "fp8" else 2
+            by = decode_bytes(b, wl, leg["tab"].desc.table_bytes, kvb)
+            if share:  # shared prefixes: the job must move each distinct slot once
+                eff = by / (lm * 1e-3) / 1e9
+                by = decode_bytes_distinct(b, wl, leg["tab"].desc.table_bytes, kvb)
             gbs = by / (lm * 1e-3) / 1e9
             legs["decode"] = {"ms": lm, "gbs": gbs, "bytes": by, "tflops": f / (lm * 1e-3) / 1e12,
                               "frac_hbm": gbs / peaks["hbm_gbs"],
                               "launches": leg["launches"]}
+            if share:
+                legs["decode"]["gbs_effective"] = eff  # every request's keys counted
             flops_step += f
             cand = ("hbm", lm, by)
         if dominant is None or cand[1] > dominant[1]:
             dominant = cand
     value = job_throughput(world, flops_step, ms, args.steps) / 1e12
+    if plain_ms is not None:
+        for leg, pm in zip(path.legs, plain_ms):
+            name = "prefill" if leg["mode"] == sa.MODE_PREFILL else "decode"
+            legs[name]["plain_ms"] = pm
+            legs[name]["speedup_vs_plain"] = pm / legs[name]["ms"]
+            legs[name]["shared_groups"] = int(leg["tab"].desc.num_groups)
 
     if dominant[0] == "tensor":
         achieved = dominant[2] / (dominant[1] * 1e-3) / 1e12
@@ -400,9 +460,11 @@ def run_ours(args):
         achieved = dominant[2] / (dominant[1] * 1e-3) / 1e9
         peak = peaks["hbm_gbs"]
         traffic = profiled_traffic("decode_sm100", f"cfg{wl.config}")
+        kern = ("prefill_kernel<128> over shared prefixes + decode_chunk_kernel<128> + "
+                "cascade_merge_kernel<128>" if share else
+                "decode_chunk_kernel<128> + decode_merge_kernel<128>")
         roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": achieved / peak, "traffic": traffic,
-                "kernel": "decode_chunk_kernel<128> + decode_merge_kernel<128>",
+                "frac": achieved / peak, "traffic": traffic, "kernel": kern,
                 "peak_kind": f"{peak_kind} copy bandwidth"}
 
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
@@ -417,7 +479,8 @@ def run_ours(args):
                        "l2": ("inputs larger than L2 (pools %.1f GB), no flush" %
                               (2 * wl.k_pool.numel() * 2 / 1e9))
                        if 2 * wl.k_pool.numel() * 2 > L2_BYTES else "inputs fit in L2",
-                       "parallelism": f"dp{world} (independent batches per GPU)"},
+                       "parallelism": f"dp{world} (independent batches per GPU)",
+                       "share_prefix": bool(share)},
             "legs": legs, "roofline": roof,
             "gpu_launches": path.launches_per_step() * args.steps,
             "clocks": clocks}
@@ -432,6 +495,26 @@ def run_ours(args):
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def time_plain_legs(wl, device, args):
+    """Per-leg ms of the same workload with plain (unshared) tables, for comparison."""
+    plain = Path(wl, device, args.kv_dtype, share=False)
+    stream = torch.cuda.current_stream(device)
+    for _ in range(args.warmup):
+        for leg in plain.legs:
+            plain.run_leg(leg)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(plain.legs) + 1)]
+    tot = [0.0] * len(plain.legs)
+    for _ in range(args.steps):
+        ev[0].record(stream)
+        for i, leg in enumerate(plain.legs):
+            plain.run_leg(leg)
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize()
+        for i in range(len(plain.legs)):
+            tot[i] += ev[i].elapsed_time(ev[i + 1])
+    return [t / args.steps for t in tot]
 
 
 def run_e2e(path, args, world):
@@ -543,7 +626,10 @@ def main():
     ap.add_argument("--steps", type=int, default=40)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", type=int, default=5, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--config", type=int, default=5, choices=[1, 2, 3, 4, 5, 6, 7])
+    ap.add_argument("--share-prefix", dest="share_prefix", action="store_true", default=None,
+                    help="build tables with SEG_ATTN_SHARE_PREFIX (default: configs 6 and 7)")
+    ap.add_argument("--no-share-prefix", dest="share_prefix", action="store_false")
     ap.add_argument("--ref-rows", type=int, default=48,
                     help="oracle rows per batch per step (bounded CPU sample)")
     ap.add_argument("--cpu-rows", type=int, default=256,

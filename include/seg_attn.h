@@ -70,8 +70,12 @@ typedef enum {
 
 enum { SEG_ATTN_MODE_PREFILL = 0, SEG_ATTN_MODE_DECODE = 1 };
 
+/* OR-ed into the mode argument of seg_attn_build_table: plan shared prefixes
+ * (see seg_attn_build_table). */
+#define SEG_ATTN_SHARE_PREFIX 0x100
+
 #define SEG_ATTN_TABLE_MAGIC 0x53454741u /* "SEGA" */
-#define SEG_ATTN_TABLE_VERSION 2u
+#define SEG_ATTN_TABLE_VERSION 3u
 
 /*
  * Description of a built segment table.  Filled by seg_attn_build_table; the
@@ -92,8 +96,9 @@ typedef struct seg_attn_table_desc {
   int32_t chunk_len;       /* decode: logical keys per split-K chunk */
   int32_t max_k_tiles;     /* prefill: largest number of 128-key tiles of one item */
   int32_t num_merge;       /* prefill: items whose key range was split over several CTAs */
-  int32_t num_parts;       /* prefill: partial-result slots of those items */
-  int32_t reserved0;
+  int32_t num_parts;       /* prefill: partial-result slots (split items, and every item of
+                              a request in a shared-prefix group) */
+  int32_t shared;          /* 1: a shared-prefix plan is present (fields below) */
   int64_t off_q_offsets;   /* [batch+1] packed query offset of each request */
   int64_t off_k_lens;      /* [batch]   keys of each request */
   int64_t off_seg_offsets; /* [batch+1] first segment of each request */
@@ -106,6 +111,31 @@ typedef struct seg_attn_table_desc {
   int64_t off_merge;       /* prefill: [num_merge][8] split items and their partial slots */
   uint64_t table_bytes;    /* size of the table buffer */
   uint64_t workspace_bytes;/* device scratch the compute call needs (may be 0) */
+  /* Shared-prefix plan (shared == 1).  Requests are cut into groups of
+     consecutive requests; group p's members map their first P_p logical keys
+     to the same slots.  The arrays above then describe each request's keys
+     from P_p on (its suffix); the group arrays below describe the shared
+     prefixes, one pseudo-request per group whose queries are all its
+     members' queries.  A request that shares nothing is a group of its own
+     with P = 0. */
+  int32_t num_groups;
+  int32_t num_group_segments;
+  int32_t num_group_work;  /* prefill-kernel pieces over the shared prefixes */
+  int32_t num_group_parts; /* partial-result slots of those pieces */
+  int32_t num_citems;      /* items whose pieces write partials for the cascade merge */
+  int32_t num_cascade;     /* output rows (prefill: tokens, decode: requests) merged by it */
+  int64_t group_total_k;   /* sum of P_p */
+  int64_t off_group_req;        /* [num_groups+1] first request of each group */
+  int64_t off_group_q_offsets;  /* [num_groups+1] first query (packed row) of each group */
+  int64_t off_group_k_lens;     /* [num_groups] P_p */
+  int64_t off_group_seg_offsets;/* [num_groups+1] */
+  int64_t off_group_seg_start;  /* [num_group_segments] */
+  int64_t off_group_seg_kstart; /* [num_group_segments] */
+  int64_t off_group_seg_len;    /* [num_group_segments] */
+  int64_t off_group_work;       /* [num_group_work][8] */
+  int64_t off_citem;            /* [num_citems][4] first slot, pieces, first query of the item */
+  int64_t off_cascade;          /* [num_cascade][8] row, request, prefix item, row in group,
+                                   suffix item, row in request */
 } seg_attn_table_desc;
 
 /*
@@ -121,14 +151,30 @@ typedef struct seg_attn_table_desc {
  *   num_slots             pool rows; every segment must lie in [0, num_slots)
  *   causal                1 = bottom-right causal mask, 0 = none (decode
  *                         always sees every key of the request)
- *   mode                  SEG_ATTN_MODE_PREFILL or SEG_ATTN_MODE_DECODE
+ *   mode                  SEG_ATTN_MODE_PREFILL or SEG_ATTN_MODE_DECODE, optionally
+ *                         OR-ed with SEG_ATTN_SHARE_PREFIX
  *   q_heads, kv_heads, head_dim   shapes as above
  *   host_out, host_out_bytes      destination (any alignment >= 16 bytes);
  *                         pass host_out = NULL to only fill desc (size query)
  *   desc                  out: table description
  *
  * Segments of different requests may share slots (read-only prefix sharing);
- * segments of one request may not.  Returns SEG_ATTN_OK or a negative status;
+ * segments of one request may not.
+ *
+ * SEG_ATTN_SHARE_PREFIX (prefix caching, Flood README "Roadmap"): the builder
+ * finds, for each pair of neighbouring requests, how many leading logical keys
+ * they map to the same slots, and cuts the batch into groups of consecutive
+ * requests so that the number of K/V tiles read is smallest (a group's common
+ * prefix is read once per 256 packed query rows instead of once per request;
+ * prefixes shorter than 256 keys are not shared; a causal prefill prefix
+ * stops where a member's new tokens begin).  The compute call then runs the
+ * tensor-core prefill kernel over each shared prefix with all the group's
+ * queries, the usual kernel over each request's remaining keys, and a merge of
+ * the two partial results by their log-sum-exp; the results equal the
+ * unshared computation up to fp32 rounding.  Callers that want sharing order
+ * requests with common prefixes next to each other.  When no group shares
+ * anything the table is the plain one (desc->shared = 0).
+ * Returns SEG_ATTN_OK or a negative status;
  * on SEG_ATTN_ERR_BUFFER_TOO_SMALL desc->table_bytes holds the needed size.
  * Host only: touches no device state.  The caller copies table_bytes of
  * host_out to device memory (16-byte aligned) and passes that copy as
@@ -177,7 +223,7 @@ int seg_attn_decode(const void* q, const void* k_pool, const void* v_pool, void*
  * word.  Kernels never trap; every wait on an mbarrier gives up after one
  * second, and a CTA that gave up drains its copies, frees its tensor memory,
  * returns, and sets bit 0 of this word (its output rows are then undefined);
- * seg_attn_kv_append sets bit 1 for a slot out of range.  Synchronous: copies from the device (implicitly synchronises
+ * seg_attn_kv_append sets bit 1 (value 2) for a slot out of range.  Synchronous: copies from the device (implicitly synchronises
  * the current device).  *value = 0 means no kernel gave up since the last call.
  */
 int seg_attn_take_device_error(int* value);
@@ -259,7 +305,7 @@ int seg_attn_pool_get_stats(const seg_attn_pool* pool, seg_attn_pool_stats* out)
  *   slots          int32 [n_tokens] device array, slot of each token
  *   k_pool, v_pool bf16 [num_slots, kv_heads, head_dim] (device)
  * A slot outside [0, num_slots) is skipped and recorded in the device error
- * word (bit 2, see seg_attn_take_device_error); nothing is written out of
+ * word (value 2, see seg_attn_take_device_error); nothing is written out of
  * bounds.  kv_heads * head_dim * 2 must be a multiple of 16 bytes.
  */
 int seg_attn_kv_append(const void* k_new, const void* v_new, const int32_t* slots,

@@ -23,11 +23,12 @@ __all__ = [
     "seg_attn_prefill", "seg_attn_decode", "seg_attn_status_string", "seg_attn_version",
     "seg_attn_take_device_error", "SegTable", "load_library", "LIB_PATH",
     "MODE_PREFILL", "MODE_DECODE", "STATUS", "SegPool", "seg_attn_kv_append",
-    "seg_attn_decode_fp8", "seg_attn_kv_append_fp8",
+    "seg_attn_decode_fp8", "seg_attn_kv_append_fp8", "SHARE_PREFIX",
 ]
 
 MODE_PREFILL = 0
 MODE_DECODE = 1
+SHARE_PREFIX = 0x100  # OR into the mode: plan shared prefixes
 STATUS = {
     "OK": 0, "INVALID_ARG": -1, "SEGMENT_OOB": -2, "SEGMENT_OVERLAP": -3, "QLEN_GT_KLEN": -4,
     "WORKSPACE": -5, "UNSUPPORTED": -6, "CUDA": -7, "BUFFER_TOO_SMALL": -8, "NO_SPACE": -9,
@@ -45,13 +46,22 @@ class seg_attn_table_desc(ctypes.Structure):
         ("num_segments", ctypes.c_int32), ("num_work", ctypes.c_int32),
         ("queries_per_tile", ctypes.c_int32), ("chunk_len", ctypes.c_int32),
         ("max_k_tiles", ctypes.c_int32), ("num_merge", ctypes.c_int32),
-        ("num_parts", ctypes.c_int32), ("reserved0", ctypes.c_int32),
+        ("num_parts", ctypes.c_int32), ("shared", ctypes.c_int32),
         ("off_q_offsets", ctypes.c_int64), ("off_k_lens", ctypes.c_int64),
         ("off_seg_offsets", ctypes.c_int64), ("off_seg_start", ctypes.c_int64),
         ("off_seg_kstart", ctypes.c_int64), ("off_seg_len", ctypes.c_int64),
         ("off_work", ctypes.c_int64), ("off_req_chunks", ctypes.c_int64),
         ("off_merge", ctypes.c_int64),
         ("table_bytes", ctypes.c_uint64), ("workspace_bytes", ctypes.c_uint64),
+        ("num_groups", ctypes.c_int32), ("num_group_segments", ctypes.c_int32),
+        ("num_group_work", ctypes.c_int32), ("num_group_parts", ctypes.c_int32),
+        ("num_citems", ctypes.c_int32), ("num_cascade", ctypes.c_int32),
+        ("group_total_k", ctypes.c_int64),
+        ("off_group_req", ctypes.c_int64), ("off_group_q_offsets", ctypes.c_int64),
+        ("off_group_k_lens", ctypes.c_int64), ("off_group_seg_offsets", ctypes.c_int64),
+        ("off_group_seg_start", ctypes.c_int64), ("off_group_seg_kstart", ctypes.c_int64),
+        ("off_group_seg_len", ctypes.c_int64), ("off_group_work", ctypes.c_int64),
+        ("off_citem", ctypes.c_int64), ("off_cascade", ctypes.c_int64),
     ]
 
 

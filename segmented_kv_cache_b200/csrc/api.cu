@@ -29,6 +29,43 @@ int check_common(const void* q, const void* k_pool, const void* v_pool, const vo
   return SEG_ATTN_OK;
 }
 
+char* at(void* base, size_t off) { return static_cast<char*>(base) + off; }
+
+// The pass over the shared prefixes (prefill kernel, every piece a partial).
+int launch_group_pass(const void* q, const void* k_pool, const void* v_pool, const void* dev_table,
+                      const seg_attn_table_desc& desc, const segattn::WorkspaceLayout& ws_at,
+                      void* workspace, float scale, cudaStream_t stream) {
+  if (desc.num_group_work == 0) return SEG_ATTN_OK;
+  const seg_attn_table_desc gd = segattn::group_pass_desc(desc);
+  segattn::PrefillLaunch a;
+  a.q = q;
+  a.k_pool = k_pool;
+  a.v_pool = v_pool;
+  a.out = nullptr;  // every piece writes to the workspace
+  a.lse = nullptr;
+  a.tab = segattn::make_view(dev_table, gd);
+  a.desc = &gd;
+  a.scale = scale;
+  a.part_o = reinterpret_cast<float*>(at(workspace, ws_at.group_o));
+  a.part_lse = reinterpret_cast<float*>(at(workspace, ws_at.group_lse));
+  return segattn::launch_prefill(a, stream);
+}
+
+int launch_cascade(const void* dev_table, const seg_attn_table_desc& desc,
+                   const segattn::WorkspaceLayout& ws_at, void* workspace, void* out, float* lse,
+                   cudaStream_t stream) {
+  segattn::CascadeLaunch c;
+  c.dev_table = dev_table;
+  c.desc = &desc;
+  c.main_o = reinterpret_cast<const float*>(at(workspace, ws_at.main_o));
+  c.main_lse = reinterpret_cast<const float*>(at(workspace, ws_at.main_lse));
+  c.group_o = reinterpret_cast<const float*>(at(workspace, ws_at.group_o));
+  c.group_lse = reinterpret_cast<const float*>(at(workspace, ws_at.group_lse));
+  c.out = out;
+  c.lse = lse;
+  return segattn::launch_cascade_merge(c, stream);
+}
+
 }  // namespace
 
 extern "C" int seg_attn_prefill(const void* q, const void* k_pool, const void* v_pool, void* out,
@@ -41,23 +78,31 @@ extern "C" int seg_attn_prefill(const void* q, const void* k_pool, const void* v
   if (desc->workspace_bytes > 0 &&
       (!workspace || workspace_bytes < desc->workspace_bytes || !aligned16(workspace)))
     return SEG_ATTN_ERR_WORKSPACE;
-  if (desc->num_work == 0) return SEG_ATTN_OK;
-  segattn::PrefillLaunch a;
-  a.q = q;
-  a.k_pool = k_pool;
-  a.v_pool = v_pool;
-  a.out = out;
-  a.lse = lse;
-  a.tab = segattn::make_view(dev_table, *desc);
-  a.desc = desc;
-  a.scale = softmax_scale;
-  a.part_o = static_cast<float*>(workspace);
-  a.part_lse = desc->workspace_bytes > 0
-                   ? reinterpret_cast<float*>(
-                         static_cast<char*>(workspace) +
-                         segattn::prefill_part_o_bytes(desc->num_parts, desc->head_dim))
-                   : nullptr;
-  return segattn::launch_prefill(a, static_cast<cudaStream_t>(stream));
+  if (desc->num_work == 0 && desc->num_group_work == 0) return SEG_ATTN_OK;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const segattn::WorkspaceLayout ws_at = segattn::workspace_layout(*desc, false);
+  if (desc->shared) {
+    rc = launch_group_pass(q, k_pool, v_pool, dev_table, *desc, ws_at, workspace, softmax_scale, st);
+    if (rc != SEG_ATTN_OK) return rc;
+  }
+  if (desc->num_work > 0) {
+    segattn::PrefillLaunch a;
+    a.q = q;
+    a.k_pool = k_pool;
+    a.v_pool = v_pool;
+    a.out = out;
+    a.lse = lse;
+    a.tab = segattn::make_view(dev_table, *desc);
+    a.desc = desc;
+    a.scale = softmax_scale;
+    a.part_o = desc->num_parts > 0 ? reinterpret_cast<float*>(at(workspace, ws_at.main_o)) : nullptr;
+    a.part_lse =
+        desc->num_parts > 0 ? reinterpret_cast<float*>(at(workspace, ws_at.main_lse)) : nullptr;
+    rc = segattn::launch_prefill(a, st);
+    if (rc != SEG_ATTN_OK) return rc;
+  }
+  if (desc->shared) return launch_cascade(dev_table, *desc, ws_at, workspace, out, lse, st);
+  return SEG_ATTN_OK;
 }
 
 namespace {
@@ -69,6 +114,8 @@ int decode_common(const void* q, const void* k_pool, const void* v_pool, const f
   int rc = check_common(q, k_pool, v_pool, out, lse, dev_table, desc, softmax_scale,
                         SEG_ATTN_MODE_DECODE);
   if (rc != SEG_ATTN_OK) return rc;
+  // the pass over shared prefixes runs on the bf16 tensor-core prefill kernel
+  if (fp8 && desc->shared) return SEG_ATTN_ERR_UNSUPPORTED;
   if (fp8 && desc->total_k > 0 &&
       (!k_scale || !v_scale || (reinterpret_cast<uintptr_t>(k_scale) & 3) ||
        (reinterpret_cast<uintptr_t>(v_scale) & 3)))
@@ -77,6 +124,13 @@ int decode_common(const void* q, const void* k_pool, const void* v_pool, const f
       (!workspace || workspace_bytes < desc->workspace_bytes || !aligned16(workspace)))
     return SEG_ATTN_ERR_WORKSPACE;
   if (desc->num_work == 0) return SEG_ATTN_OK;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const segattn::WorkspaceLayout ws_at =
+      segattn::workspace_layout(*desc, desc->workspace_bytes > 0);
+  if (desc->shared) {
+    rc = launch_group_pass(q, k_pool, v_pool, dev_table, *desc, ws_at, workspace, softmax_scale, st);
+    if (rc != SEG_ATTN_OK) return rc;
+  }
   segattn::DecodeLaunch a;
   a.q = q;
   a.k_pool = k_pool;
@@ -86,15 +140,18 @@ int decode_common(const void* q, const void* k_pool, const void* v_pool, const f
   a.tab = segattn::make_view(dev_table, *desc);
   a.desc = desc;
   a.scale = softmax_scale;
-  a.part_o = static_cast<float*>(workspace);
+  a.part_o = desc->workspace_bytes > 0 ? reinterpret_cast<float*>(at(workspace, ws_at.main_o))
+                                       : nullptr;
   a.part_lse = desc->workspace_bytes > 0
-                   ? reinterpret_cast<float*>(static_cast<char*>(workspace) +
-                                              segattn::decode_part_o_bytes(*desc))
+                   ? reinterpret_cast<float*>(at(workspace, ws_at.main_lse))
                    : nullptr;
   a.fp8 = fp8;
   a.k_scale = k_scale;
   a.v_scale = v_scale;
-  return segattn::launch_decode(a, static_cast<cudaStream_t>(stream));
+  rc = segattn::launch_decode(a, st);
+  if (rc != SEG_ATTN_OK) return rc;
+  if (desc->shared) return launch_cascade(dev_table, *desc, ws_at, workspace, out, lse, st);
+  return SEG_ATTN_OK;
 }
 
 }  // namespace

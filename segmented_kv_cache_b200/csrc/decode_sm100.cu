@@ -610,7 +610,8 @@ int launch_decode_d(const DecodeLaunch& a, cudaStream_t stream) {
   else
     decode_chunk_kernel<D><<<dim3(d.num_work, d.kv_heads), kDecodeThreads, 0, stream>>>(p);
   if (cudaGetLastError() != cudaSuccess) return SEG_ATTN_ERR_CUDA;
-  if (d.workspace_bytes > 0) {
+  // a shared-prefix table leaves every merge to the cascade merge
+  if (d.workspace_bytes > 0 && !d.shared) {
     decode_merge_kernel<D><<<dim3(d.batch, (d.q_heads + 3) / 4), 128, 0, stream>>>(p);
     if (cudaGetLastError() != cudaSuccess) return SEG_ATTN_ERR_CUDA;
   }

@@ -387,7 +387,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu,
                       mbar_wait(o_full + t, (n_tiles - 1) & 1, abort_flag, kWaitLimitNs));
     if (ok && slot >= 0) {
-      // piece of a split item: O / l and log2(sum of exp) of this key range, every row
+      // piece of a split item (or of a shared-prefix pass): O / l and log2(sum of exp)
+      // of this key range, for every row that holds a query
       const float inv = l > 0.f ? 1.f / l : 0.f;
       const int64_t prow = (int64_t)slot * kItemRows + t * kTileRows + row;
       float* po = p.part_o + prow * D;
@@ -402,13 +403,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[e] = 0u;
         }
+        if (row_valid) {
 #pragma unroll
-        for (int e = 0; e < 32; e += 4)
-          *reinterpret_cast<float4*>(po + 32 * c + e) =
-              make_float4(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv,
-                          __uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(po + 32 * c + e) =
+                make_float4(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv,
+                            __uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
+        }
       }
-      p.part_lse[prow] = l > 0.f ? m_ref * sl2 + log2f(l) : -INFINITY;
+      if (row_valid) p.part_lse[prow] = l > 0.f ? m_ref * sl2 + log2f(l) : -INFINITY;
     } else if (ok) {
       const float inv = l > 0.f ? 1.f / l : 0.f;
       __nv_bfloat16* orow = p.out + ((int64_t)(tok0 + qi) * p.q_heads + head) * D;

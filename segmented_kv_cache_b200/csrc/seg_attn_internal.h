@@ -16,6 +16,8 @@ constexpr int kItemRows = kTileRows * kTilesPerItem;  // query rows of one prefi
 constexpr int kMinPieceTiles = 8;       // shortest K range a split prefill piece gets
 constexpr int kPieceOverheadTiles = 2;  // per-piece cost (prologue, epilogue) in K tiles
 constexpr int kMaxSplit = 4;            // most pieces one prefill item is cut into
+constexpr int kMaxGroupSplit = 32;      // the same for a pass over a shared prefix
+constexpr int kMinSharedKeys = 256;     // shortest prefix worth a pass of its own
 
 // Device views of the table arrays (device pointers into dev_table).
 struct TableView {
@@ -29,6 +31,32 @@ struct TableView {
   const int4* merge;          // prefill [num_merge][2]
   const int32_t* req_chunks;  // [B+1] (decode)
 };
+
+// The pass over the shared prefixes is the prefill kernel run on a table of its
+// own: one pseudo-request per group (its members' queries, non-causal, the
+// prefix keys), every piece writing a partial.  This description of it points
+// into the same table buffer.
+inline seg_attn_table_desc group_pass_desc(const seg_attn_table_desc& d) {
+  seg_attn_table_desc g = d;
+  g.mode = SEG_ATTN_MODE_PREFILL;
+  g.causal = 0;
+  g.batch = d.num_groups;
+  g.total_k = d.group_total_k;
+  g.num_segments = d.num_group_segments;
+  g.num_work = d.num_group_work;
+  g.num_merge = 0;
+  g.num_parts = d.num_group_parts;
+  g.shared = 0;
+  g.off_q_offsets = d.off_group_q_offsets;
+  g.off_k_lens = d.off_group_k_lens;
+  g.off_seg_offsets = d.off_group_seg_offsets;
+  g.off_seg_start = d.off_group_seg_start;
+  g.off_seg_kstart = d.off_group_seg_kstart;
+  g.off_seg_len = d.off_group_seg_len;
+  g.off_work = d.off_group_work;
+  g.off_merge = 0;
+  return g;
+}
 
 inline TableView make_view(const void* dev_table, const seg_attn_table_desc& d) {
   const int32_t* t = static_cast<const int32_t*>(dev_table);
@@ -91,5 +119,48 @@ inline size_t prefill_part_o_bytes(int64_t slots, int head_dim) {
 inline size_t decode_part_o_bytes(const seg_attn_table_desc& d) {
   return align_up((size_t)d.num_work * d.q_heads * d.head_dim * sizeof(float), 256);
 }
+
+// Byte offsets of the partial results in the workspace: the main pass's
+// (prefill pieces [slot][kItemRows][D] + [slot][kItemRows], or decode chunks
+// [chunk][Hq][D] + [chunk][Hq]), then the shared-prefix pass's pieces.
+struct WorkspaceLayout {
+  size_t main_o = 0, main_lse = 0, group_o = 0, group_lse = 0, total = 0;
+};
+inline WorkspaceLayout workspace_layout(const seg_attn_table_desc& d, bool decode_partials) {
+  WorkspaceLayout w;
+  size_t at = 0;
+  if (d.mode == SEG_ATTN_MODE_PREFILL) {
+    if (d.num_parts > 0) {
+      at = prefill_part_o_bytes(d.num_parts, d.head_dim);
+      w.main_lse = at;
+      at += align_up((size_t)d.num_parts * kItemRows * sizeof(float), 256);
+    }
+  } else if (decode_partials || d.shared) {
+    at = decode_part_o_bytes(d);
+    w.main_lse = at;
+    at += align_up((size_t)d.num_work * d.q_heads * sizeof(float), 256);
+  }
+  if (d.shared && d.num_group_parts > 0) {
+    w.group_o = at;
+    at += prefill_part_o_bytes(d.num_group_parts, d.head_dim);
+    w.group_lse = at;
+    at += align_up((size_t)d.num_group_parts * kItemRows * sizeof(float), 256);
+  }
+  w.total = at;
+  return w;
+}
+
+// Merge of the shared-prefix partials with each request's own partials.
+struct CascadeLaunch {
+  const void* dev_table;
+  const seg_attn_table_desc* desc;
+  const float* main_o;
+  const float* main_lse;
+  const float* group_o;
+  const float* group_lse;
+  void* out;
+  float* lse;
+};
+int launch_cascade_merge(const CascadeLaunch& a, cudaStream_t stream);
 
 }  // namespace segattn

@@ -13,6 +13,10 @@
 //   decode:  split-K chunks of logical keys (per-block partial attention with
 //            a per-request reduction, FlashAccel article, "data layout
 //            optimisation"), sized so the grid covers the 148 SMs many times.
+// With SEG_ATTN_SHARE_PREFIX (prefix caching, Flood README "Roadmap") it also
+// finds requests whose leading keys sit in the same slots and plans one pass of
+// the prefill kernel over each shared prefix with all the sharing requests'
+// queries, the usual work over each request's remaining keys, and a merge.
 #include <stdint.h>
 #include <string.h>
 
@@ -30,6 +34,8 @@
 namespace {
 
 using segattn::align_up;
+using Row8 = std::array<int32_t, 8>;
+using Row4 = std::array<int32_t, 4>;
 
 bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 
@@ -43,15 +49,188 @@ struct Layout {
   }
 };
 
+// A request's keys as a segment list (start, len) in logical order.
+struct Segs {
+  std::vector<int32_t> start, len;
+  int64_t keys() const {
+    int64_t k = 0;
+    for (int32_t l : len) k += l;
+    return k;
+  }
+};
+
+// Leading logical keys that two segment lists map to the same slots.
+int64_t common_prefix(const Segs& a, const Segs& b) {
+  size_t ia = 0, ib = 0;
+  int64_t oa = 0, ob = 0, n = 0;
+  for (;;) {
+    while (ia < a.len.size() && oa >= a.len[ia]) ++ia, oa = 0;
+    while (ib < b.len.size() && ob >= b.len[ib]) ++ib, ob = 0;
+    if (ia == a.len.size() || ib == b.len.size()) return n;
+    if ((int64_t)a.start[ia] + oa != (int64_t)b.start[ib] + ob) return n;
+    const int64_t step = std::min<int64_t>(a.len[ia] - oa, b.len[ib] - ob);
+    n += step;
+    oa += step;
+    ob += step;
+  }
+}
+
+// Keys [from, from + count) of a segment list, as a segment list.
+Segs cut(const Segs& s, int64_t from, int64_t count) {
+  Segs out;
+  int64_t logical = 0;
+  for (size_t i = 0; i < s.len.size() && count > 0; ++i) {
+    const int64_t lo = std::max<int64_t>(from, logical), hi = logical + s.len[i];
+    if (lo < hi) {
+      const int64_t take = std::min(hi - lo, count);
+      out.start.push_back((int32_t)(s.start[i] + (lo - logical)));
+      out.len.push_back((int32_t)take);
+      from = lo + take;
+      count -= take;
+    }
+    logical = hi;
+  }
+  return out;
+}
+
+// One prefill item: (request, kv head, query tiles from q0) over `tiles` K tiles.
+// `cascade` items write every piece as a partial for the shared-prefix merge.
+struct PItem {
+  int32_t r, g, q0, tiles;
+  bool cascade;
+};
+
+struct Pieces {
+  std::vector<Row8> work;       // pieces, longest first
+  std::vector<Row8> merge;      // split items that are not cascade items
+  std::vector<int32_t> citem;   // per item: its index in `citems`, or -1
+  int32_t slots = 0;            // partial-result slots
+};
+
+// Cut items into pieces along their K tiles when that shortens the
+// longest-first schedule on the SMs.  Each CTA runs one piece; the schedule is
+// simulated by assigning pieces longest first to the least loaded SM (what the
+// block scheduler does with a grid in that order) and the split factor with the
+// shortest makespan wins (ties keep fewer splits).
+void plan_pieces(const std::vector<PItem>& items, int max_split, std::vector<Row4>& citems,
+                 Pieces& out) {
+  auto pieces_of = [](int32_t tiles, int f) {
+    if (f <= 1 || tiles < 2 * segattn::kMinPieceTiles) return 1;
+    return std::min(f, tiles / segattn::kMinPieceTiles);
+  };
+  auto makespan = [&](int f) {
+    std::vector<int64_t> cost;
+    for (const PItem& it : items) {
+      const int p = pieces_of(it.tiles, f);
+      for (int j = 0; j < p; ++j)
+        cost.push_back((int64_t)it.tiles * (j + 1) / p - (int64_t)it.tiles * j / p +
+                       segattn::kPieceOverheadTiles);
+    }
+    std::sort(cost.begin(), cost.end(), std::greater<int64_t>());
+    std::priority_queue<int64_t, std::vector<int64_t>, std::greater<int64_t>> sm;
+    for (int i = 0; i < segattn::kSmCount; ++i) sm.push(0);
+    int64_t span_max = 0;
+    for (int64_t c : cost) {
+      const int64_t t = sm.top() + c;
+      sm.pop();
+      sm.push(t);
+      span_max = std::max(span_max, t);
+    }
+    return span_max;
+  };
+  int best_f = 1;
+  int64_t best = makespan(1);
+  for (int f = 2; f <= max_split; ++f) {
+    const int64_t m = makespan(f);
+    if (m * 100 < best * 98) {
+      best = m;
+      best_f = f;
+    }
+  }
+  out.citem.assign(items.size(), -1);
+  for (size_t i = 0; i < items.size(); ++i) {
+    const PItem& it = items[i];
+    const int p = pieces_of(it.tiles, best_f);
+    const bool slotted = p > 1 || it.cascade;
+    const int32_t slot0 = slotted ? out.slots : -1;
+    if (slotted) out.slots += p;
+    if (it.cascade) {
+      out.citem[i] = (int32_t)citems.size();
+      citems.push_back({slot0, p, it.q0, 0});
+    } else if (p > 1) {
+      out.merge.push_back({it.r, it.g, it.q0, slot0, p, 0, 0, 0});
+    }
+    for (int j = 0; j < p; ++j) {
+      const int32_t kt0 = (int32_t)((int64_t)it.tiles * j / p);
+      const int32_t kt1 = (int32_t)((int64_t)it.tiles * (j + 1) / p);
+      out.work.push_back({it.r, it.g, it.q0, kt0, kt1, slotted ? slot0 + j : -1, 0, 0});
+    }
+  }
+  // longest first; stable keeps (request, query tile, head, piece) order among equals
+  std::stable_sort(out.work.begin(), out.work.end(), [](const Row8& a, const Row8& b) {
+    return a[4] - a[3] > b[4] - b[3];
+  });
+}
+
+// Cut the batch into groups of consecutive requests that share a prefix.
+// A group [j, i) shares P = min(common prefix of neighbours, cap of each
+// member) keys; it saves, per kv head, the K tiles of P that its members would
+// have read separately (once per 256-row item each) minus those read once per
+// item of the group's packed queries.  Dynamic programme over group ends for
+// the largest total saving; on ties the larger last group wins (fewer groups).
+std::vector<int32_t> choose_groups(const std::vector<Segs>& segs, const std::vector<int32_t>& ql,
+                                   const std::vector<int64_t>& cap, int64_t span,
+                                   std::vector<int64_t>& shared_keys) {
+  const int B = (int)segs.size();
+  std::vector<int64_t> lcp(B, 0);
+  for (int r = 1; r < B; ++r) lcp[r] = common_prefix(segs[r - 1], segs[r]);
+  auto reads = [&](int64_t q) { return (q + span - 1) / span; };
+  std::vector<int64_t> best(B + 1, 0);
+  std::vector<int32_t> from(B + 1, 0);
+  for (int i = 1; i <= B; ++i) {
+    best[i] = best[i - 1];
+    from[i] = i - 1;
+    int64_t P = cap[i - 1], sum_q = ql[i - 1], sep = reads(ql[i - 1]);
+    for (int j = i - 2; j >= 0; --j) {
+      P = std::min({P, lcp[j + 1], cap[j]});
+      if (P < segattn::kMinSharedKeys) break;
+      sum_q += ql[j];
+      sep += reads(ql[j]);
+      const int64_t tiles = (P + segattn::kTileKeys - 1) / segattn::kTileKeys;
+      const int64_t save = (sep - reads(sum_q)) * tiles;
+      if (save > 0 && best[j] + save >= best[i]) {
+        best[i] = best[j] + save;
+        from[i] = j;
+      }
+    }
+  }
+  std::vector<int32_t> starts;  // first request of each group, then B
+  for (int i = B; i > 0; i = from[i]) starts.push_back(from[i]);
+  std::reverse(starts.begin(), starts.end());
+  starts.push_back(B);
+  shared_keys.assign(starts.size() - 1, 0);
+  for (size_t p = 0; p + 1 < starts.size(); ++p) {
+    const int j = starts[p], i = starts[p + 1];
+    if (i - j < 2) continue;
+    int64_t P = cap[j];
+    for (int r = j + 1; r < i; ++r) P = std::min({P, lcp[r], cap[r]});
+    shared_keys[p] = P;
+  }
+  return starts;
+}
+
 }  // namespace
 
 extern "C" int seg_attn_build_table(int batch, const int32_t* q_lens, const int32_t* seg_counts,
                                     const int32_t* seg_starts, const int32_t* seg_lens,
-                                    int64_t num_slots, int causal, int mode, int q_heads,
+                                    int64_t num_slots, int causal, int mode_flags, int q_heads,
                                     int kv_heads, int head_dim, void* host_out,
                                     size_t host_out_bytes, seg_attn_table_desc* desc) {
   if (!desc) return SEG_ATTN_ERR_INVALID_ARG;
   memset(desc, 0, sizeof(*desc));
+  if ((mode_flags & ~(SEG_ATTN_SHARE_PREFIX | 0xff)) != 0) return SEG_ATTN_ERR_INVALID_ARG;
+  const int mode = mode_flags & 0xff;
+  const bool want_share = (mode_flags & SEG_ATTN_SHARE_PREFIX) != 0;
   if (batch < 0 || (mode != SEG_ATTN_MODE_PREFILL && mode != SEG_ATTN_MODE_DECODE) ||
       (causal != 0 && causal != 1) || num_slots < 0)
     return SEG_ATTN_ERR_INVALID_ARG;
@@ -67,16 +246,17 @@ extern "C" int seg_attn_build_table(int batch, const int32_t* q_lens, const int3
   if (num_slots * (int64_t)kv_heads > (int64_t)std::numeric_limits<int32_t>::max())
     return SEG_ATTN_ERR_UNSUPPORTED;
 
-  int64_t nseg = 0;
+  int64_t nseg_in = 0;
   for (int r = 0; r < batch; ++r) {
     if (seg_counts[r] < 0) return SEG_ATTN_ERR_INVALID_ARG;
-    nseg += seg_counts[r];
+    nseg_in += seg_counts[r];
   }
-  if (nseg > std::numeric_limits<int32_t>::max()) return SEG_ATTN_ERR_UNSUPPORTED;
-  if (nseg > 0 && (!seg_starts || !seg_lens)) return SEG_ATTN_ERR_INVALID_ARG;
+  if (nseg_in > std::numeric_limits<int32_t>::max()) return SEG_ATTN_ERR_UNSUPPORTED;
+  if (nseg_in > 0 && (!seg_starts || !seg_lens)) return SEG_ATTN_ERR_INVALID_ARG;
 
   const int32_t kI32Max = std::numeric_limits<int32_t>::max();
   std::vector<int32_t> ql(batch), kl(batch);
+  std::vector<Segs> segs(batch);
   int64_t total_q = 0, total_k = 0;
   {
     int64_t s0 = 0;
@@ -93,6 +273,8 @@ extern "C" int seg_attn_build_table(int batch, const int32_t* q_lens, const int3
         if (st < 0 || st + ln > num_slots) return SEG_ATTN_ERR_SEGMENT_OOB;
         k += ln;
         if (ln > 0) runs.emplace_back(st, ln);
+        segs[r].start.push_back((int32_t)st);
+        segs[r].len.push_back((int32_t)ln);
       }
       std::sort(runs.begin(), runs.end());
       for (size_t i = 1; i < runs.size(); ++i)
@@ -108,88 +290,65 @@ extern "C" int seg_attn_build_table(int batch, const int32_t* q_lens, const int3
     }
   }
   if (total_q > kI32Max) return SEG_ATTN_ERR_UNSUPPORTED;
+  const int32_t qpt = segattn::kTileRows / group;  // queries per 128-row tile
+  const int64_t span = (int64_t)qpt * segattn::kTilesPerItem;
 
-  // ---- work plan
-  std::vector<int4> work;                      // decode chunks
-  std::vector<std::array<int32_t, 8>> pwork;   // prefill pieces
-  std::vector<std::array<int32_t, 8>> pmerge;  // prefill items split over several pieces
-  std::vector<int32_t> req_chunks;
-  int32_t queries_per_tile = 0, chunk_len = 0, max_k_tiles = 0, part_slots = 0;
+  // ---- shared prefixes: groups of consecutive requests, each request's own keys
+  std::vector<int32_t> gstart;   // first request of each group, then batch
+  std::vector<int64_t> gkeys;    // shared keys of each group
+  std::vector<int32_t> req_group(batch, -1);
+  std::vector<int64_t> pre(batch, 0);  // keys request r takes from its group's prefix
+  bool shared = false;
+  if (want_share && batch > 1) {
+    std::vector<int64_t> cap(batch);
+    for (int r = 0; r < batch; ++r)
+      cap[r] = (mode == SEG_ATTN_MODE_PREFILL && causal) ? (int64_t)kl[r] - ql[r] : kl[r];
+    gstart = choose_groups(segs, ql, cap, span, gkeys);
+    for (size_t p = 0; p + 1 < gstart.size(); ++p)
+      for (int r = gstart[p]; r < gstart[p + 1]; ++r) {
+        req_group[r] = (int32_t)p;
+        pre[r] = gkeys[p];
+        shared |= gkeys[p] > 0;
+      }
+  }
+  // the arrays of the main pass describe each request's keys after its shared prefix
+  std::vector<Segs> own(batch);
+  std::vector<int32_t> okl(batch);
+  for (int r = 0; r < batch; ++r) {
+    own[r] = shared && pre[r] > 0 ? cut(segs[r], pre[r], (int64_t)kl[r] - pre[r]) : segs[r];
+    okl[r] = (int32_t)(kl[r] - pre[r]);
+  }
+  int64_t nseg = 0;
+  for (int r = 0; r < batch; ++r) nseg += (int64_t)own[r].len.size();
+  auto in_shared_group = [&](int r) { return shared && pre[r] > 0; };
+
+  // ---- work plan of the main pass
+  std::vector<int4> work;  // decode chunks
+  Pieces main_pieces, group_pieces;
+  std::vector<Row4> citems;
+  std::vector<int32_t> req_chunks, main_citem;  // main_citem: first cascade item of (r, q0 block)
+  int32_t chunk_len = 0, max_k_tiles = 0;
+  std::vector<int64_t> main_item_base(batch, -1);
   if (mode == SEG_ATTN_MODE_PREFILL) {
-    queries_per_tile = segattn::kTileRows / group;
-    const int32_t span = queries_per_tile * segattn::kTilesPerItem;
-    struct Item { int32_t r, g, q0, tiles; };
-    std::vector<Item> items;
+    std::vector<PItem> items;
     for (int r = 0; r < batch; ++r) {
-      const int64_t prior = (int64_t)kl[r] - ql[r];
-      for (int32_t q0 = 0; q0 < ql[r]; q0 += span) {
+      const int64_t prior = (int64_t)okl[r] - ql[r];
+      main_item_base[r] = (int64_t)items.size();
+      for (int32_t q0 = 0; q0 < ql[r]; q0 += (int32_t)span) {
         const int64_t q_end = std::min<int64_t>(ql[r], (int64_t)q0 + span);
-        const int64_t visible = causal ? std::min<int64_t>(kl[r], prior + q_end) : kl[r];
+        const int64_t visible = causal ? std::min<int64_t>(okl[r], prior + q_end) : okl[r];
         const int32_t tiles = (int32_t)((visible + segattn::kTileKeys - 1) / segattn::kTileKeys);
-        for (int g = 0; g < kv_heads; ++g) items.push_back({r, g, q0, tiles});
+        for (int g = 0; g < kv_heads; ++g) items.push_back({r, g, q0, tiles, in_shared_group(r)});
         max_k_tiles = std::max(max_k_tiles, tiles);
       }
     }
-    // Each CTA runs one piece (a contiguous range of an item's K tiles).  Pick how
-    // far to split long items by simulating the longest-first assignment of pieces
-    // to the SMs (what the block scheduler does with a grid in that order) and
-    // keeping the factor with the shortest makespan; ties keep fewer splits.
-    auto pieces_of = [](int32_t tiles, int f) {
-      if (f <= 1 || tiles < 2 * segattn::kMinPieceTiles) return 1;
-      return std::min(f, tiles / segattn::kMinPieceTiles);
-    };
-    auto makespan = [&](int f) {
-      std::vector<int64_t> cost;
-      for (const Item& it : items) {
-        const int p = pieces_of(it.tiles, f);
-        for (int j = 0; j < p; ++j)
-          cost.push_back((int64_t)it.tiles * (j + 1) / p - (int64_t)it.tiles * j / p +
-                         segattn::kPieceOverheadTiles);
-      }
-      std::sort(cost.begin(), cost.end(), std::greater<int64_t>());
-      std::priority_queue<int64_t, std::vector<int64_t>, std::greater<int64_t>> sm;
-      for (int i = 0; i < segattn::kSmCount; ++i) sm.push(0);
-      int64_t span_max = 0;
-      for (int64_t c : cost) {
-        const int64_t t = sm.top() + c;
-        sm.pop();
-        sm.push(t);
-        span_max = std::max(span_max, t);
-      }
-      return span_max;
-    };
-    int best_f = 1;
-    int64_t best = makespan(1);
-    for (int f = 2; f <= segattn::kMaxSplit; ++f) {
-      const int64_t m = makespan(f);
-      if (m * 100 < best * 98) {
-        best = m;
-        best_f = f;
-      }
-    }
-    for (const Item& it : items) {
-      const int p = pieces_of(it.tiles, best_f);
-      const int32_t slot0 = p > 1 ? part_slots : -1;
-      if (p > 1) {
-        pmerge.push_back({it.r, it.g, it.q0, slot0, p, 0, 0, 0});
-        part_slots += p;
-      }
-      for (int j = 0; j < p; ++j) {
-        const int32_t kt0 = (int32_t)((int64_t)it.tiles * j / p);
-        const int32_t kt1 = (int32_t)((int64_t)it.tiles * (j + 1) / p);
-        pwork.push_back({it.r, it.g, it.q0, kt0, kt1, p > 1 ? slot0 + j : -1, 0, 0});
-      }
-    }
-    // longest first; stable keeps (request, query tile, head, piece) order among equals
-    std::stable_sort(pwork.begin(), pwork.end(),
-                     [](const std::array<int32_t, 8>& a, const std::array<int32_t, 8>& b) {
-                       return a[4] - a[3] > b[4] - b[3];
-                     });
+    plan_pieces(items, segattn::kMaxSplit, citems, main_pieces);
+    main_citem = main_pieces.citem;
   } else {
     int64_t L = 2048;
     auto ctas = [&](int64_t len) {
       int64_t n = 0;
-      for (int r = 0; r < batch; ++r) n += std::max<int64_t>(1, (kl[r] + len - 1) / len);
+      for (int r = 0; r < batch; ++r) n += std::max<int64_t>(1, (okl[r] + len - 1) / len);
       return n * kv_heads;
     };
     while (L > 256 && ctas(L) < 4 * segattn::kSmCount) L /= 2;
@@ -197,17 +356,75 @@ extern "C" int seg_attn_build_table(int batch, const int32_t* q_lens, const int3
     req_chunks.resize(batch + 1);
     req_chunks[0] = 0;
     for (int r = 0; r < batch; ++r) {
-      const int32_t n = (int32_t)std::max<int64_t>(1, (kl[r] + L - 1) / L);
+      const int32_t n = (int32_t)std::max<int64_t>(1, (okl[r] + L - 1) / L);
       for (int32_t c = 0; c < n; ++c) {
         const int32_t kb = (int32_t)(c * L);
-        const int32_t ke = (int32_t)std::min<int64_t>(kl[r], (int64_t)(c + 1) * L);
-        work.push_back(make_int4(r, kb, ke, n));
+        const int32_t ke = (int32_t)std::min<int64_t>(okl[r], (int64_t)(c + 1) * L);
+        // chunk count 0 marks a request whose result the cascade merge completes
+        work.push_back(make_int4(r, kb, ke, in_shared_group(r) ? 0 : n));
       }
       req_chunks[r + 1] = req_chunks[r] + n;
     }
   }
-  const size_t n_work = mode == SEG_ATTN_MODE_PREFILL ? pwork.size() : work.size();
+  const size_t n_work = mode == SEG_ATTN_MODE_PREFILL ? main_pieces.work.size() : work.size();
   if (n_work > (size_t)kI32Max) return SEG_ATTN_ERR_UNSUPPORTED;
+
+  // ---- shared-prefix pass and cascade rows
+  std::vector<int32_t> gq_off, greq;      // per group: first query row, first request
+  std::vector<Segs> gsegs;
+  std::vector<int64_t> group_item_base;   // first item of each group's prefix pass
+  std::vector<Row8> cascade;
+  int64_t group_total_k = 0, ngseg = 0;
+  if (shared) {
+    const int ng = (int)gstart.size() - 1;
+    gq_off.assign(ng + 1, 0);
+    greq.assign(gstart.begin(), gstart.end());
+    gsegs.resize(ng);
+    group_item_base.assign(ng, -1);
+    std::vector<int64_t> q_off(batch + 1, 0);
+    for (int r = 0; r < batch; ++r) q_off[r + 1] = q_off[r] + ql[r];
+    std::vector<PItem> items;
+    for (int p = 0; p < ng; ++p) {
+      gq_off[p] = (int32_t)q_off[gstart[p]];
+      const int64_t gq = q_off[gstart[p + 1]] - q_off[gstart[p]];
+      if (gkeys[p] > 0) {
+        gsegs[p] = cut(segs[gstart[p]], 0, gkeys[p]);
+        group_total_k += gkeys[p];
+        group_item_base[p] = (int64_t)items.size();
+        const int32_t tiles = (int32_t)((gkeys[p] + segattn::kTileKeys - 1) / segattn::kTileKeys);
+        for (int32_t q0 = 0; q0 < gq; q0 += (int32_t)span)
+          for (int g = 0; g < kv_heads; ++g) items.push_back({p, g, q0, tiles, true});
+      }
+      ngseg += (int64_t)gsegs[p].len.size();
+    }
+    gq_off[ng] = (int32_t)total_q;
+    // the prefix passes are short and few: allow more pieces so they fill the SMs
+    plan_pieces(items, segattn::kMaxGroupSplit, citems, group_pieces);
+    if (group_pieces.work.size() > (size_t)kI32Max) return SEG_ATTN_ERR_UNSUPPORTED;
+    // rows the cascade merge completes (citem of kv head g = the listed one + g)
+    for (int r = 0; r < batch; ++r) {
+      const int p = req_group[r];
+      const bool pre_r = gkeys[p] > 0;
+      if (mode == SEG_ATTN_MODE_DECODE) {
+        if (!pre_r && req_chunks[r + 1] - req_chunks[r] == 1) continue;
+        int32_t pc = -1, pl = 0;
+        if (pre_r) {
+          pl = (int32_t)(r - gstart[p]);
+          pc = group_pieces.citem[group_item_base[p] + (pl / span) * kv_heads];
+        }
+        cascade.push_back({r, r, pc, pl, -1, 0, 0, 0});
+      } else if (pre_r) {
+        for (int32_t i = 0; i < ql[r]; ++i) {
+          const int64_t row = q_off[r] + i;
+          const int32_t pl = (int32_t)(row - gq_off[p]);
+          const int32_t pc = group_pieces.citem[group_item_base[p] + (pl / span) * kv_heads];
+          const int32_t sc = main_citem[main_item_base[r] + (i / span) * kv_heads];
+          cascade.push_back({(int32_t)row, r, pc, pl, sc, i, 0, 0});
+        }
+      }
+    }
+    if (cascade.size() > (size_t)kI32Max) return SEG_ATTN_ERR_UNSUPPORTED;
+  }
 
   // ---- layout
   Layout lay;
@@ -219,7 +436,18 @@ extern "C" int seg_attn_build_table(int batch, const int32_t* q_lens, const int3
   desc->off_seg_len = lay.take(nseg);
   desc->off_work = lay.take((mode == SEG_ATTN_MODE_PREFILL ? 8 : 4) * (int64_t)n_work);
   desc->off_req_chunks = lay.take(mode == SEG_ATTN_MODE_DECODE ? batch + 1 : 0);
-  desc->off_merge = lay.take(8 * (int64_t)pmerge.size());
+  desc->off_merge = lay.take(8 * (int64_t)main_pieces.merge.size());
+  const int ng = shared ? (int)gstart.size() - 1 : 0;
+  desc->off_group_req = lay.take(shared ? ng + 1 : 0);
+  desc->off_group_q_offsets = lay.take(shared ? ng + 1 : 0);
+  desc->off_group_k_lens = lay.take(ng);
+  desc->off_group_seg_offsets = lay.take(shared ? ng + 1 : 0);
+  desc->off_group_seg_start = lay.take(ngseg);
+  desc->off_group_seg_kstart = lay.take(ngseg);
+  desc->off_group_seg_len = lay.take(ngseg);
+  desc->off_group_work = lay.take(8 * (int64_t)group_pieces.work.size());
+  desc->off_citem = lay.take(4 * (int64_t)citems.size());
+  desc->off_cascade = lay.take(8 * (int64_t)cascade.size());
 
   desc->magic = SEG_ATTN_TABLE_MAGIC;
   desc->version = SEG_ATTN_TABLE_VERSION;
@@ -234,23 +462,26 @@ extern "C" int seg_attn_build_table(int batch, const int32_t* q_lens, const int3
   desc->total_k = total_k;
   desc->num_segments = (int32_t)nseg;
   desc->num_work = (int32_t)n_work;
-  desc->num_merge = (int32_t)pmerge.size();
-  desc->num_parts = part_slots;
-  desc->queries_per_tile = queries_per_tile;
+  desc->num_merge = (int32_t)main_pieces.merge.size();
+  desc->num_parts = main_pieces.slots;
+  desc->shared = shared ? 1 : 0;
+  desc->queries_per_tile = mode == SEG_ATTN_MODE_PREFILL || shared ? qpt : 0;
   desc->chunk_len = chunk_len;
   desc->max_k_tiles = max_k_tiles;
+  desc->num_groups = ng;
+  desc->num_group_segments = (int32_t)ngseg;
+  desc->num_group_work = (int32_t)group_pieces.work.size();
+  desc->num_group_parts = group_pieces.slots;
+  desc->num_citems = (int32_t)citems.size();
+  desc->num_cascade = (int32_t)cascade.size();
+  desc->group_total_k = group_total_k;
   desc->table_bytes = (uint64_t)lay.n * sizeof(int32_t);
-  desc->workspace_bytes = 0;
-  if (mode == SEG_ATTN_MODE_PREFILL && part_slots > 0)
-    desc->workspace_bytes = segattn::prefill_part_o_bytes(part_slots, head_dim) +
-                            align_up((size_t)part_slots * segattn::kItemRows * sizeof(float), 256);
-  if (mode == SEG_ATTN_MODE_DECODE) {
-    bool multi = false;
-    for (int r = 0; r < batch; ++r) multi |= (req_chunks[r + 1] - req_chunks[r]) > 1;
-    if (multi)
-      desc->workspace_bytes = segattn::decode_part_o_bytes(*desc) +
-                              align_up((size_t)desc->num_work * q_heads * sizeof(float), 256);
-  }
+  desc->workspace_bytes = segattn::workspace_layout(*desc, [&] {
+    if (mode != SEG_ATTN_MODE_DECODE) return false;
+    for (int r = 0; r < batch; ++r)
+      if (req_chunks[r + 1] - req_chunks[r] > 1) return true;
+    return false;
+  }()).total;
 
   if (!host_out) return SEG_ATTN_OK;  // size query
   if (host_out_bytes < desc->table_bytes) return SEG_ATTN_ERR_BUFFER_TOO_SMALL;
@@ -258,38 +489,51 @@ extern "C" int seg_attn_build_table(int batch, const int32_t* q_lens, const int3
 
   int32_t* t = static_cast<int32_t*>(host_out);
   memset(t, 0, desc->table_bytes);
+  auto write_csr = [&](const std::vector<Segs>& lists, int32_t* s_off, int32_t* s_start,
+                       int32_t* s_kstart, int32_t* s_len) {
+    int32_t s0 = 0;
+    s_off[0] = 0;
+    for (size_t r = 0; r < lists.size(); ++r) {
+      int32_t logical = 0;
+      for (size_t s = 0; s < lists[r].len.size(); ++s, ++s0) {
+        s_start[s0] = lists[r].start[s];
+        s_len[s0] = lists[r].len[s];
+        s_kstart[s0] = logical;
+        logical += lists[r].len[s];
+      }
+      s_off[r + 1] = s0;
+    }
+  };
   int32_t* q_off = t + desc->off_q_offsets;
   int32_t* k_len = t + desc->off_k_lens;
-  int32_t* s_off = t + desc->off_seg_offsets;
-  int32_t* s_start = t + desc->off_seg_start;
-  int32_t* s_kstart = t + desc->off_seg_kstart;
-  int32_t* s_len = t + desc->off_seg_len;
   q_off[0] = 0;
-  s_off[0] = 0;
-  int64_t s0 = 0;
   for (int r = 0; r < batch; ++r) {
     q_off[r + 1] = q_off[r] + ql[r];
-    k_len[r] = kl[r];
-    s_off[r + 1] = (int32_t)(s0 + seg_counts[r]);
-    int32_t logical = 0;
-    for (int s = 0; s < seg_counts[r]; ++s) {
-      s_start[s0 + s] = seg_starts[s0 + s];
-      s_len[s0 + s] = seg_lens[s0 + s];
-      s_kstart[s0 + s] = logical;
-      logical += seg_lens[s0 + s];
-    }
-    s0 += seg_counts[r];
+    k_len[r] = okl[r];
   }
+  write_csr(own, t + desc->off_seg_offsets, t + desc->off_seg_start, t + desc->off_seg_kstart,
+            t + desc->off_seg_len);
+  auto put_rows = [&](int64_t off, const auto& rows) {
+    for (size_t i = 0; i < rows.size(); ++i)
+      memcpy(t + off + rows[i].size() * i, rows[i].data(), rows[i].size() * sizeof(int32_t));
+  };
   if (mode == SEG_ATTN_MODE_PREFILL) {
-    for (size_t i = 0; i < pwork.size(); ++i)
-      memcpy(t + desc->off_work + 8 * i, pwork[i].data(), 8 * sizeof(int32_t));
-    for (size_t i = 0; i < pmerge.size(); ++i)
-      memcpy(t + desc->off_merge + 8 * i, pmerge[i].data(), 8 * sizeof(int32_t));
-  } else if (!work.empty()) {
-    memcpy(t + desc->off_work, work.data(), work.size() * sizeof(int4));
-  }
-  if (mode == SEG_ATTN_MODE_DECODE)
+    put_rows(desc->off_work, main_pieces.work);
+    put_rows(desc->off_merge, main_pieces.merge);
+  } else {
+    if (!work.empty()) memcpy(t + desc->off_work, work.data(), work.size() * sizeof(int4));
     memcpy(t + desc->off_req_chunks, req_chunks.data(), req_chunks.size() * sizeof(int32_t));
+  }
+  if (shared) {
+    memcpy(t + desc->off_group_req, greq.data(), greq.size() * sizeof(int32_t));
+    memcpy(t + desc->off_group_q_offsets, gq_off.data(), gq_off.size() * sizeof(int32_t));
+    for (int p = 0; p < ng; ++p) t[desc->off_group_k_lens + p] = (int32_t)gkeys[p];
+    write_csr(gsegs, t + desc->off_group_seg_offsets, t + desc->off_group_seg_start,
+              t + desc->off_group_seg_kstart, t + desc->off_group_seg_len);
+    put_rows(desc->off_group_work, group_pieces.work);
+    put_rows(desc->off_citem, citems);
+    put_rows(desc->off_cascade, cascade);
+  }
   return SEG_ATTN_OK;
 }
 
@@ -297,7 +541,6 @@ extern "C" size_t seg_attn_workspace_size(const seg_attn_table_desc* desc) {
   if (!desc || desc->magic != SEG_ATTN_TABLE_MAGIC) return 0;
   return (size_t)desc->workspace_bytes;
 }
-
 extern "C" const char* seg_attn_status_string(int status) {
   switch (status) {
     case SEG_ATTN_OK: return "ok";

@@ -35,6 +35,8 @@ CONFIG_NAMES = {
     3: "chunked prefill varlen (16 req, 2048 new tokens, prior 0-8192)",
     4: "batched decode (128 req, k 1024-32768)",
     5: "long-context mix (8 decode at k=131072 + 1 prefill chunk 2048 over 131072)",
+    6: "shared-prefix decode (8 groups x 8 req, prefix 8192-32768 + own 512-4096)",
+    7: "shared-prefix chunked prefill (4 groups x 8 req, prefix 4096-16384, chunks 4-32)",
 }
 
 
@@ -173,26 +175,84 @@ def _structure(cfg: int, gen: torch.Generator, context_scale: float = 1.0):
         return dict(q_heads=64, kv_heads=8, head_dim=128, num_slots=slots,
                     batches=[("decode", [1] * 8, lens_all[:8], True),
                              ("prefill", [2048], lens_all[8:], True)], qk_std=0.5)
+    if cfg in (6, 7):
+        return _shared_structure(cfg, gen)
     raise ValueError(f"unknown config {cfg}")
+
+
+def _shared_structure(cfg: int, gen: torch.Generator):
+    """Requests in groups of consecutive requests that share a prefix (prefix caching):
+    every member's segment list starts with the group's prefix segments (the same
+    slots), then lists its own segments.
+      6: decode, 8 groups x 8 requests; prefix U{8192..32768} keys in U{1..4}
+         segments; each request's own keys U{512..4096} in U{1..4} segments.
+      7: causal chunked prefill, 4 groups x 8 requests; prefix U{4096..16384} in
+         U{1..4} segments; each request's own prior context U{0..1024} plus a new
+         chunk of U{4..32} queries (short chunks: multi-token verification, short
+         turns), in U{1..3} segments.
+    Draw order: per group the prefix length, its segment count and cuts, then per
+    member its own lengths, segment count and cuts."""
+    groups, members = (8, 8) if cfg == 6 else (4, 8)
+    unique, q_lens, seg_ids = [], [], []
+    for _ in range(groups):
+        if cfg == 6:
+            P = int(torch.randint(8192, 32769, (1,), generator=gen))
+        else:
+            P = int(torch.randint(4096, 16385, (1,), generator=gen))
+        n = int(torch.randint(1, 5, (1,), generator=gen))
+        prefix_ids = []
+        for ln in split_uniform_cuts(P, n, gen):
+            prefix_ids.append(len(unique))
+            unique.append(ln)
+        for _ in range(members):
+            if cfg == 6:
+                q, own = 1, int(torch.randint(512, 4097, (1,), generator=gen))
+                n_own = int(torch.randint(1, 5, (1,), generator=gen))
+            else:
+                prior = int(torch.randint(0, 1025, (1,), generator=gen))
+                q = int(torch.randint(4, 33, (1,), generator=gen))
+                own = prior + q
+                n_own = int(torch.randint(1, 4, (1,), generator=gen))
+            ids = list(prefix_ids)
+            for ln in split_uniform_cuts(own, n_own, gen):
+                ids.append(len(unique))
+                unique.append(ln)
+            q_lens.append(q)
+            seg_ids.append(ids)
+    slots = math.ceil(1.1 * sum(unique))
+    mode = "decode" if cfg == 6 else "prefill"
+    return dict(q_heads=64, kv_heads=8, head_dim=128, num_slots=slots, unique=unique,
+                batches=[(mode, q_lens, seg_ids, True)], qk_std=1.0)
 
 
 def make_workload(cfg: int, device: str = "cpu", values: bool = True,
                   seed: Optional[int] = None, context_scale: float = 1.0) -> Workload:
-    """Build config ``cfg`` (1..5).  Seed defaults to cfg - 1."""
+    """Build config ``cfg`` (1..7).  Seed defaults to cfg - 1."""
     seed = cfg - 1 if seed is None else seed
     gen = torch.Generator(device="cpu").manual_seed(seed)
     st = _structure(cfg, gen, context_scale)
     batches = []
-    all_lens = []
-    for mode, q_lens, seg_lens, causal in st["batches"]:
-        batches.append(Batch(mode=mode, q_lens=list(q_lens), seg_starts=[], seg_lens=seg_lens,
-                             causal=causal))
-        for s in seg_lens:
-            all_lens.extend(s)
-    starts = place_segments(all_lens, st["num_slots"], gen)
-    it = iter(starts)
-    for b in batches:
-        b.seg_starts = [[next(it) for _ in s] for s in b.seg_lens]
+    if "unique" in st:
+        # segments listed by id into one list of distinct segments (shared prefixes)
+        unique = st["unique"]
+        for mode, q_lens, seg_ids, causal in st["batches"]:
+            batches.append(Batch(mode=mode, q_lens=list(q_lens), seg_starts=[],
+                                 seg_lens=[[unique[i] for i in ids] for ids in seg_ids],
+                                 causal=causal))
+        starts = place_segments(unique, st["num_slots"], gen)
+        for b, (_, _, seg_ids, _) in zip(batches, st["batches"]):
+            b.seg_starts = [[starts[i] for i in ids] for ids in seg_ids]
+    else:
+        all_lens = []
+        for mode, q_lens, seg_lens, causal in st["batches"]:
+            batches.append(Batch(mode=mode, q_lens=list(q_lens), seg_starts=[],
+                                 seg_lens=seg_lens, causal=causal))
+            for s in seg_lens:
+                all_lens.extend(s)
+        starts = place_segments(all_lens, st["num_slots"], gen)
+        it = iter(starts)
+        for b in batches:
+            b.seg_starts = [[next(it) for _ in s] for s in b.seg_lens]
     live = torch.zeros(st["num_slots"], dtype=torch.bool)
     for b in batches:
         for ss, ll in zip(b.seg_starts, b.seg_lens):

@@ -2,6 +2,7 @@
 from __future__ import annotations
 
 import math
+import random
 
 import numpy as np
 import torch
@@ -27,7 +28,7 @@ def run_cuda(q, k_pool, v_pool, q_lens, seg_starts, seg_lens, num_slots, causal,
     ws = None
     if tab.workspace_bytes:
         ws = torch.empty(tab.workspace_bytes, dtype=torch.uint8, device=q.device)
-    fn = sa.seg_attn_prefill if mode == sa.MODE_PREFILL else sa.seg_attn_decode
+    fn = sa.seg_attn_prefill if (mode & 0xff) == sa.MODE_PREFILL else sa.seg_attn_decode
     fn(q, k_pool, v_pool, out, lse, tab.device, tab.desc, scale, ws, stream)
     return out, lse, tab
 
@@ -115,3 +116,71 @@ def random_case(seed, batch, hq, hkv, d, causal, max_k, nseg_max=4, q_mode="chun
             v[s:s + l] = torch.randn(l, hkv, d, generator=g).to(torch.bfloat16)
     return dict(q_lens=q_lens, seg_starts=seg_starts, seg_lens=seg_lens, q=q, k_pool=k, v_pool=v,
                 num_slots=slots, scale=1.0 / math.sqrt(d), causal=causal)
+
+
+def slots_of(starts, lens):
+    return [s + t for s, l in zip(starts, lens) for t in range(l)]
+
+
+def shared_case(seed, B, decode, max_prefix=1200):
+    """Requests drawn from a few prefix trees: each shares a random-length prefix with
+    its predecessor (sometimes re-cut into other segments), then has its own keys."""
+    rnd = random.Random(seed)
+    pool_next = [0]
+
+    def fresh(n):
+        s = pool_next[0] + rnd.randint(0, 5)
+        pool_next[0] = s + n
+        return (s, n)
+
+    reqs = []
+    prev = None
+    for r in range(B):
+        segs = []
+        if prev is not None and rnd.random() < 0.75:
+            # take a prefix of the previous request's slots, maybe cut differently
+            ps = slots_of(*prev)
+            take = rnd.randint(0, len(ps))
+            run_start, run_len = None, 0
+            for x in ps[:take]:
+                if run_start is not None and x == run_start + run_len and rnd.random() < 0.97:
+                    run_len += 1
+                else:
+                    if run_start is not None:
+                        segs.append((run_start, run_len))
+                    run_start, run_len = x, 1
+            if run_start is not None:
+                segs.append((run_start, run_len))
+        else:
+            segs.append(fresh(rnd.randint(0, max_prefix)))
+        for _ in range(rnd.randint(0 if segs else 1, 3)):
+            segs.append(fresh(rnd.randint(1, 300)))
+        segs = [s for s in segs if s[1] > 0] or [fresh(1)]
+        starts, lens = [s for s, _ in segs], [l for _, l in segs]
+        reqs.append((starts, lens))
+        prev = (starts, lens)
+    k = [sum(l) for _, l in reqs]
+    if decode:
+        q = [1] * B
+    else:
+        q = [rnd.randint(0, min(kk, 40)) for kk in k]
+    return reqs, q, pool_next[0] + 10
+
+
+def shared_values(reqs, q_lens, num_slots, hq, hkv, d, seed, device="cuda"):
+    """Q and pools for a shared_case: the slots any request uses get N(0,1) bf16 values,
+    every other slot NaN (drawn on the CPU)."""
+    g = torch.Generator().manual_seed(seed)
+    live = torch.zeros(num_slots, dtype=torch.bool)
+    for starts, lens in reqs:
+        for s, l in zip(starts, lens):
+            live[s:s + l] = True
+    k = torch.full((num_slots, hkv, d), float("nan"))
+    v = torch.full((num_slots, hkv, d), float("nan"))
+    n = int(live.sum())
+    k[live] = torch.randn(n, hkv, d, generator=g)
+    v[live] = torch.randn(n, hkv, d, generator=g)
+    q = torch.randn(sum(q_lens), hq, d, generator=g)
+    return dict(q=q.to(torch.bfloat16), k_pool=k.to(torch.bfloat16), v_pool=v.to(torch.bfloat16),
+                q_lens=list(q_lens), seg_starts=[s for s, _ in reqs],
+                seg_lens=[l for _, l in reqs], num_slots=num_slots, scale=1.0 / math.sqrt(d))

@@ -117,6 +117,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tok0 = __ldg(p.tab.q_offsets + req);
   const int q_len = __ldg(p.tab.q_offsets + req + 1) - tok0;
   const int k_len = __ldg(p.tab.k_lens + req);
+  // Only query tile 0 holds queries (a short chunk, or the packed queries of a
+  // small shared-prefix group): tile 1 is skipped and its S columns become a
+  // second S buffer of tile 0, so the next tile's S = QK^T overlaps this tile's
+  // softmax.  Uniform over the CTA.
+  const bool single = q_len - q0 <= p.qpt;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -151,8 +156,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     int k_issued = 0, v_issued = 0;
     if (n_tiles > 0) {
       if (lane == 0) {
-        mbar_expect_tx(q_full, 2 * TILE);
-        for (int t = 0; t < 2; ++t)
+        const int q_tiles = single ? 1 : 2;
+        mbar_expect_tx(q_full, q_tiles * TILE);
+        for (int t = 0; t < q_tiles; ++t)
           for (int h = 0; h < HALVES; ++h)
             tma_load_3d(sQ + t * TILE + h * kHalfBytes, &tm_q, q_full, 64 * h, g * p.group,
                         tok0 + q0 + t * p.qpt);
@@ -221,57 +227,94 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
       const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
       const uint32_t tS0 = tmem + 256, tO0 = tmem;
-      auto issue_qk = [&](int t, int st) {
+      // S buffer `sb` = Q tile `qt` . K stage `st`^T;  O tile `ot` += P (in S buffer `sb`) . V stage `st`
+      auto issue_qk = [&](int qt, int sb, int st) {
 #pragma unroll
         for (int k = 0; k < KSTEPS; ++k) {
           const uint32_t off = (k >> 2) * kHalfBytes + (k & 3) * 32;
-          mma_ss(tS0 + 128 * t, sdesc_sw128(q_addr + t * TILE + off, 16, 1024),
+          mma_ss(tS0 + 128 * sb, sdesc_sw128(q_addr + qt * TILE + off, 16, 1024),
                  sdesc_sw128(k_addr + st * TILE + off, 16, 1024), idesc_qk, k > 0 ? 1u : 0u);
         }
       };
-      auto issue_pv = [&](int t, int st, bool acc) {
+      auto issue_pv = [&](int ot, int sb, int st, bool acc) {
 #pragma unroll
         for (int k = 0; k < kTileKeys / 16; ++k)
-          mma_ts(tO0 + 128 * t, tS0 + 128 * t + 8 * k,
+          mma_ts(tO0 + 128 * ot, tS0 + 128 * sb + 8 * k,
                  sdesc_sw128(v_addr + st * TILE + k * 2048, kHalfBytes, 1024), idesc_pv,
                  (acc || k > 0) ? 1u : 0u);
       };
       bool ok = mbar_wait(q_full, 0, abort_flag, kWaitLimitNs) &&
                 mbar_wait(k_full + 0, 0, abort_flag, kWaitLimitNs);
-      if (ok) {
-        tc_fence_after();
-        issue_qk(0, 0);
-        mma_commit(s_full + 0);
-        issue_qk(1, 0);
-        mma_commit(s_full + 1);
-        mma_commit(k_empty + 0);
-      }
-      for (int i = 0; ok && i < n_tiles; ++i) {
-        const int st = i & 1;
-        const uint32_t ph = (i >> 1) & 1;
-        const bool more = i + 1 < n_tiles;
-        const int st1 = (i + 1) & 1;
-        const uint32_t ph1 = ((i + 1) >> 1) & 1;
-        if (!(ok = mbar_wait(v_full + st, ph, abort_flag, kWaitLimitNs))) break;
-        if (!(ok = mbar_wait(p_full + 0, i & 1, abort_flag, kWaitLimitNs))) break;
-        tc_fence_after();
-        issue_pv(0, st, i > 0);
-        mma_commit(o_full + 0);
-        if (more) {
-          if (!(ok = mbar_wait(k_full + st1, ph1, abort_flag, kWaitLimitNs))) break;
+      if (single) {
+        // one query tile, S double-buffered: K tile i uses S buffer i & 1.  While the
+        // softmax works on buffer i & 1, S of tile i + 1 is already in the other one;
+        // right after PV(i) has read P(i), S of tile i + 2 goes into the freed buffer
+        // (tensor-core operations of one CTA run in issue order).
+        if (ok) {
           tc_fence_after();
-          issue_qk(0, st1);
+          issue_qk(0, 0, 0);
           mma_commit(s_full + 0);
+          mma_commit(k_empty + 0);
         }
-        if (!(ok = mbar_wait(p_full + 1, i & 1, abort_flag, kWaitLimitNs))) break;
-        tc_fence_after();
-        issue_pv(1, st, i > 0);
-        mma_commit(o_full + 1);
-        mma_commit(v_empty + st);
-        if (more) {
-          issue_qk(1, st1);
+        if (ok && n_tiles > 1 && (ok = mbar_wait(k_full + 1, 0, abort_flag, kWaitLimitNs))) {
+          tc_fence_after();
+          issue_qk(0, 1, 1);
           mma_commit(s_full + 1);
-          mma_commit(k_empty + st1);
+          mma_commit(k_empty + 1);
+        }
+        for (int i = 0; ok && i < n_tiles; ++i) {
+          const int b = i & 1;
+          const uint32_t ph = (i >> 1) & 1;
+          if (!(ok = mbar_wait(v_full + b, ph, abort_flag, kWaitLimitNs))) break;
+          if (!(ok = mbar_wait(p_full + b, ph, abort_flag, kWaitLimitNs))) break;
+          tc_fence_after();
+          issue_pv(0, b, b, i > 0);
+          mma_commit(o_full + 0);
+          mma_commit(v_empty + b);
+          if (i + 2 < n_tiles) {
+            if (!(ok = mbar_wait(k_full + b, ph ^ 1, abort_flag, kWaitLimitNs))) break;
+            tc_fence_after();
+            issue_qk(0, b, b);
+            mma_commit(s_full + b);
+            mma_commit(k_empty + b);
+          }
+        }
+      } else {
+        if (ok) {
+          tc_fence_after();
+          issue_qk(0, 0, 0);
+          mma_commit(s_full + 0);
+          issue_qk(1, 1, 0);
+          mma_commit(s_full + 1);
+          mma_commit(k_empty + 0);
+        }
+        for (int i = 0; ok && i < n_tiles; ++i) {
+          const int st = i & 1;
+          const uint32_t ph = (i >> 1) & 1;
+          const bool more = i + 1 < n_tiles;
+          const int st1 = (i + 1) & 1;
+          const uint32_t ph1 = ((i + 1) >> 1) & 1;
+          if (!(ok = mbar_wait(v_full + st, ph, abort_flag, kWaitLimitNs))) break;
+          if (!(ok = mbar_wait(p_full + 0, i & 1, abort_flag, kWaitLimitNs))) break;
+          tc_fence_after();
+          issue_pv(0, 0, st, i > 0);
+          mma_commit(o_full + 0);
+          if (more) {
+            if (!(ok = mbar_wait(k_full + st1, ph1, abort_flag, kWaitLimitNs))) break;
+            tc_fence_after();
+            issue_qk(0, 0, st1);
+            mma_commit(s_full + 0);
+          }
+          if (!(ok = mbar_wait(p_full + 1, i & 1, abort_flag, kWaitLimitNs))) break;
+          tc_fence_after();
+          issue_pv(1, 1, st, i > 0);
+          mma_commit(o_full + 1);
+          mma_commit(v_empty + st);
+          if (more) {
+            issue_qk(1, 1, st1);
+            mma_commit(s_full + 1);
+            mma_commit(k_empty + st1);
+          }
         }
       }
       // all MMAs finished before tensor memory is released
@@ -279,7 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(mma_done, 0, nullptr, kWaitLimitNs);
     }
     __syncwarp();
-  } else {
+  } else if (!single || warp < 6) {
     // ------------------------------------------------------------ softmax + epilogue
     const int t = (warp - 2) >> 2;
     const int quad = warp & 3;
@@ -289,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool row_valid = qi < q_len;
     const int vis = p.causal ? min(k_len, k_len - q_len + qi + 1) : k_len;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-    const uint32_t tS = lane_base + 256 + 128 * t;
+    uint32_t tS = lane_base + 256 + 128 * t;  // S buffer of the current K tile
     const uint32_t tO = lane_base + 128 * t;
     const float sl2 = p.scale_log2;
     float m_ref = -INFINITY;  // raw score units
@@ -371,17 +414,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       return true;
     };
-    for (int i = 0; i < n_tiles; ++i) {
-      if (!(ok = __all_sync(0xffffffffu, mbar_wait(s_full + t, i & 1, abort_flag, kWaitLimitNs))))
-        break;
+    // one K tile of softmax on S buffer sb (phase sph of its barriers)
+    auto run_tile = [&](int i, int sb, uint32_t sph) -> bool {
+      tS = lane_base + 256 + 128 * sb;
+      if (!__all_sync(0xffffffffu, mbar_wait(s_full + sb, sph, abort_flag, kWaitLimitNs)))
+        return false;
       tc_fence_after();
       const bool masked = __any_sync(0xffffffffu, (kt0 + i + 1) * kTileKeys > vis);
       if (masked) mask_tile(i);
-      ok = softmax_tile(i);
-      if (!ok) break;
+      if (!softmax_tile(i)) return false;
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(p_full + t);
+      mbar_arrive(p_full + sb);
+      return true;
+    };
+    if (single) {
+      // S buffers alternate; unrolled by two so each buffer's address is fixed
+      for (int i = 0; ok && i < n_tiles; i += 2) {
+        const uint32_t sph = (i >> 1) & 1;
+        ok = run_tile(i, 0, sph);
+        if (ok && i + 1 < n_tiles) ok = run_tile(i + 1, 1, sph);
+      }
+    } else {
+      for (int i = 0; ok && i < n_tiles; ++i) ok = run_tile(i, t, i & 1);
     }
     if (ok && n_tiles > 0)
       ok = __all_sync(0xffffffffu,

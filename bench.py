@@ -99,10 +99,11 @@ def launches_of(desc):
     """Kernel launches one compute call makes for a built table."""
     shared = desc.shared == 1
     n = 0
-    if shared and desc.num_group_work > 0:
-        n += 1  # pass over the shared prefixes
+    if shared and desc.num_group_work > 0:  # pass over the shared prefixes (two-tile, one-tile)
+        n += (desc.num_group_work > desc.num_group_single) + (desc.num_group_single > 0)
     if desc.mode == sa.MODE_PREFILL:
-        n += (1 if desc.num_work > 0 else 0) + (1 if desc.num_merge > 0 else 0)
+        n += (desc.num_work > desc.num_single) + (desc.num_single > 0)
+        n += 1 if desc.num_merge > 0 else 0
     else:
         n += 1 if desc.num_work > 0 else 0
         n += 1 if (desc.workspace_bytes > 0 and not shared) else 0

@@ -124,6 +124,9 @@ typedef struct seg_attn_table_desc {
   int32_t num_group_parts; /* partial-result slots of those pieces */
   int32_t num_citems;      /* items whose pieces write partials for the cascade merge */
   int32_t num_cascade;     /* output rows (prefill: tokens, decode: requests) merged by it */
+  int32_t num_single;      /* prefill: the last num_single work items hold queries in their
+                              first 128-row tile only (they run a one-tile kernel) */
+  int32_t num_group_single;/* the same for the pieces of the shared-prefix pass */
   int64_t group_total_k;   /* sum of P_p */
   int64_t off_group_req;        /* [num_groups+1] first request of each group */
   int64_t off_group_q_offsets;  /* [num_groups+1] first query (packed row) of each group */

@@ -56,6 +56,7 @@ class seg_attn_table_desc(ctypes.Structure):
         ("num_groups", ctypes.c_int32), ("num_group_segments", ctypes.c_int32),
         ("num_group_work", ctypes.c_int32), ("num_group_parts", ctypes.c_int32),
         ("num_citems", ctypes.c_int32), ("num_cascade", ctypes.c_int32),
+        ("num_single", ctypes.c_int32), ("num_group_single", ctypes.c_int32),
         ("group_total_k", ctypes.c_int64),
         ("off_group_req", ctypes.c_int64), ("off_group_q_offsets", ctypes.c_int64),
         ("off_group_k_lens", ctypes.c_int64), ("off_group_seg_offsets", ctypes.c_int64),

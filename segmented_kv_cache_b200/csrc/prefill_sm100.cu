@@ -64,6 +64,7 @@ struct PrefillParams {
   int q_heads, kv_heads, group, qpt, causal;
   float* part_o;    // split items: [slot][kItemRows][D], O / l of the piece
   float* part_lse;  // split items: [slot][kItemRows], log2 of the piece's sum of exp
+  int work_base;    // first work item of this launch
 };
 
 // Q (2 tiles) + K ring (2) + V ring (2) + barriers + alignment slack.  The
@@ -80,7 +81,10 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-template <int D>
+// SINGLE: every item of the launch has queries in its first query tile only
+// (the planner lists those items last and launches them separately, so each
+// instantiation keeps its own register allocation).
+template <int D, bool SINGLE>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_k3,
@@ -111,7 +115,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // piece: keys tiles [kt0, kt1) of item (request, kv head g, query tiles from q0);
   // slot >= 0 when the item is split and this piece writes a partial result
-  const int4 w0 = p.tab.work[2 * blockIdx.x], w1 = p.tab.work[2 * blockIdx.x + 1];
+  const int item = p.work_base + blockIdx.x;
+  const int4 w0 = p.tab.work[2 * item], w1 = p.tab.work[2 * item + 1];
   const int req = w0.x, g = w0.y, q0 = w0.z, kt0 = w0.w, slot = w1.y;
   const int n_tiles = w1.x - kt0;
   const int tok0 = __ldg(p.tab.q_offsets + req);
@@ -120,8 +125,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Only query tile 0 holds queries (a short chunk, or the packed queries of a
   // small shared-prefix group): tile 1 is skipped and its S columns become a
   // second S buffer of tile 0, so the next tile's S = QK^T overlaps this tile's
-  // softmax.  Uniform over the CTA.
-  const bool single = q_len - q0 <= p.qpt;
+  // softmax.
+  constexpr bool single = SINGLE;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -414,11 +419,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       return true;
     };
+    // A warp whose 32 rows hold no query (past the end of the chunk) only keeps
+    // step with the barriers: its P rows feed only output rows nobody reads.
+    const bool warp_live = __any_sync(0xffffffffu, row_valid);
     // one K tile of softmax on S buffer sb (phase sph of its barriers)
     auto run_tile = [&](int i, int sb, uint32_t sph) -> bool {
       tS = lane_base + 256 + 128 * sb;
       if (!__all_sync(0xffffffffu, mbar_wait(s_full + sb, sph, abort_flag, kWaitLimitNs)))
         return false;
+      if (!warp_live) {
+        mbar_arrive(p_full + sb);
+        return true;
+      }
       tc_fence_after();
       const bool masked = __any_sync(0xffffffffu, (kt0 + i + 1) * kTileKeys > vis);
       if (masked) mask_tile(i);
@@ -438,6 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
       for (int i = 0; ok && i < n_tiles; ++i) ok = run_tile(i, t, i & 1);
     }
+    if (!warp_live) ok = false;  // nothing to write
     if (ok && n_tiles > 0)
       ok = __all_sync(0xffffffffu,
                       mbar_wait(o_full + t, (n_tiles - 1) & 1, abort_flag, kWaitLimitNs));
@@ -618,11 +631,24 @@ int launch_prefill_d(const PrefillLaunch& a, cudaStream_t stream) {
   p.part_o = a.part_o;
   p.part_lse = a.part_lse;
   constexpr size_t smem = prefill_smem_bytes<D>();
-  if (cudaFuncSetAttribute(prefill_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem) != cudaSuccess)
-    return SEG_ATTN_ERR_CUDA;
-  prefill_kernel<D><<<d.num_work, kThreads, smem, stream>>>(tq, tk, tv, tk3, tv3, p);
-  if (cudaGetLastError() != cudaSuccess) return SEG_ATTN_ERR_CUDA;
+  // two-tile items first, then the single-tile items listed at the end
+  const int n_single = d.num_single, n_two = d.num_work - d.num_single;
+  if (n_two > 0) {
+    if (cudaFuncSetAttribute(prefill_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+      return SEG_ATTN_ERR_CUDA;
+    p.work_base = 0;
+    prefill_kernel<D, false><<<n_two, kThreads, smem, stream>>>(tq, tk, tv, tk3, tv3, p);
+    if (cudaGetLastError() != cudaSuccess) return SEG_ATTN_ERR_CUDA;
+  }
+  if (n_single > 0) {
+    if (cudaFuncSetAttribute(prefill_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+      return SEG_ATTN_ERR_CUDA;
+    p.work_base = n_two;
+    prefill_kernel<D, true><<<n_single, kThreads, smem, stream>>>(tq, tk, tv, tk3, tv3, p);
+    if (cudaGetLastError() != cudaSuccess) return SEG_ATTN_ERR_CUDA;
+  }
   if (d.num_merge > 0) {
     prefill_merge_kernel<D><<<dim3(d.num_merge, 4), 256, 0, stream>>>(p);
     if (cudaGetLastError() != cudaSuccess) return SEG_ATTN_ERR_CUDA;

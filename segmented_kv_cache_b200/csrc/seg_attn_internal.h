@@ -18,6 +18,9 @@ constexpr int kPieceOverheadTiles = 2;  // per-piece cost (prologue, epilogue) i
 constexpr int kMaxSplit = 4;            // most pieces one prefill item is cut into
 constexpr int kMaxGroupSplit = 32;      // the same for a pass over a shared prefix
 constexpr int kMinSharedKeys = 256;     // shortest prefix worth a pass of its own
+// decode: key chunks are halved (down to 256 keys) until the grid has this many
+// CTAs -- 4 waves at 2 CTAs per SM, so the last wave's tail stays short
+constexpr int kDecodeTargetCtas = 8 * kSmCount;
 
 // Device views of the table arrays (device pointers into dev_table).
 struct TableView {
@@ -46,6 +49,7 @@ inline seg_attn_table_desc group_pass_desc(const seg_attn_table_desc& d) {
   g.num_work = d.num_group_work;
   g.num_merge = 0;
   g.num_parts = d.num_group_parts;
+  g.num_single = d.num_group_single;
   g.shared = 0;
   g.off_q_offsets = d.off_group_q_offsets;
   g.off_k_lens = d.off_group_k_lens;

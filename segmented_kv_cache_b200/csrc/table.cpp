@@ -94,17 +94,19 @@ Segs cut(const Segs& s, int64_t from, int64_t count) {
 }
 
 // One prefill item: (request, kv head, query tiles from q0) over `tiles` K tiles.
-// `cascade` items write every piece as a partial for the shared-prefix merge.
+// `cascade` items write every piece as a partial for the shared-prefix merge;
+// `single` items hold queries in their first 128-row query tile only.
 struct PItem {
   int32_t r, g, q0, tiles;
-  bool cascade;
+  bool cascade, single;
 };
 
 struct Pieces {
-  std::vector<Row8> work;       // pieces, longest first
+  std::vector<Row8> work;       // two-tile pieces longest first, then single-tile ones
   std::vector<Row8> merge;      // split items that are not cascade items
   std::vector<int32_t> citem;   // per item: its index in `citems`, or -1
   int32_t slots = 0;            // partial-result slots
+  int32_t single = 0;           // single-tile pieces (the tail of `work`)
 };
 
 // Cut items into pieces along their K tiles when that shortens the
@@ -147,9 +149,15 @@ void plan_pieces(const std::vector<PItem>& items, int max_split, std::vector<Row
       best_f = f;
     }
   }
+  // The one-tile kernel runs a pass only when every item of it is single-tile: a
+  // second launch for a few single-tile items would serialise behind the first
+  // launch's tail (those items then run two-tile, their empty tile's softmax skipped).
+  const bool all_single =
+      std::all_of(items.begin(), items.end(), [](const PItem& it) { return it.single; });
   out.citem.assign(items.size(), -1);
   for (size_t i = 0; i < items.size(); ++i) {
-    const PItem& it = items[i];
+    PItem it = items[i];
+    it.single = all_single;
     const int p = pieces_of(it.tiles, best_f);
     const bool slotted = p > 1 || it.cascade;
     const int32_t slot0 = slotted ? out.slots : -1;
@@ -163,11 +171,15 @@ void plan_pieces(const std::vector<PItem>& items, int max_split, std::vector<Row
     for (int j = 0; j < p; ++j) {
       const int32_t kt0 = (int32_t)((int64_t)it.tiles * j / p);
       const int32_t kt1 = (int32_t)((int64_t)it.tiles * (j + 1) / p);
-      out.work.push_back({it.r, it.g, it.q0, kt0, kt1, slotted ? slot0 + j : -1, 0, 0});
+      out.work.push_back({it.r, it.g, it.q0, kt0, kt1, slotted ? slot0 + j : -1,
+                          it.single ? 1 : 0, 0});
+      out.single += it.single ? 1 : 0;
     }
   }
-  // longest first; stable keeps (request, query tile, head, piece) order among equals
+  // two-tile pieces, then single-tile pieces (word 6), each longest first; stable
+  // keeps (request, query tile, head, piece) order among equals
   std::stable_sort(out.work.begin(), out.work.end(), [](const Row8& a, const Row8& b) {
+    if (a[6] != b[6]) return a[6] < b[6];
     return a[4] - a[3] > b[4] - b[3];
   });
 }
@@ -338,7 +350,9 @@ extern "C" int seg_attn_build_table(int batch, const int32_t* q_lens, const int3
         const int64_t q_end = std::min<int64_t>(ql[r], (int64_t)q0 + span);
         const int64_t visible = causal ? std::min<int64_t>(okl[r], prior + q_end) : okl[r];
         const int32_t tiles = (int32_t)((visible + segattn::kTileKeys - 1) / segattn::kTileKeys);
-        for (int g = 0; g < kv_heads; ++g) items.push_back({r, g, q0, tiles, in_shared_group(r)});
+        const bool single = ql[r] - q0 <= qpt;
+        for (int g = 0; g < kv_heads; ++g)
+          items.push_back({r, g, q0, tiles, in_shared_group(r), single});
         max_k_tiles = std::max(max_k_tiles, tiles);
       }
     }
@@ -351,7 +365,7 @@ extern "C" int seg_attn_build_table(int batch, const int32_t* q_lens, const int3
       for (int r = 0; r < batch; ++r) n += std::max<int64_t>(1, (okl[r] + len - 1) / len);
       return n * kv_heads;
     };
-    while (L > 256 && ctas(L) < 4 * segattn::kSmCount) L /= 2;
+    while (L > 256 && ctas(L) < segattn::kDecodeTargetCtas) L /= 2;
     chunk_len = (int32_t)L;
     req_chunks.resize(batch + 1);
     req_chunks[0] = 0;
@@ -393,7 +407,7 @@ extern "C" int seg_attn_build_table(int batch, const int32_t* q_lens, const int3
         group_item_base[p] = (int64_t)items.size();
         const int32_t tiles = (int32_t)((gkeys[p] + segattn::kTileKeys - 1) / segattn::kTileKeys);
         for (int32_t q0 = 0; q0 < gq; q0 += (int32_t)span)
-          for (int g = 0; g < kv_heads; ++g) items.push_back({p, g, q0, tiles, true});
+          for (int g = 0; g < kv_heads; ++g) items.push_back({p, g, q0, tiles, true, gq - q0 <= qpt});
       }
       ngseg += (int64_t)gsegs[p].len.size();
     }
@@ -474,6 +488,8 @@ extern "C" int seg_attn_build_table(int batch, const int32_t* q_lens, const int3
   desc->num_group_parts = group_pieces.slots;
   desc->num_citems = (int32_t)citems.size();
   desc->num_cascade = (int32_t)cascade.size();
+  desc->num_single = main_pieces.single;
+  desc->num_group_single = group_pieces.single;
   desc->group_total_k = group_total_k;
   desc->table_bytes = (uint64_t)lay.n * sizeof(int32_t);
   desc->workspace_bytes = segattn::workspace_layout(*desc, [&] {

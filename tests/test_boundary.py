@@ -203,3 +203,20 @@ def test_prefill_without_split_needs_no_workspace():
     assert d.num_merge == 0 and d.num_parts == 0 and d.workspace_bytes == 0
     work = np.array(view(tab, d.off_work, 8 * d.num_work)).reshape(-1, 8)
     assert (work[:, 5] == -1).all() and (work[:, 3] == 0).all()
+
+
+def test_prefill_one_tile_kernel_only_for_all_single_tile_passes():
+    # G = 8: 16 queries per 128-row tile, 32 per item.
+    # Requests of 10 and 7 queries: every item holds queries in its first tile only.
+    tab = build([10, 7], [[(0, 300)], [(400, 200)]], num_slots=900, hq=16, hkv=2)
+    d = tab.desc
+    work = np.array(view(tab, d.off_work, 8 * d.num_work)).reshape(-1, 8)
+    assert d.num_single == d.num_work == 4 and (work[:, 6] == 1).all()
+    lens = work[:, 4] - work[:, 3]
+    assert list(lens) == sorted(lens, reverse=True)
+    # a request of 40 queries adds an item with two query tiles: one two-tile launch
+    tab = build([40, 10, 7], [[(0, 300)], [(400, 200)], [(700, 100)]], num_slots=900, hq=16,
+                hkv=2)
+    d = tab.desc
+    work = np.array(view(tab, d.off_work, 8 * d.num_work)).reshape(-1, 8)
+    assert d.num_single == 0 and (work[:, 6] == 0).all()

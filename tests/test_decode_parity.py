@@ -81,14 +81,15 @@ def test_decode_ragged_chunk_tails_and_tiny_segments():
 
 
 def test_decode_split_choice_does_not_change_result():
-    # alone, the request is cut into 256-key chunks and merged; as one of 600 copies
-    # sharing its (read-only) segments the planner picks 2048-key chunks, so the
-    # same request takes the single-chunk path
+    # alone, the request is cut into 256-key chunks and merged; as one of 1200 copies
+    # sharing its (read-only) segments (1200 CTAs at 2048-key chunks, more than the
+    # planner's 8 x 148 target) the planner keeps 2048-key chunks, so the same
+    # request takes the single-chunk path
     case = random_case(10, batch=1, hq=8, hkv=1, d=128, causal=True, max_k=2000, q_mode="decode")
     c = _dev(case)
     out1, lse1, t1 = run_cuda(c["q"], c["k_pool"], c["v_pool"], None, c["seg_starts"],
                               c["seg_lens"], c["num_slots"], True, sa.MODE_DECODE, c["scale"])
-    rep = 600
+    rep = 1200
     out2, lse2, t2 = run_cuda(c["q"].repeat(rep, 1, 1), c["k_pool"], c["v_pool"], None,
                               c["seg_starts"] * rep, c["seg_lens"] * rep, c["num_slots"], True,
                               sa.MODE_DECODE, c["scale"])

@@ -4,8 +4,10 @@ Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline / reference
 legs of ``bench.py`` may import this package.  The product path never does.
 
 The arithmetic lives in ``seg_attn_oracle.c`` (plain two-pass softmax
-attention in double precision that walks the segment lists itself); this file
-compiles it with gcc on first use and marshals arguments through ctypes.
+attention in double precision that walks the segment lists itself) and
+``seg_la_oracle.c`` (the simple-GLA linear-attention recurrence, token by
+token); this file compiles them with gcc on first use and marshals arguments
+through ctypes.
 """
 from __future__ import annotations
 
@@ -19,6 +21,7 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "seg_attn_oracle.c")
+_SRC_LA = os.path.join(_HERE, "seg_la_oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
 _lock = threading.Lock()
 _libs = {}
@@ -30,10 +33,11 @@ def build(force: bool = False, mutant: int = 0) -> str:
     ``mutant`` > 0 builds a copy with one planted mistake (see the C source),
     used only by the tests that check the pins catch such mistakes."""
     path = _LIB if mutant == 0 else os.path.join(_HERE, f"liboracle_mut{mutant}.so")
-    if force or not os.path.exists(path) or os.path.getmtime(path) < os.path.getmtime(_SRC):
+    newest = max(os.path.getmtime(_SRC), os.path.getmtime(_SRC_LA))
+    if force or not os.path.exists(path) or os.path.getmtime(path) < newest:
         tmp = path + f".tmp{os.getpid()}"
         subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
-                               f"-DORACLE_MUTANT={mutant}", "-o", tmp, _SRC, "-lm"])
+                               f"-DORACLE_MUTANT={mutant}", "-o", tmp, _SRC, _SRC_LA, "-lm"])
         os.replace(tmp, path)
     return path
 
@@ -58,6 +62,9 @@ def _load(mutant: int = 0):
             lib.oracle_rows_fp8.restype = ctypes.c_int
             lib.oracle_e4m3_decode.argtypes = [P, ctypes.c_int64, P]
             lib.oracle_e4m3_decode.restype = None
+            lib.oracle_la.argtypes = [ctypes.c_int, P, P, P, P, P, ctypes.c_int, ctypes.c_int,
+                                      ctypes.c_double, P, ctypes.c_int64, P, P, P]
+            lib.oracle_la.restype = ctypes.c_int
             _libs[mutant] = lib
     return _libs[mutant]
 
@@ -166,3 +173,32 @@ def attention_fp8(q_lens, seg_starts, seg_lens, q, k_pool, v_pool, k_scale, v_sc
     if rows is None:
         o, l = o.view(-1, hq, d), l.view(-1, hq)
     return o, l
+
+
+def linear_attention(q_lens, q, k, v, g, scale, state_in=None, in_slot=None, mutant=0):
+    """Oracle of segment linear attention (simple GLA) for one batch.
+
+    ``q, k, v`` bf16 [T, H, d] (CPU), ``g`` [T, H] log-decays (any float dtype, taken as
+    float64), ``state_in`` [N, H, d, d] states of the pool (or None), ``in_slot`` per
+    request (-1 or None: zero initial state).  Returns (out [T, H, d], state [B, H, d, d])
+    in float64."""
+    lib = _load(mutant)
+    ql = _i32(q_lens)
+    batch = ql.size
+    T, H, d = q.shape
+    slots = _i32(in_slot if in_slot is not None else [-1] * batch)
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    gd = np.ascontiguousarray(g.detach().cpu().double().numpy().reshape(-1))
+    if state_in is not None:
+        st = np.ascontiguousarray(state_in.detach().cpu().double().numpy())
+        n_in = st.shape[0]
+    else:
+        st, n_in = np.zeros(1), 0
+    out = np.zeros((T, H, d), dtype=np.float64)
+    state = np.zeros((batch, H, d, d), dtype=np.float64)
+    rc = lib.oracle_la(batch, _ptr(ql), _ptr(qb), _ptr(kb), _ptr(vb), _ptr(gd), H, d,
+                       float(scale), _ptr(st) if n_in else ctypes.c_void_p(0), n_in, _ptr(slots),
+                       _ptr(out), _ptr(state))
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments")
+    return torch.from_numpy(out), torch.from_numpy(state)

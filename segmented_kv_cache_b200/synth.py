@@ -27,7 +27,7 @@ from typing import List, Optional
 import torch
 
 __all__ = ["Batch", "Workload", "make_workload", "CONFIG_NAMES", "split_uniform_cuts",
-           "place_segments", "fp8_pools"]
+           "place_segments", "fp8_pools", "LAWorkload", "make_la_workload", "LA_CONFIGS"]
 
 CONFIG_NAMES = {
     1: "tiny causal prefill (2 req, q=k=16/33, 4/1 heads, d64)",
@@ -283,3 +283,68 @@ def fp8_pools(k_pool: torch.Tensor, v_pool: torch.Tensor):
     k8, ks = one(k_pool)
     v8, vs = one(v_pool)
     return k8, v8, ks, vs
+
+
+# --------------------------------------------------------------------------- linear attention
+# Shapes of the Flood README "Kernels > Seg-linear-attn" table: 16 heads, 16 kv
+# heads, head_dim 128; prefill batch 1 and 2 at 1024 tokens, decode batch 64 and 256.
+LA_CONFIGS = {
+    "la-prefill-1x1024": dict(mode="prefill", batch=1, q_len=1024, seed=11),
+    "la-prefill-2x1024": dict(mode="prefill", batch=2, q_len=1024, seed=12),
+    "la-decode-64": dict(mode="decode", batch=64, q_len=1, seed=13),
+    "la-decode-256": dict(mode="decode", batch=256, q_len=1, seed=14),
+}
+
+
+@dataclass
+class LAWorkload:
+    """One call of segment linear attention: packed tokens of every request, the state
+    pool and each request's slots (in_slot -1: the request starts from a zero state)."""
+    name: str
+    mode: str
+    heads: int
+    head_dim: int
+    q_lens: List[int]
+    q: torch.Tensor          # bf16 [T, H, d]
+    k: torch.Tensor
+    v: torch.Tensor
+    g: torch.Tensor          # fp32 [T, H], log of the per-token decay
+    state_pool: torch.Tensor  # fp32 [num_state_slots, H, d, d]
+    in_slot: List[int]
+    out_slot: List[int]
+    scale: float
+
+
+def make_la_workload(name: str, device: str = "cpu", seed: Optional[int] = None,
+                     heads: int = 16, head_dim: int = 128, q_lens: Optional[List[int]] = None,
+                     fresh: Optional[bool] = None) -> LAWorkload:
+    """Inputs of a linear-attention config (``LA_CONFIGS``) or, with ``q_lens`` given, of a
+    custom batch.  q, k, v ~ N(0, 1) in bf16; g = log(sigmoid(x)) / 16 with x ~ N(0, 1)
+    (per-token decay exp(g) in (0.94, 1)); the pool has 2 state slots per request, every
+    state ~ 4 * N(0, 1) (the size a state reaches under that decay); decode requests read
+    their state from a random slot and write it back there, prefill requests start from a
+    zero state (``fresh``) and write a slot of their own.  Draw order: slots -> q -> k ->
+    v -> g -> states, on a generator seeded with the config seed."""
+    cfg = LA_CONFIGS.get(name, {})
+    mode = cfg.get("mode", "prefill")
+    if q_lens is None:
+        q_lens = [cfg["q_len"]] * cfg["batch"]
+    seed = cfg.get("seed", 0) if seed is None else seed
+    fresh = (mode == "prefill") if fresh is None else fresh
+    B = len(q_lens)
+    gen = torch.Generator(device="cpu").manual_seed(seed)
+    perm = torch.randperm(2 * B, generator=gen).tolist()
+    out_slot = perm[:B]
+    in_slot = [-1] * B if fresh else list(out_slot)
+    vgen = torch.Generator(device=device).manual_seed(seed)
+    T = sum(q_lens)
+    q = _values((T, heads, head_dim), vgen, device)
+    k = _values((T, heads, head_dim), vgen, device)
+    v = _values((T, heads, head_dim), vgen, device)
+    x = torch.randn((T, heads), generator=vgen, device=device, dtype=torch.float32)
+    g = torch.nn.functional.logsigmoid(x) / 16.0
+    states = torch.randn((2 * B, heads, head_dim, head_dim), generator=vgen, device=device,
+                         dtype=torch.float32) * 4.0
+    return LAWorkload(name=name, mode=mode, heads=heads, head_dim=head_dim, q_lens=list(q_lens),
+                      q=q, k=k, v=v, g=g, state_pool=states, in_slot=in_slot, out_slot=out_slot,
+                      scale=1.0 / math.sqrt(head_dim))

@@ -226,7 +226,9 @@ int seg_attn_decode(const void* q, const void* k_pool, const void* v_pool, void*
  * word.  Kernels never trap; every wait on an mbarrier gives up after one
  * second, and a CTA that gave up drains its copies, frees its tensor memory,
  * returns, and sets bit 0 of this word (its output rows are then undefined);
- * seg_attn_kv_append sets bit 1 (value 2) for a slot out of range.  Synchronous: copies from the device (implicitly synchronises
+ * seg_attn_kv_append sets bit 1 (value 2) for a slot out of range; a
+ * segment linear attention prefill kernel (seg_la.h) that gave up sets bit 2
+ * (value 4).  Synchronous: copies from the device (implicitly synchronises
  * the current device).  *value = 0 means no kernel gave up since the last call.
  */
 int seg_attn_take_device_error(int* value);

@@ -24,6 +24,8 @@ __all__ = [
     "seg_attn_take_device_error", "SegTable", "load_library", "LIB_PATH",
     "MODE_PREFILL", "MODE_DECODE", "STATUS", "SegPool", "seg_attn_kv_append",
     "seg_attn_decode_fp8", "seg_attn_kv_append_fp8", "SHARE_PREFIX",
+    "seg_la_table_desc", "seg_la_build_table", "seg_la_workspace_size", "seg_la_prefill",
+    "seg_la_decode", "LATable",
 ]
 
 MODE_PREFILL = 0
@@ -63,6 +65,21 @@ class seg_attn_table_desc(ctypes.Structure):
         ("off_group_seg_start", ctypes.c_int64), ("off_group_seg_kstart", ctypes.c_int64),
         ("off_group_seg_len", ctypes.c_int64), ("off_group_work", ctypes.c_int64),
         ("off_citem", ctypes.c_int64), ("off_cascade", ctypes.c_int64),
+    ]
+
+
+class seg_la_table_desc(ctypes.Structure):
+    """Mirror of ``seg_la_table_desc`` in include/seg_la.h."""
+    _fields_ = [
+        ("magic", ctypes.c_uint32), ("version", ctypes.c_uint32),
+        ("mode", ctypes.c_int32), ("batch", ctypes.c_int32), ("heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32), ("chunk_len", ctypes.c_int32),
+        ("num_chunks", ctypes.c_int32),
+        ("total_q", ctypes.c_int64), ("num_state_slots", ctypes.c_int64),
+        ("off_q_offsets", ctypes.c_int64), ("off_in_slot", ctypes.c_int64),
+        ("off_out_slot", ctypes.c_int64), ("off_req_chunks", ctypes.c_int64),
+        ("off_chunks", ctypes.c_int64),
+        ("table_bytes", ctypes.c_uint64), ("workspace_bytes", ctypes.c_uint64),
     ]
 
 
@@ -126,6 +143,15 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         lib.seg_attn_kv_append_fp8.restype = I
         lib.seg_attn_decode_fp8.argtypes = [P, P, P, P, P, P, P, P, D, ctypes.c_float, P, SZ, P]
         lib.seg_attn_decode_fp8.restype = I
+        LD = ctypes.POINTER(seg_la_table_desc)
+        lib.seg_la_build_table.argtypes = [I, P, P, P, I64, I, I, I, P, SZ, LD]
+        lib.seg_la_build_table.restype = I
+        lib.seg_la_workspace_size.argtypes = [LD]
+        lib.seg_la_workspace_size.restype = SZ
+        lib.seg_la_prefill.argtypes = [P, P, P, P, P, P, P, LD, ctypes.c_float, P, SZ, P]
+        lib.seg_la_prefill.restype = I
+        lib.seg_la_decode.argtypes = [P, P, P, P, P, P, P, LD, ctypes.c_float, P]
+        lib.seg_la_decode.restype = I
         _lib = lib
         return lib
 
@@ -334,3 +360,72 @@ def seg_attn_decode_fp8(q, k_pool, v_pool, k_scale, v_scale, out, lse, dev_table
                                  int(ws_bytes), _stream_ptr(stream))
     if rc != 0:
         raise SegAttnError("seg_attn_decode_fp8", rc)
+
+
+# ----------------------------------------------------------------- segment linear attention
+def seg_la_build_table(q_lens, in_slot, out_slot, num_state_slots: int, mode: int, heads: int,
+                       head_dim: int, pin: bool = False):
+    """Returns (host table int32 tensor, seg_la_table_desc).  ``q_lens`` may be None in decode
+    mode.  Raises SegAttnError."""
+    lib = load_library()
+    ins, outs = _i32(in_slot), _i32(out_slot)
+    ql = _i32(q_lens) if q_lens is not None else None
+    desc = seg_la_table_desc()
+    args = [int(ins.size), _np_ptr(ql), _np_ptr(ins), _np_ptr(outs), int(num_state_slots),
+            int(mode), int(heads), int(head_dim)]
+    rc = lib.seg_la_build_table(*args, ctypes.c_void_p(0), 0, ctypes.byref(desc))
+    if rc != 0:
+        raise SegAttnError("seg_la_build_table", rc)
+    host = torch.zeros(max(1, (desc.table_bytes + 3) // 4), dtype=torch.int32, pin_memory=pin)
+    rc = lib.seg_la_build_table(*args, ctypes.c_void_p(host.data_ptr()), int(desc.table_bytes),
+                                ctypes.byref(desc))
+    if rc != 0:
+        raise SegAttnError("seg_la_build_table", rc)
+    return host, desc
+
+
+def seg_la_workspace_size(desc: seg_la_table_desc) -> int:
+    return int(load_library().seg_la_workspace_size(ctypes.byref(desc)))
+
+
+def seg_la_prefill(q, k, v, g, out, state_pool, dev_table, desc, scale, workspace=None,
+                   stream=None) -> None:
+    """Chunked simple-GLA prefill on ``stream`` (default: torch's current stream)."""
+    lib = load_library()
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    rc = lib.seg_la_prefill(_dptr(q), _dptr(k), _dptr(v), _dptr(g), _dptr(out), _dptr(state_pool),
+                            _dptr(dev_table), ctypes.byref(desc), float(scale), _dptr(workspace),
+                            int(ws_bytes), _stream_ptr(stream))
+    if rc != 0:
+        raise SegAttnError("seg_la_prefill", rc)
+
+
+def seg_la_decode(q, k, v, g, out, state_pool, dev_table, desc, scale, stream=None) -> None:
+    """One-token simple-GLA decode on ``stream`` (default: torch's current stream)."""
+    lib = load_library()
+    rc = lib.seg_la_decode(_dptr(q), _dptr(k), _dptr(v), _dptr(g), _dptr(out), _dptr(state_pool),
+                           _dptr(dev_table), ctypes.byref(desc), float(scale), _stream_ptr(stream))
+    if rc != 0:
+        raise SegAttnError("seg_la_decode", rc)
+
+
+@dataclass
+class LATable:
+    """A built linear-attention table: host copy, description, device copy."""
+    host: torch.Tensor
+    desc: seg_la_table_desc
+    device: Optional[torch.Tensor] = None
+
+    @classmethod
+    def build(cls, q_lens, in_slot, out_slot, num_state_slots, mode, heads, head_dim, pin=False):
+        host, desc = seg_la_build_table(q_lens, in_slot, out_slot, num_state_slots, mode, heads,
+                                        head_dim, pin=pin)
+        return cls(host=host, desc=desc)
+
+    def to(self, device, non_blocking=False) -> "LATable":
+        self.device = self.host.to(device, non_blocking=non_blocking)
+        return self
+
+    @property
+    def workspace_bytes(self) -> int:
+        return seg_la_workspace_size(self.desc)

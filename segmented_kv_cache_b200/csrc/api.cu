@@ -6,6 +6,7 @@
 
 #include "seg_attn.h"
 #include "seg_attn_internal.h"
+#include "seg_la_internal.h"
 
 namespace {
 
@@ -180,6 +181,9 @@ extern "C" int seg_attn_take_device_error(int* value) {
   if (rc != SEG_ATTN_OK) return rc;
   rc = segattn::take_append_error(&append_err);
   if (rc != SEG_ATTN_OK) return rc;
-  *value = (wait_err ? 1 : 0) | (append_err ? 2 : 0);
+  int la_err = 0;
+  rc = segla::take_la_error(&la_err);
+  if (rc != SEG_ATTN_OK) return rc;
+  *value = (wait_err ? 1 : 0) | (append_err ? 2 : 0) | (la_err ? 4 : 0);
   return SEG_ATTN_OK;
 }

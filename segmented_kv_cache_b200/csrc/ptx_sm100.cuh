@@ -133,6 +133,24 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int m, int n, bool b_mn_ma
          | ((uint32_t)(m >> 4) << 24);           // M / 16
 }
 
+// The same with A's major-ness chosen too (bit 15): A MN-major means the M index
+// is the contiguous one in shared memory (an operand used transposed).
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_ab(int m, int n, bool a_mn_major,
+                                                         bool b_mn_major) {
+  return idesc_bf16_f32(m, n, b_mn_major) | ((a_mn_major ? 1u : 0u) << 15);
+}
+
+// Make this thread's ordinary shared-memory writes visible to the tensor cores
+// (async proxy) before they read the same bytes.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Barrier over `count` threads (a multiple of 32) on hardware barrier `id` (1..15).
+__device__ __forceinline__ void named_barrier(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                        uint32_t accumulate) {
   asm volatile(

@@ -27,14 +27,16 @@ def declared_functions():
     for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
         text = open(h).read()
         text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-        names += re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b(seg_attn_\w+)\s*\(", text, re.M)
+        names += re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b(seg_(?:attn|la)_\w+)\s*\(",
+                            text, re.M)
     return sorted(set(names))
 
 
 def test_every_declared_symbol_is_exported(built_library):
     names = declared_functions()
     assert {"seg_attn_build_table", "seg_attn_prefill", "seg_attn_decode",
-            "seg_attn_workspace_size", "seg_attn_status_string"} <= set(names)
+            "seg_attn_workspace_size", "seg_attn_status_string", "seg_la_build_table",
+            "seg_la_prefill", "seg_la_decode", "seg_la_workspace_size"} <= set(names)
     for n in names:
         assert hasattr(built_library, n), n
 

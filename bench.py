@@ -621,6 +621,102 @@ def run_kv_append(args):
     return 0
 
 
+def la_algorithmic(w):
+    """(bytes, flops) a linear-attention call must move / do: q, k, v, g read, out written,
+    states read and written once; prefill flops of the chunked form (Q K^T, P V, Q S and
+    the chunk state K'^T V per 128-token chunk)."""
+    T, H, d = w.q.shape
+    B = len(w.q_lens)
+    state = d * d * 4
+    by = 4 * T * H * d * 2 + T * H * 4
+    by += sum(state * H for s in w.in_slot if s >= 0) + sum(state * H for s in w.out_slot if s >= 0)
+    if w.mode == "decode":
+        return by, 6.0 * B * H * d * d
+    fl = 0.0
+    for n in w.q_lens:
+        for t0 in range(0, n, 128):
+            c = min(128, n - t0)
+            fl += H * (4.0 * c * c * d + 4.0 * c * d * d)
+    return by, fl
+
+
+def run_linear(args):
+    """Segment linear attention on the shapes of the Flood README "Seg-linear-attn" table;
+    one JSON line with the per-call latency of each shape."""
+    import oracle
+    device = torch.device("cuda", 0)
+    peaks, kind = load_peaks()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    res = {}
+    for name in synth.LA_CONFIGS:
+        w = synth.make_la_workload(name, device=str(device))
+        mode = sa.MODE_PREFILL if w.mode == "prefill" else sa.MODE_DECODE
+        tab = sa.LATable.build(w.q_lens if mode == sa.MODE_PREFILL else None, w.in_slot,
+                               w.out_slot, w.state_pool.shape[0], mode, w.heads, w.head_dim,
+                               pin=True).to(device)
+        out = torch.empty_like(w.q)
+        pool0 = w.state_pool.clone()
+        ws = (torch.empty(tab.workspace_bytes, dtype=torch.uint8, device=device)
+              if tab.workspace_bytes else None)
+
+        def call():
+            if mode == sa.MODE_PREFILL:
+                sa.seg_la_prefill(w.q, w.k, w.v, w.g, out, w.state_pool, tab.device, tab.desc,
+                                  w.scale, ws)
+            else:
+                sa.seg_la_decode(w.q, w.k, w.v, w.g, out, w.state_pool, tab.device, tab.desc,
+                                 w.scale)
+        for _ in range(args.warmup):
+            call()
+        torch.cuda.synchronize()
+        times = []
+        for _ in range(args.steps):
+            flush.zero_()  # L2 cold for every call
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            call()
+            e1.record()
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1) * 1e3)
+        assert sa.seg_attn_take_device_error() == 0
+        us = statistics.median(times)
+        by, fl = la_algorithmic(w)
+        gbs = by / (us * 1e-6) / 1e9
+        entry = {"us": us, "us_min": min(times), "launches": 3 if mode == sa.MODE_PREFILL else 1,
+                 "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
+                              "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "bytes": by,
+                              "traffic": None},
+                 "tflops": fl / (us * 1e-6) / 1e12}
+        # parity spot check of this run's outputs (first request / first rows), state reset
+        w.state_pool.copy_(pool0)
+        call()
+        torch.cuda.synchronize()
+        n = min(w.q_lens[0], 256) if mode == sa.MODE_PREFILL else 1
+        s0 = w.in_slot[0]
+        st = pool0[s0:s0 + 1].cpu() if s0 >= 0 else None
+        args_o = ([n], w.q[:n].cpu(), w.k[:n].cpu(), w.v[:n].cpu(), w.g[:n].cpu(), w.scale, st,
+                  [0 if s0 >= 0 else -1])
+        t0 = time.perf_counter()
+        ro, _ = oracle.linear_attention(*args_o)
+        secs = time.perf_counter() - t0
+        err = (out[:n].double().cpu() - ro).abs()
+        entry["parity_sample"] = {"rows": n, "max_abs_over_rms": float(err.max() / ro.pow(2).mean().sqrt())}
+        entry["cpu_baseline"] = {"value": secs * 1e6 * sum(w.q_lens) / n,
+                                 "unit": "us (oracle, scaled from the sample)",
+                                 "cores": cpu_cores(), "kind": "oracle",
+                                 "sample": f"request 0, first {n} tokens, all heads"}
+        res[name] = entry
+        del w, tab, out, pool0, ws
+        torch.cuda.empty_cache()
+    print(json.dumps({"metric": "seg-linear-attn latency per call (16/16 heads, d 128)",
+                      "unit": "us", "higher_is_better": False, "n_gpus": 1, "steps": args.steps,
+                      "warmup": args.warmup, "dtype": "bf16 (fp32 state)", "data": "synthetic",
+                      "config": {"workload": "Seg-linear-attn table shapes",
+                                 "l2": "flushed before every timed call (256 MB write)"},
+                      "peak_kind": f"{kind} copy bandwidth", "shapes": res}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -640,6 +736,8 @@ def main():
                     help="cache type of the decode legs (fp8: E4M3 with per-kv-head scales)")
     ap.add_argument("--kv-append", action="store_true",
                     help="measure the KV-append kernel instead of the attention step")
+    ap.add_argument("--linear", action="store_true",
+                    help="measure segment linear attention on the Seg-linear-attn table shapes")
     ap.add_argument("--context-scale", type=float, default=1.0,
                     help="shorten the long-context mix (profiling captures only; 1.0 = as specified)")
     ap.add_argument("--no-e2e", action="store_true")
@@ -649,6 +747,8 @@ def main():
         print("note: fewer than 3 warm-up steps", file=sys.stderr)
     if args.kv_append:
         return run_kv_append(args)
+    if args.linear:
+        return run_linear(args)
     return run_reference(args) if args.impl == "reference" else run_ours(args)
 
 

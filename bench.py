@@ -225,7 +225,7 @@ class Path:
         self.device = device
         self.legs = []
         self.kv_dtype = kv_dtype
-        if kv_dtype == "fp8":  # decode legs read E4M3 copies of the pools
+        if kv_dtype == "fp8":  # every leg reads E4M3 copies of the pools
             self.k8, self.v8, self.ks, self.vs = synth.fp8_pools(wl.k_pool, wl.v_pool)
         for b in wl.batches:
             mode = sa.MODE_PREFILL if b.mode == "prefill" else sa.MODE_DECODE
@@ -243,10 +243,11 @@ class Path:
                                   launches=launches))
 
     def run_leg(self, leg, stream=None):
-        if leg["mode"] == sa.MODE_DECODE and self.kv_dtype == "fp8":
-            sa.seg_attn_decode_fp8(leg["batch"].q, self.k8, self.v8, self.ks, self.vs, leg["out"],
-                                   leg["lse"], leg["tab"].device, leg["tab"].desc, self.wl.scale,
-                                   leg["ws"], stream)
+        if self.kv_dtype == "fp8":
+            fn = (sa.seg_attn_prefill_fp8 if leg["mode"] == sa.MODE_PREFILL
+                  else sa.seg_attn_decode_fp8)
+            fn(leg["batch"].q, self.k8, self.v8, self.ks, self.vs, leg["out"], leg["lse"],
+               leg["tab"].device, leg["tab"].desc, self.wl.scale, leg["ws"], stream)
             return
         fn = sa.seg_attn_prefill if leg["mode"] == sa.MODE_PREFILL else sa.seg_attn_decode
         fn(leg["batch"].q, self.wl.k_pool, self.wl.v_pool, leg["out"], leg["lse"],
@@ -453,9 +454,11 @@ def run_ours(args):
     if dominant[0] == "tensor":
         achieved = dominant[2] / (dominant[1] * 1e-3) / 1e12
         peak = peaks["bf16_tflops_sustained"]
-        traffic = profiled_traffic("prefill_sm100", f"cfg{wl.config}")
+        fp8 = args.kv_dtype == "fp8"
+        traffic = None if fp8 else profiled_traffic("prefill_sm100", f"cfg{wl.config}")
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": traffic, "kernel": "prefill_kernel<128>",
+                "frac": achieved / peak, "traffic": traffic,
+                "kernel": "prefill_kernel<128> (E4M3 cache)" if fp8 else "prefill_kernel<128>",
                 "peak_kind": f"{peak_kind} sustained bf16 (cuBLAS 8192^3 loop)"}
     else:
         achieved = dominant[2] / (dominant[1] * 1e-3) / 1e9
@@ -470,7 +473,8 @@ def run_ours(args):
 
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if args.kv_dtype == "bf16" else "e4m3 cache, f16 products",
             "data": "synthetic",
             "config": {"workload": workload_name(wl) + ("" if args.context_scale == 1.0 else
                                                        f" (context x{args.context_scale})"),
@@ -481,7 +485,7 @@ def run_ours(args):
                               (2 * wl.k_pool.numel() * 2 / 1e9))
                        if 2 * wl.k_pool.numel() * 2 > L2_BYTES else "inputs fit in L2",
                        "parallelism": f"dp{world} (independent batches per GPU)",
-                       "share_prefix": bool(share)},
+                       "share_prefix": bool(share), "kv_cache": args.kv_dtype},
             "legs": legs, "roofline": roof,
             "gpu_launches": path.launches_per_step() * args.steps,
             "clocks": clocks}
@@ -490,6 +494,8 @@ def run_ours(args):
         line["e2e"] = run_e2e(path, args, world)
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"], line["parity_sample"] = run_cpu_baseline(path, args)
+        if args.kv_dtype == "fp8":  # the oracle sample reads the bf16 pools
+            line["parity_sample"]["note"] = "vs the bf16 cache: includes E4M3 quantisation"
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist:
@@ -729,11 +735,11 @@ def main():
     ap.add_argument("--no-share-prefix", dest="share_prefix", action="store_false")
     ap.add_argument("--ref-rows", type=int, default=48,
                     help="oracle rows per batch per step (bounded CPU sample)")
-    ap.add_argument("--cpu-rows", type=int, default=256,
+    ap.add_argument("--cpu-rows", type=int, default=1536,
                     help="oracle rows per batch for the cpu_baseline leg of our arm")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--kv-dtype", choices=["bf16", "fp8"], default="bf16",
-                    help="cache type of the decode legs (fp8: E4M3 with per-kv-head scales)")
+                    help="KV cache type of every leg (fp8: E4M3 with per-kv-head scales)")
     ap.add_argument("--kv-append", action="store_true",
                     help="measure the KV-append kernel instead of the attention step")
     ap.add_argument("--linear", action="store_true",

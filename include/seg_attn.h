@@ -333,6 +333,26 @@ int seg_attn_decode_fp8(const void* q, const void* k_pool, const void* v_pool, c
                         size_t workspace_bytes, void* stream);
 
 /*
+ * seg_attn_prefill_fp8 -- seg_attn_prefill over an FP8 KV cache (Flood README,
+ * "Roadmap": segment attention especially with FP8 kvcache), so chunked
+ * prefill and decode can share one E4M3 cache.
+ *   k_pool, v_pool  uint8 E4M3 codes [num_slots, kv_heads, head_dim] (16-byte
+ *                   aligned); the cached value is code * k_scale[g] (v_scale[g])
+ *   k_scale, v_scale  device fp32 [kv_heads], per-kv-head dequantisation scales
+ * Computes exactly what seg_attn_prefill computes on the dequantised pools, up
+ * to rounding: every product is f16 x f16 -> fp32 (codes widen exactly; queries
+ * become f16, so |q| must stay below 65504 and values under 2^-14 lose bits;
+ * P is f16).  out / lse / table / workspace exactly as seg_attn_prefill.  A
+ * shared-prefix table (SEG_ATTN_SHARE_PREFIX) returns SEG_ATTN_ERR_UNSUPPORTED;
+ * missing or misaligned scales return SEG_ATTN_ERR_INVALID_ARG.
+ */
+int seg_attn_prefill_fp8(const void* q, const void* k_pool, const void* v_pool,
+                         const float* k_scale, const float* v_scale, void* out, float* lse,
+                         const void* dev_table, const seg_attn_table_desc* desc,
+                         float softmax_scale, void* workspace, size_t workspace_bytes,
+                         void* stream);
+
+/*
  * seg_attn_kv_append_fp8 -- quantise the bf16 K/V rows of new tokens to E4M3
  * (code = round-to-nearest-even(x / scale[g]), saturated to +-448) and write
  * them into their slots of FP8 pools.  Same slot rules as seg_attn_kv_append.

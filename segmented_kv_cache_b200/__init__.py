@@ -23,7 +23,7 @@ __all__ = [
     "seg_attn_prefill", "seg_attn_decode", "seg_attn_status_string", "seg_attn_version",
     "seg_attn_take_device_error", "SegTable", "load_library", "LIB_PATH",
     "MODE_PREFILL", "MODE_DECODE", "STATUS", "SegPool", "seg_attn_kv_append",
-    "seg_attn_decode_fp8", "seg_attn_kv_append_fp8", "SHARE_PREFIX",
+    "seg_attn_decode_fp8", "seg_attn_prefill_fp8", "seg_attn_kv_append_fp8", "SHARE_PREFIX",
     "seg_la_table_desc", "seg_la_build_table", "seg_la_workspace_size", "seg_la_prefill",
     "seg_la_decode", "LATable",
 ]
@@ -141,8 +141,9 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         lib.seg_attn_kv_append.restype = I
         lib.seg_attn_kv_append_fp8.argtypes = [P, P, P, I64, I, I, P, P, P, P, I64, P]
         lib.seg_attn_kv_append_fp8.restype = I
-        lib.seg_attn_decode_fp8.argtypes = [P, P, P, P, P, P, P, P, D, ctypes.c_float, P, SZ, P]
-        lib.seg_attn_decode_fp8.restype = I
+        for fn in (lib.seg_attn_decode_fp8, lib.seg_attn_prefill_fp8):
+            fn.argtypes = [P, P, P, P, P, P, P, P, D, ctypes.c_float, P, SZ, P]
+            fn.restype = I
         LD = ctypes.POINTER(seg_la_table_desc)
         lib.seg_la_build_table.argtypes = [I, P, P, P, I64, I, I, I, P, SZ, LD]
         lib.seg_la_build_table.restype = I
@@ -349,17 +350,30 @@ def seg_attn_kv_append_fp8(k_new, v_new, slots, k_scale, v_scale, k_pool, v_pool
         raise SegAttnError("seg_attn_kv_append_fp8", rc)
 
 
+def _compute_fp8(fn_name, q, k_pool, v_pool, k_scale, v_scale, out, lse, dev_table, desc,
+                 softmax_scale, workspace, stream):
+    lib = load_library()
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    rc = getattr(lib, fn_name)(_dptr(q), _dptr(k_pool), _dptr(v_pool), _dptr(k_scale),
+                               _dptr(v_scale), _dptr(out), _dptr(lse), _dptr(dev_table),
+                               ctypes.byref(desc), float(softmax_scale), _dptr(workspace),
+                               int(ws_bytes), _stream_ptr(stream))
+    if rc != 0:
+        raise SegAttnError(fn_name, rc)
+
+
 def seg_attn_decode_fp8(q, k_pool, v_pool, k_scale, v_scale, out, lse, dev_table, desc,
                         softmax_scale, workspace=None, stream=None) -> None:
     """Decode over E4M3 pools (uint8 [S, Hkv, d]) with per-kv-head fp32 scales."""
-    lib = load_library()
-    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
-    rc = lib.seg_attn_decode_fp8(_dptr(q), _dptr(k_pool), _dptr(v_pool), _dptr(k_scale),
-                                 _dptr(v_scale), _dptr(out), _dptr(lse), _dptr(dev_table),
-                                 ctypes.byref(desc), float(softmax_scale), _dptr(workspace),
-                                 int(ws_bytes), _stream_ptr(stream))
-    if rc != 0:
-        raise SegAttnError("seg_attn_decode_fp8", rc)
+    _compute_fp8("seg_attn_decode_fp8", q, k_pool, v_pool, k_scale, v_scale, out, lse, dev_table,
+                 desc, softmax_scale, workspace, stream)
+
+
+def seg_attn_prefill_fp8(q, k_pool, v_pool, k_scale, v_scale, out, lse, dev_table, desc,
+                         softmax_scale, workspace=None, stream=None) -> None:
+    """Chunked prefill over E4M3 pools (uint8 [S, Hkv, d]) with per-kv-head fp32 scales."""
+    _compute_fp8("seg_attn_prefill_fp8", q, k_pool, v_pool, k_scale, v_scale, out, lse,
+                 dev_table, desc, softmax_scale, workspace, stream)
 
 
 # ----------------------------------------------------------------- segment linear attention

@@ -69,13 +69,21 @@ int launch_cascade(const void* dev_table, const seg_attn_table_desc& desc,
 
 }  // namespace
 
-extern "C" int seg_attn_prefill(const void* q, const void* k_pool, const void* v_pool, void* out,
-                                float* lse, const void* dev_table, const seg_attn_table_desc* desc,
-                                float softmax_scale, void* workspace, size_t workspace_bytes,
-                                void* stream) {
+namespace {
+
+int prefill_common(const void* q, const void* k_pool, const void* v_pool, const float* k_scale,
+                   const float* v_scale, bool fp8, void* out, float* lse, const void* dev_table,
+                   const seg_attn_table_desc* desc, float softmax_scale, void* workspace,
+                   size_t workspace_bytes, void* stream) {
   int rc = check_common(q, k_pool, v_pool, out, lse, dev_table, desc, softmax_scale,
                         SEG_ATTN_MODE_PREFILL);
   if (rc != SEG_ATTN_OK) return rc;
+  // shared-prefix plans run their prefix pass on the bf16 cache only
+  if (fp8 && desc->shared) return SEG_ATTN_ERR_UNSUPPORTED;
+  if (fp8 && desc->total_k > 0 &&
+      (!k_scale || !v_scale || (reinterpret_cast<uintptr_t>(k_scale) & 3) ||
+       (reinterpret_cast<uintptr_t>(v_scale) & 3)))
+    return SEG_ATTN_ERR_INVALID_ARG;
   if (desc->workspace_bytes > 0 &&
       (!workspace || workspace_bytes < desc->workspace_bytes || !aligned16(workspace)))
     return SEG_ATTN_ERR_WORKSPACE;
@@ -99,11 +107,33 @@ extern "C" int seg_attn_prefill(const void* q, const void* k_pool, const void* v
     a.part_o = desc->num_parts > 0 ? reinterpret_cast<float*>(at(workspace, ws_at.main_o)) : nullptr;
     a.part_lse =
         desc->num_parts > 0 ? reinterpret_cast<float*>(at(workspace, ws_at.main_lse)) : nullptr;
+    a.fp8 = fp8;
+    a.k_scale = k_scale;
+    a.v_scale = v_scale;
     rc = segattn::launch_prefill(a, st);
     if (rc != SEG_ATTN_OK) return rc;
   }
   if (desc->shared) return launch_cascade(dev_table, *desc, ws_at, workspace, out, lse, st);
   return SEG_ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" int seg_attn_prefill(const void* q, const void* k_pool, const void* v_pool, void* out,
+                                float* lse, const void* dev_table, const seg_attn_table_desc* desc,
+                                float softmax_scale, void* workspace, size_t workspace_bytes,
+                                void* stream) {
+  return prefill_common(q, k_pool, v_pool, nullptr, nullptr, false, out, lse, dev_table, desc,
+                        softmax_scale, workspace, workspace_bytes, stream);
+}
+
+extern "C" int seg_attn_prefill_fp8(const void* q, const void* k_pool, const void* v_pool,
+                                    const float* k_scale, const float* v_scale, void* out,
+                                    float* lse, const void* dev_table,
+                                    const seg_attn_table_desc* desc, float softmax_scale,
+                                    void* workspace, size_t workspace_bytes, void* stream) {
+  return prefill_common(q, k_pool, v_pool, k_scale, v_scale, true, out, lse, dev_table, desc,
+                        softmax_scale, workspace, workspace_bytes, stream);
 }
 
 namespace {

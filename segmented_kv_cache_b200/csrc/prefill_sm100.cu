@@ -52,6 +52,9 @@ __device__ int g_device_error;  // non-zero once a bounded wait gave up
 namespace {
 
 constexpr int kThreads = 320;
+// FP8 cache: two more warps (10, 11) widen E4M3 code tiles to f16 in shared memory
+constexpr int kThreadsFp8 = 384;
+constexpr int kConvThreads = 64;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
 constexpr float kRescaleLog2 = 8.0f;
 constexpr uint32_t kHalfBytes = 128 * 128;  // 128 rows x 64 bf16 (one swizzle-128B panel)
@@ -65,14 +68,18 @@ struct PrefillParams {
   float* part_o;    // split items: [slot][kItemRows][D], O / l of the piece
   float* part_lse;  // split items: [slot][kItemRows], log2 of the piece's sum of exp
   int work_base;    // first work item of this launch
+  const float* k_scale;  // FP8 cache: [kv_heads] dequantisation scales (value = code * scale)
+  const float* v_scale;
 };
 
 // Q (2 tiles) + K ring (2) + V ring (2) + barriers + alignment slack.  The
 // d = 64 variant asks for more than half the SM's shared memory as well, so
 // one CTA owns an SM and its 512 tensor-memory columns.
-template <int D>
+// The FP8 variant adds one staging tile of raw codes each for K and V.
+template <int D, bool FP8>
 constexpr size_t prefill_smem_bytes() {
-  constexpr size_t need = 6 * (D / 64) * (size_t)kHalfBytes + 256 + 1024;
+  constexpr size_t need =
+      6 * (D / 64) * (size_t)kHalfBytes + (FP8 ? 2 * kTileKeys * D : 0) + 256 + 1024;
   return need < 120 * 1024 ? 120 * 1024 : need;
 }
 
@@ -81,11 +88,52 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// Eight bf16 (one 16-byte chunk) -> eight f16 in place; exact for |x| in
+// [2^-14, 65504], rounded below (f16 subnormals), infinite above.
+__device__ __forceinline__ void bf16x8_to_f16x8(uint4& v) {
+  uint32_t* w = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    w[i] = ptx::pack_f16x2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xffff0000u));
+}
+
+// One tile of E4M3 codes (kTileKeys rows of D bytes, plain row-major) -> f16
+// in the 128-byte-swizzled K-major layout the tensor cores read (the layout a
+// tiled TMA load of a bf16 tile produces): row r, 16-byte chunk c of 64-column
+// half h lands at h * kHalfBytes + r * 128 + ((c ^ (r & 7)) * 16).
+template <int D>
+__device__ __forceinline__ void widen_tile(const uint8_t* src, uint8_t* dst, int ct) {
+  constexpr int kUnits = kTileKeys * D / 16;  // 16 codes per unit
+#pragma unroll 4
+  for (int u = ct; u < kUnits; u += kConvThreads) {
+    const int r = u / (D / 16), j = u % (D / 16);
+    const uint4 w = *reinterpret_cast<const uint4*>(src + r * D + 16 * j);
+    uint4 a, b;
+    a.x = ptx::e4m3x2_to_f16x2(w.x);
+    a.y = ptx::e4m3x2_to_f16x2(w.x >> 16);
+    a.z = ptx::e4m3x2_to_f16x2(w.y);
+    a.w = ptx::e4m3x2_to_f16x2(w.y >> 16);
+    b.x = ptx::e4m3x2_to_f16x2(w.z);
+    b.y = ptx::e4m3x2_to_f16x2(w.z >> 16);
+    b.z = ptx::e4m3x2_to_f16x2(w.w);
+    b.w = ptx::e4m3x2_to_f16x2(w.w >> 16);
+    uint8_t* rowp = dst + (j >> 2) * kHalfBytes + r * 128;
+    const int c0 = (j & 3) * 2;
+    *reinterpret_cast<uint4*>(rowp + ((c0 ^ (r & 7)) << 4)) = a;
+    *reinterpret_cast<uint4*>(rowp + (((c0 + 1) ^ (r & 7)) << 4)) = b;
+  }
+}
+
 // SINGLE: every item of the launch has queries in its first query tile only
 // (the planner lists those items last and launches them separately, so each
 // instantiation keeps its own register allocation).
-template <int D, bool SINGLE>
-__global__ void __launch_bounds__(kThreads, 1)
+// FP8: the pools hold E4M3 codes (value = code * scale of the kv head).  Code
+// tiles are staged by TMA as raw bytes and widened to f16 (exact) by warps 10
+// and 11 into the K/V rings; queries are converted bf16 -> f16 in shared memory
+// and P is f16, so every product is f16 x f16 -> f32.  The K scale is folded
+// into the softmax scale, the V scale into the output.
+template <int D, bool SINGLE, bool FP8>
+__global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_k3,
                    const __grid_constant__ CUtensorMap tm_v3, const PrefillParams p) {
@@ -99,7 +147,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sQ = sm;
   uint8_t* sK = sm + 2 * TILE;
   uint8_t* sV = sm + 4 * TILE;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + 6 * TILE);
+  uint8_t* sStK = sm + 6 * TILE;            // FP8: raw code tile of K
+  uint8_t* sStV = sStK + kTileKeys * D;     // FP8: raw code tile of V
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + 6 * TILE + (FP8 ? 2 * kTileKeys * D : 0));
   uint64_t* q_full = bars + 0;
   uint64_t* k_full = bars + 1;   // [2]
   uint64_t* k_empty = bars + 3;  // [2]
@@ -109,7 +159,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* p_full = bars + 11;  // [2]
   uint64_t* o_full = bars + 13;  // [2]
   uint64_t* mma_done = bars + 15;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  uint64_t* kst_full = bars + 16;   // FP8: code staging of K filled (TMA bytes)
+  uint64_t* kst_empty = bars + 17;  // FP8: code staging of K read by the converters
+  uint64_t* vst_full = bars + 18;
+  uint64_t* vst_empty = bars + 19;
+  uint64_t* q_conv = bars + 20;     // FP8: query tiles converted to f16
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 21);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -131,15 +186,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(k_full + s, 1);
+      // FP8: the ring is filled by the converter threads, not by TMA
+      mbar_init(k_full + s, FP8 ? kConvThreads : 1);
       mbar_init(k_empty + s, 1);
-      mbar_init(v_full + s, 1);
+      mbar_init(v_full + s, FP8 ? kConvThreads : 1);
       mbar_init(v_empty + s, 1);
       mbar_init(s_full + s, 1);
       mbar_init(p_full + s, 128);
       mbar_init(o_full + s, 1);
     }
     mbar_init(mma_done, 1);
+    if (FP8) {
+      mbar_init(kst_full, 1);
+      mbar_init(kst_empty, kConvThreads);
+      mbar_init(vst_full, 1);
+      mbar_init(vst_empty, kConvThreads);
+      mbar_init(q_conv, (SINGLE ? 1 : 2) * 128);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -205,6 +268,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                           rows[2], rows[3]);
           }
         };
+        // FP8: raw code rows (D bytes each) into the staging tile, no swizzle
+        auto load_codes = [&](uint8_t* dst, const CUtensorMap* tiled, const CUtensorMap* rowmap,
+                              uint64_t* bar) {
+          if (lane == 0) mbar_expect_tx(bar, kTileKeys * D);
+          __syncwarp();
+          if (contiguous) {
+            if (lane == 0) tma_load_3d(dst, tiled, bar, 0, g, slot0);
+          } else {
+            tma_gather4(dst + lane * 4 * D, rowmap, bar, 0, rows[0], rows[1], rows[2], rows[3]);
+          }
+        };
+        if (FP8) {
+          if (!__all_sync(0xffffffffu, mbar_wait(kst_empty, (i & 1) ^ 1, abort_flag, kWaitLimitNs, true))) break;
+          load_codes(sStK, &tm_k3, &tm_k, kst_full);
+          ++k_issued;
+          if (!__all_sync(0xffffffffu, mbar_wait(vst_empty, (i & 1) ^ 1, abort_flag, kWaitLimitNs, true))) break;
+          load_codes(sStV, &tm_v3, &tm_v, vst_full);
+          ++v_issued;
+          continue;
+        }
         if (!__all_sync(0xffffffffu, mbar_wait(k_empty + st, ph ^ 1, abort_flag, kWaitLimitNs, true))) break;
         load_tile(sK + st * TILE, &tm_k3, &tm_k, k_full + st);
         ++k_issued;
@@ -212,8 +295,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         load_tile(sV + st * TILE, &tm_v3, &tm_v, v_full + st);
         ++v_issued;
       }
-      // never leave the CTA with copies in flight
-      for (int s = 0; s < 2; ++s) {
+      // never leave the CTA with copies in flight (FP8: a staged copy is issued
+      // only after the converters read the previous one, so the last is enough)
+      if (FP8) {
+        if (k_issued > 0) mbar_wait(kst_full, (k_issued - 1) & 1, nullptr, kWaitLimitNs);
+        if (v_issued > 0) mbar_wait(vst_full, (v_issued - 1) & 1, nullptr, kWaitLimitNs);
+      }
+      for (int s = 0; !FP8 && s < 2; ++s) {
         if (k_issued > s) {
           const int last = s + 2 * ((k_issued - 1 - s) / 2);
           mbar_wait(k_full + s, (last >> 1) & 1, nullptr, kWaitLimitNs);
@@ -228,8 +316,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && n_tiles > 0) {
-      const uint32_t idesc_qk = idesc_bf16_f32(128, 128, false);
-      const uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
+      const uint32_t idesc_qk =
+          FP8 ? idesc_f16_f32(128, 128, false) : idesc_bf16_f32(128, 128, false);
+      const uint32_t idesc_pv = FP8 ? idesc_f16_f32(128, D, true) : idesc_bf16_f32(128, D, true);
       const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
       const uint32_t tS0 = tmem + 256, tO0 = tmem;
       // S buffer `sb` = Q tile `qt` . K stage `st`^T;  O tile `ot` += P (in S buffer `sb`) . V stage `st`
@@ -248,7 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                  sdesc_sw128(v_addr + st * TILE + k * 2048, kHalfBytes, 1024), idesc_pv,
                  (acc || k > 0) ? 1u : 0u);
       };
-      bool ok = mbar_wait(q_full, 0, abort_flag, kWaitLimitNs) &&
+      bool ok = mbar_wait(FP8 ? q_conv : q_full, 0, abort_flag, kWaitLimitNs) &&
                 mbar_wait(k_full + 0, 0, abort_flag, kWaitLimitNs);
       if (single) {
         // one query tile, S double-buffered: K tile i uses S buffer i & 1.  While the
@@ -327,6 +416,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(mma_done, 0, nullptr, kWaitLimitNs);
     }
     __syncwarp();
+  } else if (FP8 && warp >= 10) {
+    // ------------------------------------------------------------ FP8 code widening
+    // Staged E4M3 tile -> f16 K (V) ring slot, then make the generic-proxy
+    // writes visible to the tensor cores before signalling the ring slot full.
+    const int ct = threadIdx.x - 10 * 32;
+    bool ok = true;
+    for (int i = 0; ok && i < n_tiles; ++i) {
+      const int st = i & 1;
+      const uint32_t ph = (i >> 1) & 1;
+      if (!(ok = mbar_wait(kst_full, i & 1, abort_flag, kWaitLimitNs) &&
+                 mbar_wait(k_empty + st, ph ^ 1, abort_flag, kWaitLimitNs)))
+        break;
+      widen_tile<D>(sStK, sK + st * TILE, ct);
+      fence_proxy_async_smem();
+      mbar_arrive(k_full + st);
+      mbar_arrive(kst_empty);
+      if (!(ok = mbar_wait(vst_full, i & 1, abort_flag, kWaitLimitNs) &&
+                 mbar_wait(v_empty + st, ph ^ 1, abort_flag, kWaitLimitNs)))
+        break;
+      widen_tile<D>(sStV, sV + st * TILE, ct);
+      fence_proxy_async_smem();
+      mbar_arrive(v_full + st);
+      mbar_arrive(vst_empty);
+    }
   } else if (!single || warp < 6) {
     // ------------------------------------------------------------ softmax + epilogue
     const int t = (warp - 2) >> 2;
@@ -339,10 +452,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     uint32_t tS = lane_base + 256 + 128 * t;  // S buffer of the current K tile
     const uint32_t tO = lane_base + 128 * t;
-    const float sl2 = p.scale_log2;
+    // FP8: scores are q . code * k_scale, so the K scale joins the softmax scale
+    const float sl2 = FP8 ? p.scale_log2 * __ldg(p.k_scale + g) : p.scale_log2;
     float m_ref = -INFINITY;  // raw score units
     float l = 0.f;
     bool ok = true;
+    if (FP8 && n_tiles > 0) {
+      // this thread's query row of tile t: bf16 -> f16 in place (elementwise, so
+      // the swizzled order of the 16-byte chunks within the row does not matter)
+      ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, abort_flag, kWaitLimitNs));
+      if (ok) {
+#pragma unroll
+        for (int h = 0; h < HALVES; ++h)
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            uint4* chunk = reinterpret_cast<uint4*>(sQ + t * TILE + h * kHalfBytes + row * 128 + c * 16);
+            uint4 v = *chunk;
+            bf16x8_to_f16x8(v);
+            *chunk = v;
+          }
+        fence_proxy_async_smem();
+        mbar_arrive(q_conv);
+      }
+    }
     // Causal / tail mask of tile i, applied in place in tensor memory (-inf in
     // the columns this row must not see).  Only tiles where some row of the warp
     // needs it pay for it; the softmax itself never compares per element.
@@ -397,7 +529,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float pb = ex2(fmaf(f(sv[c][2 * e + 1]), sl2, -base));
           ls[0] += pa;
           ls[1] += pb;
-          pk[e] = pack_bf16(pa, pb);
+          pk[e] = FP8 ? pack_f16x2(pa, pb) : pack_bf16(pa, pb);
         }
         tmem_st16(tS + 16 * c, pk);
       }
@@ -457,7 +589,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok && slot >= 0) {
       // piece of a split item (or of a shared-prefix pass): O / l and log2(sum of exp)
       // of this key range, for every row that holds a query
-      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const float inv = l > 0.f ? (FP8 ? __ldg(p.v_scale + g) : 1.f) / l : 0.f;
       const int64_t prow = (int64_t)slot * kItemRows + t * kTileRows + row;
       float* po = p.part_o + prow * D;
       if (n_tiles > 0) tc_fence_after();
@@ -481,7 +613,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (row_valid) p.part_lse[prow] = l > 0.f ? m_ref * sl2 + log2f(l) : -INFINITY;
     } else if (ok) {
-      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const float inv = l > 0.f ? (FP8 ? __ldg(p.v_scale + g) : 1.f) / l : 0.f;
       __nv_bfloat16* orow = p.out + ((int64_t)(tok0 + qi) * p.q_heads + head) * D;
       if (n_tiles > 0) tc_fence_after();
 #pragma unroll
@@ -580,17 +712,33 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
+// bf16 maps are 128-byte swizzled (tensor-core operand layout); byte maps
+// (E4M3 codes, staged for widening) are plain row-major.
 bool encode(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims,
-            const cuuint64_t* strides, const cuuint32_t* box) {
+            const cuuint64_t* strides, const cuuint32_t* box, bool bytes = false) {
   auto fn = encode_fn();
   if (!fn) return false;
   const cuuint32_t elem[3] = {1, 1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides,
-            box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  return fn(map, bytes ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank,
+            const_cast<void*>(base), dims, strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            bytes ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D>
+template <int D, bool SINGLE, bool FP8>
+int launch_items(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                 const CUtensorMap& tk3, const CUtensorMap& tv3, const PrefillParams& p, int n,
+                 cudaStream_t stream) {
+  constexpr size_t smem = prefill_smem_bytes<D, FP8>();
+  if (cudaFuncSetAttribute(prefill_kernel<D, SINGLE, FP8>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return SEG_ATTN_ERR_CUDA;
+  prefill_kernel<D, SINGLE, FP8><<<n, FP8 ? kThreadsFp8 : kThreads, smem, stream>>>(tq, tk, tv, tk3,
+                                                                                  tv3, p);
+  return cudaGetLastError() == cudaSuccess ? SEG_ATTN_OK : SEG_ATTN_ERR_CUDA;
+}
+
+template <int D, bool FP8>
 int launch_prefill_d(const PrefillLaunch& a, cudaStream_t stream) {
   const seg_attn_table_desc& d = *a.desc;
   const int group = d.q_heads / d.kv_heads;
@@ -604,19 +752,24 @@ int launch_prefill_d(const PrefillLaunch& a, cudaStream_t stream) {
   {
     const int64_t rows = d.num_slots * d.kv_heads;
     const bool empty = rows == 0 || d.total_k == 0;
+    // bf16: 64-column boxes (one swizzle panel); FP8: whole D-byte code rows
+    constexpr int kElem = FP8 ? 1 : 2;
+    constexpr cuuint32_t kBoxCols = FP8 ? D : 64;
     const cuuint64_t dims[2] = {(cuuint64_t)D, empty ? 1ull : (cuuint64_t)rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-    const cuuint32_t box[2] = {64, 1};
+    const cuuint64_t strides[1] = {(cuuint64_t)D * kElem};
+    const cuuint32_t box[2] = {kBoxCols, 1};
     // with no keys no tile is ever loaded; the query buffer stands in as a valid address
-    if (!encode(&tk, empty ? a.q : a.k_pool, 2, dims, strides, box)) return SEG_ATTN_ERR_CUDA;
-    if (!encode(&tv, empty ? a.q : a.v_pool, 2, dims, strides, box)) return SEG_ATTN_ERR_CUDA;
+    if (!encode(&tk, empty ? a.q : a.k_pool, 2, dims, strides, box, FP8)) return SEG_ATTN_ERR_CUDA;
+    if (!encode(&tv, empty ? a.q : a.v_pool, 2, dims, strides, box, FP8)) return SEG_ATTN_ERR_CUDA;
     // the same pools as [slots][kv heads][d]: 128 consecutive slots of one head per box
     const cuuint64_t dims3[3] = {(cuuint64_t)D, (cuuint64_t)d.kv_heads,
                                  empty ? 1ull : (cuuint64_t)d.num_slots};
-    const cuuint64_t strides3[2] = {(cuuint64_t)D * 2, (cuuint64_t)d.kv_heads * D * 2};
-    const cuuint32_t box3[3] = {64, 1, (cuuint32_t)kTileKeys};
-    if (!encode(&tk3, empty ? a.q : a.k_pool, 3, dims3, strides3, box3)) return SEG_ATTN_ERR_CUDA;
-    if (!encode(&tv3, empty ? a.q : a.v_pool, 3, dims3, strides3, box3)) return SEG_ATTN_ERR_CUDA;
+    const cuuint64_t strides3[2] = {(cuuint64_t)D * kElem, (cuuint64_t)d.kv_heads * D * kElem};
+    const cuuint32_t box3[3] = {kBoxCols, 1, (cuuint32_t)kTileKeys};
+    if (!encode(&tk3, empty ? a.q : a.k_pool, 3, dims3, strides3, box3, FP8))
+      return SEG_ATTN_ERR_CUDA;
+    if (!encode(&tv3, empty ? a.q : a.v_pool, 3, dims3, strides3, box3, FP8))
+      return SEG_ATTN_ERR_CUDA;
   }
   PrefillParams p;
   p.out = static_cast<__nv_bfloat16*>(a.out);
@@ -630,24 +783,19 @@ int launch_prefill_d(const PrefillLaunch& a, cudaStream_t stream) {
   p.causal = d.causal;
   p.part_o = a.part_o;
   p.part_lse = a.part_lse;
-  constexpr size_t smem = prefill_smem_bytes<D>();
+  p.k_scale = a.k_scale;
+  p.v_scale = a.v_scale;
   // two-tile items first, then the single-tile items listed at the end
   const int n_single = d.num_single, n_two = d.num_work - d.num_single;
   if (n_two > 0) {
-    if (cudaFuncSetAttribute(prefill_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
-      return SEG_ATTN_ERR_CUDA;
     p.work_base = 0;
-    prefill_kernel<D, false><<<n_two, kThreads, smem, stream>>>(tq, tk, tv, tk3, tv3, p);
-    if (cudaGetLastError() != cudaSuccess) return SEG_ATTN_ERR_CUDA;
+    const int rc = launch_items<D, false, FP8>(tq, tk, tv, tk3, tv3, p, n_two, stream);
+    if (rc != SEG_ATTN_OK) return rc;
   }
   if (n_single > 0) {
-    if (cudaFuncSetAttribute(prefill_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
-      return SEG_ATTN_ERR_CUDA;
     p.work_base = n_two;
-    prefill_kernel<D, true><<<n_single, kThreads, smem, stream>>>(tq, tk, tv, tk3, tv3, p);
-    if (cudaGetLastError() != cudaSuccess) return SEG_ATTN_ERR_CUDA;
+    const int rc = launch_items<D, true, FP8>(tq, tk, tv, tk3, tv3, p, n_single, stream);
+    if (rc != SEG_ATTN_OK) return rc;
   }
   if (d.num_merge > 0) {
     prefill_merge_kernel<D><<<dim3(d.num_merge, 4), 256, 0, stream>>>(p);
@@ -659,8 +807,11 @@ int launch_prefill_d(const PrefillLaunch& a, cudaStream_t stream) {
 }  // namespace
 
 int launch_prefill(const PrefillLaunch& a, cudaStream_t stream) {
-  return a.desc->head_dim == 128 ? launch_prefill_d<128>(a, stream)
-                                 : launch_prefill_d<64>(a, stream);
+  if (a.fp8)
+    return a.desc->head_dim == 128 ? launch_prefill_d<128, true>(a, stream)
+                                   : launch_prefill_d<64, true>(a, stream);
+  return a.desc->head_dim == 128 ? launch_prefill_d<128, false>(a, stream)
+                                 : launch_prefill_d<64, false>(a, stream);
 }
 
 int take_device_error(int* value) {

@@ -247,6 +247,25 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16
       : "memory");
 }
 
+// Instruction descriptor, kind::f16: f16 x f16 -> f32 (A and B both f16).
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int m, int n, bool b_mn_major) {
+  return idesc_bf16_f32(m, n, b_mn_major) & ~((1u << 7) | (1u << 10));
+}
+
+// Two E4M3 codes (low byte first) -> two f16 (exact: every E4M3 value is an f16).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
+  uint32_t y;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(y) : "h"(static_cast<unsigned short>(two_codes)));
+  return y;
+}
+
+// Two fp32 -> f16 pair, round to nearest even (lo in the low half).
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t y;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(y) : "f"(hi), "f"(lo));
+  return y;
+}
+
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

@@ -88,6 +88,9 @@ struct PrefillLaunch {
   float scale;
   float* part_o;    // [slots][kItemRows][D] fp32, normalised per piece (split items only)
   float* part_lse;  // [slots][kItemRows] fp32, log2 domain
+  bool fp8 = false;                // pools hold E4M3 codes
+  const float* k_scale = nullptr;  // [Hkv] device, FP8 only
+  const float* v_scale = nullptr;
 };
 
 struct DecodeLaunch {

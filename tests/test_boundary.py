@@ -222,3 +222,23 @@ def test_prefill_one_tile_kernel_only_for_all_single_tile_passes():
     d = tab.desc
     work = np.array(view(tab, d.off_work, 8 * d.num_work)).reshape(-1, 8)
     assert d.num_single == 0 and (work[:, 6] == 0).all()
+
+
+def test_fp8_calls_reject_missing_scales_and_shared_tables():
+    # host-side checks of the FP8 entry points; nothing is launched
+    fake = torch.zeros(16, dtype=torch.uint8)
+    p = lambda: ctypes.c_void_p(fake.data_ptr())
+    lib = sa.load_library()
+    for fn, mode in (("seg_attn_prefill_fp8", sa.MODE_PREFILL),
+                     ("seg_attn_decode_fp8", sa.MODE_DECODE)):
+        tab = build([1] if mode == sa.MODE_DECODE else [2], [[(10, 5)]], mode=mode)
+        call = lambda ks, vs, dsc: getattr(lib, fn)(p(), p(), p(), ks, vs, p(), None, p(),
+                                                    ctypes.byref(dsc), 0.1, p(), 1 << 20, None)
+        assert call(None, p(), tab.desc) == S["INVALID_ARG"]
+        assert call(p(), None, tab.desc) == S["INVALID_ARG"]
+        assert call(ctypes.c_void_p(fake.data_ptr() + 2), p(), tab.desc) == S["INVALID_ARG"]
+        shared = build([1, 1] if mode == sa.MODE_DECODE else [2, 2],
+                       [[(0, 300), (400, 5)], [(0, 300), (500, 7)]], num_slots=600,
+                       mode=mode | sa.SHARE_PREFIX)
+        assert shared.desc.shared
+        assert call(p(), p(), shared.desc) == S["UNSUPPORTED"]

@@ -116,3 +116,130 @@ def test_fp8_config4_sampled_requests():
     rows = sub["q_rows"].cuda()
     compare(out[rows], lse[rows], ref_o, ref_l, "fp8 config 4")
     assert sa.seg_attn_take_device_error() == 0
+
+
+# ----------------------------------------------------------------- prefill over the FP8 cache
+def _run_fp8_prefill(case):
+    q = case["q"].cuda()
+    hq, d = q.shape[1], q.shape[2]
+    tab = sa.SegTable.build(case["q_lens"], case["seg_starts"], case["seg_lens"],
+                            case["num_slots"], case["causal"], sa.MODE_PREFILL, hq,
+                            case["k8"].shape[1], d).to("cuda")
+    out = torch.full_like(q, float("nan"))
+    lse = torch.full(q.shape[:2], float("nan"), dtype=torch.float32, device="cuda")
+    ws = (torch.empty(tab.workspace_bytes, dtype=torch.uint8, device="cuda")
+          if tab.workspace_bytes else None)
+    sa.seg_attn_prefill_fp8(q, case["k8"].cuda(), case["v8"].cuda(), case["ks"].cuda(),
+                            case["vs"].cuda(), out, lse, tab.device, tab.desc, case["scale"], ws)
+    torch.cuda.synchronize()
+    return out, lse, tab
+
+
+def _check_fp8_prefill(case, what):
+    out, lse, tab = _run_fp8_prefill(case)
+    ref_o, ref_l = oracle.attention_fp8(case["q_lens"], case["seg_starts"], case["seg_lens"],
+                                        case["q"], case["k8"], case["v8"], case["ks"], case["vs"],
+                                        case["scale"], case["causal"])
+    compare(out, lse, ref_o, ref_l, what)
+    return tab
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("hq,hkv", [(8, 1), (16, 4), (64, 8), (8, 8)])
+@pytest.mark.parametrize("causal", [True, False])
+def test_fp8_prefill_random(d, hq, hkv, causal):
+    # chunked prefill over prior context, ragged chunks and segments, several tiles
+    case = _fp8_case(random_case(400 + d + hq + hkv + causal, batch=4, hq=hq, hkv=hkv, d=d,
+                                 causal=causal, max_k=1500, nseg_max=5))
+    _check_fp8_prefill(case, f"fp8 prefill d{d} {hq}/{hkv} causal={causal}")
+
+
+def test_fp8_prefill_full_causal_and_tiny_segments():
+    # whole-sequence causal prefill; one request cut into 1-3 slot runs so most tiles
+    # are row-gathered rather than loaded as one box
+    case = random_case(411, batch=3, hq=16, hkv=2, d=128, causal=True, max_k=700, q_mode="full")
+    g = torch.Generator().manual_seed(3)
+    s1, l1 = [], []
+    for s0, l0 in zip(case["seg_starts"][1], case["seg_lens"][1]):
+        pos = s0
+        while pos < s0 + l0:
+            step = min(int(torch.randint(1, 4, (1,), generator=g)), s0 + l0 - pos)
+            s1.append(pos)
+            l1.append(step)
+            pos += step
+    case["seg_starts"][1], case["seg_lens"][1] = s1, l1
+    _check_fp8_prefill(_fp8_case(case), "fp8 full causal, tiny segments")
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_fp8_prefill_split_items_merge(causal):
+    # a few query tiles over a long context: items split along their keys, pieces merged
+    g = torch.Generator().manual_seed(41)
+    k_len, q_len, hq, hkv, d = 20000, 64, 16, 2, 128
+    seg_lens = synth.split_uniform_cuts(k_len, 5, g)
+    S = k_len + 300
+    starts = synth.place_segments(seg_lens, S, g)
+    k = torch.full((S, hkv, d), float("nan")).to(torch.bfloat16)
+    v = k.clone()
+    for s0, l in zip(starts, seg_lens):
+        k[s0:s0 + l] = torch.randn(l, hkv, d, generator=g).to(torch.bfloat16)
+        v[s0:s0 + l] = torch.randn(l, hkv, d, generator=g).to(torch.bfloat16)
+    case = _fp8_case(dict(q=torch.randn(q_len, hq, d, generator=g).to(torch.bfloat16), k_pool=k,
+                          v_pool=v, q_lens=[q_len], seg_starts=[starts], seg_lens=[seg_lens],
+                          num_slots=S, scale=d ** -0.5, causal=causal))
+    tab = _check_fp8_prefill(case, "fp8 split items")
+    assert tab.desc.num_merge > 0
+
+
+def test_fp8_prefill_short_chunks_one_tile_items():
+    # chunks of at most 16 queries at G = 8: every item holds queries in its first
+    # query tile only, so the one-tile kernel runs
+    g = torch.Generator().manual_seed(43)
+    case = random_case(413, batch=6, hq=64, hkv=8, d=128, causal=True, max_k=3000)
+    case["q_lens"] = [int(torch.randint(1, 17, (1,), generator=g)) for _ in case["q_lens"]]
+    case["q"] = torch.randn(sum(case["q_lens"]), 64, 128, generator=g).to(torch.bfloat16)
+    tab = _check_fp8_prefill(_fp8_case(case), "fp8 short chunks")
+    assert tab.desc.num_single == tab.desc.num_work
+
+
+def test_fp8_prefill_zero_keys_and_empty_requests():
+    case = random_case(414, batch=4, hq=8, hkv=2, d=64, causal=False, max_k=300)
+    case["seg_starts"][1], case["seg_lens"][1] = [], []  # no keys: O = 0, lse = -inf
+    case["q_lens"][2] = 0
+    g = torch.Generator().manual_seed(44)
+    case["q"] = torch.randn(sum(case["q_lens"]), 8, 64, generator=g).to(torch.bfloat16)
+    _check_fp8_prefill(_fp8_case(case), "fp8 zero keys / empty request")
+
+
+def test_fp8_prefill_large_scores_trigger_rescale():
+    case = random_case(415, batch=2, hq=8, hkv=1, d=128, causal=True, max_k=800, q_mode="full")
+    case["scale"] = 0.5
+    _check_fp8_prefill(_fp8_case(case), "fp8 rescale")
+
+
+def test_fp8_prefill_config5_sampled_rows():
+    wl = synth.make_workload(5, device="cuda")
+    b = wl.batches[1]
+    k8, v8, ks, vs = synth.fp8_pools(wl.k_pool, wl.v_pool)
+    tab = sa.SegTable.build(b.q_lens, b.seg_starts, b.seg_lens, wl.num_slots, True,
+                            sa.MODE_PREFILL, wl.q_heads, wl.kv_heads, wl.head_dim).to("cuda")
+    out = torch.empty_like(b.q)
+    lse = torch.empty(b.q.shape[:2], dtype=torch.float32, device="cuda")
+    ws = (torch.empty(tab.workspace_bytes, dtype=torch.uint8, device="cuda")
+          if tab.workspace_bytes else None)
+    sa.seg_attn_prefill_fp8(b.q, k8, v8, ks, vs, out, lse, tab.device, tab.desc, wl.scale, ws)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out.float()).all()
+    wl8 = synth.Workload(config=5, name="", q_heads=wl.q_heads, kv_heads=wl.kv_heads,
+                         head_dim=wl.head_dim, num_slots=wl.num_slots, scale=wl.scale,
+                         batches=[b], k_pool=k8, v_pool=v8)
+    sub = compact_requests(wl8, b, [0])
+    g = torch.Generator().manual_seed(6)
+    toks = torch.cat([torch.tensor([0, 2047]), torch.randint(0, 2048, (14,), generator=g)])
+    heads = torch.randint(0, wl.q_heads, (toks.numel(),), generator=g)
+    ref_o, ref_l = oracle.attention_fp8(sub["q_lens"], sub["seg_starts"], sub["seg_lens"],
+                                        sub["q"], sub["k_pool"], sub["v_pool"], ks.cpu(),
+                                        vs.cpu(), wl.scale, True, rows=(toks.numpy(), heads.numpy()))
+    compare(out[toks.cuda(), heads.cuda()], lse[toks.cuda(), heads.cuda()], ref_o, ref_l,
+            "fp8 config 5 prefill")
+    assert sa.seg_attn_take_device_error() == 0

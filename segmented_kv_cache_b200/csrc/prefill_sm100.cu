@@ -100,27 +100,34 @@ __device__ __forceinline__ void bf16x8_to_f16x8(uint4& v) {
 // One tile of E4M3 codes (kTileKeys rows of D bytes, plain row-major) -> f16
 // in the 128-byte-swizzled K-major layout the tensor cores read (the layout a
 // tiled TMA load of a bf16 tile produces): row r, 16-byte chunk c of 64-column
-// half h lands at h * kHalfBytes + r * 128 + ((c ^ (r & 7)) * 16).
+// half h lands at h * kHalfBytes + r * 128 + ((c ^ (r & 7)) * 16).  Thread ct
+// owns one 16-code column j of rows r0, r0 + step, ... with step a multiple of
+// 8, so the swizzle phase r & 7 and both store offsets are fixed per thread and
+// the unrolled loop needs no address arithmetic.
 template <int D>
 __device__ __forceinline__ void widen_tile(const uint8_t* src, uint8_t* dst, int ct) {
-  constexpr int kUnits = kTileKeys * D / 16;  // 16 codes per unit
-#pragma unroll 4
-  for (int u = ct; u < kUnits; u += kConvThreads) {
-    const int r = u / (D / 16), j = u % (D / 16);
-    const uint4 w = *reinterpret_cast<const uint4*>(src + r * D + 16 * j);
-    uint4 a, b;
-    a.x = ptx::e4m3x2_to_f16x2(w.x);
-    a.y = ptx::e4m3x2_to_f16x2(w.x >> 16);
-    a.z = ptx::e4m3x2_to_f16x2(w.y);
-    a.w = ptx::e4m3x2_to_f16x2(w.y >> 16);
-    b.x = ptx::e4m3x2_to_f16x2(w.z);
-    b.y = ptx::e4m3x2_to_f16x2(w.z >> 16);
-    b.z = ptx::e4m3x2_to_f16x2(w.w);
-    b.w = ptx::e4m3x2_to_f16x2(w.w >> 16);
-    uint8_t* rowp = dst + (j >> 2) * kHalfBytes + r * 128;
-    const int c0 = (j & 3) * 2;
-    *reinterpret_cast<uint4*>(rowp + ((c0 ^ (r & 7)) << 4)) = a;
-    *reinterpret_cast<uint4*>(rowp + (((c0 + 1) ^ (r & 7)) << 4)) = b;
+  constexpr int kCols = D / 16;                   // 16-code units per row
+  constexpr int kRowStep = kConvThreads / kCols;  // 8 (d = 128) or 16 (d = 64)
+  static_assert(kRowStep % 8 == 0, "rows of one thread must share the swizzle phase");
+  const int j = ct % kCols, r0 = ct / kCols;
+  const int sw = r0 & 7, c0 = (j & 3) * 2;
+  const uint8_t* s = src + r0 * D + 16 * j;
+  uint8_t* d = dst + (j >> 2) * kHalfBytes + r0 * 128;
+  const int o0 = (c0 ^ sw) << 4, o1 = ((c0 + 1) ^ sw) << 4;
+#pragma unroll
+  for (int k = 0; k < kTileKeys / kRowStep; ++k) {
+    const uint4 w = *reinterpret_cast<const uint4*>(s + k * kRowStep * D);
+    uint4 lo, hi;
+    lo.x = ptx::e4m3x2_to_f16x2(w.x);
+    lo.y = ptx::e4m3x2_to_f16x2(w.x >> 16);
+    lo.z = ptx::e4m3x2_to_f16x2(w.y);
+    lo.w = ptx::e4m3x2_to_f16x2(w.y >> 16);
+    hi.x = ptx::e4m3x2_to_f16x2(w.z);
+    hi.y = ptx::e4m3x2_to_f16x2(w.z >> 16);
+    hi.z = ptx::e4m3x2_to_f16x2(w.w);
+    hi.w = ptx::e4m3x2_to_f16x2(w.w >> 16);
+    *reinterpret_cast<uint4*>(d + k * kRowStep * 128 + o0) = lo;
+    *reinterpret_cast<uint4*>(d + k * kRowStep * 128 + o1) = hi;
   }
 }
 

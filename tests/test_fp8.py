@@ -10,7 +10,7 @@ import oracle
 import segmented_kv_cache_b200 as sa
 from segmented_kv_cache_b200 import synth
 
-from helpers import compact_requests, compare, random_case
+from helpers import compact_requests, compare, random_case, slots_of
 
 pytestmark = pytest.mark.gpu
 
@@ -243,3 +243,19 @@ def test_fp8_prefill_config5_sampled_rows():
     compare(out[toks.cuda(), heads.cuda()], lse[toks.cuda(), heads.cuda()], ref_o, ref_l,
             "fp8 config 5 prefill")
     assert sa.seg_attn_take_device_error() == 0
+
+
+@pytest.mark.parametrize("boost", [12.0, 100.0])
+def test_fp8_prefill_late_score_jump(boost):
+    # as the bf16 case: the reference max moves mid-row; P is f16 here, so a tile
+    # whose scores jump by more than 2^15 must be redone from its own max
+    case = random_case(417, batch=1, hq=8, hkv=1, d=128, causal=True, max_k=1200, q_mode="full")
+    g = torch.Generator().manual_seed(29)
+    u = torch.randn(128, generator=g)
+    u = u / u.norm()
+    case["q"] = (case["q"].float() + 3.0 * u).to(torch.bfloat16)
+    k_len = sum(case["seg_lens"][0])
+    slots = slots_of(case["seg_starts"][0], case["seg_lens"][0])
+    for j in (k_len // 2, (3 * k_len) // 4):
+        case["k_pool"][slots[j], 0] = (boost * u).to(torch.bfloat16)
+    _check_fp8_prefill(_fp8_case(case), f"fp8 late score jump x{boost}")

@@ -7,7 +7,7 @@ import oracle
 import segmented_kv_cache_b200 as sa
 from segmented_kv_cache_b200 import synth
 
-from helpers import compact_requests, compare, random_case, run_batch, run_cuda
+from helpers import compact_requests, compare, random_case, run_batch, run_cuda, slots_of
 
 pytestmark = pytest.mark.gpu
 
@@ -125,6 +125,24 @@ def test_prefill_large_scores_trigger_rescale():
     case = random_case(24, batch=2, hq=8, hkv=1, d=128, causal=True, max_k=800, q_mode="full")
     case["scale"] = 0.5
     _check(case, "rescale")
+
+
+@pytest.mark.parametrize("boost", [12.0, 25.0, 100.0])
+def test_prefill_late_score_jump(boost):
+    # one key deep in the context aligned with a direction every query leans on: its
+    # score jumps past all earlier ones by a few to many powers of two, so the
+    # reference max moves mid-row (deferred to the next tile, or the tile is redone)
+    case = random_case(27, batch=1, hq=8, hkv=1, d=128, causal=True, max_k=1200, q_mode="full")
+    g = torch.Generator().manual_seed(28)
+    u = torch.randn(128, generator=g)
+    u = u / u.norm()
+    q = case["q"].float() + 3.0 * u
+    case["q"] = q.to(torch.bfloat16)
+    k_len = sum(case["seg_lens"][0])
+    slots = slots_of(case["seg_starts"][0], case["seg_lens"][0])
+    for j in (k_len // 2, (3 * k_len) // 4):
+        case["k_pool"][slots[j], 0] = (boost * u).to(torch.bfloat16)
+    _check(case, f"late score jump x{boost}")
 
 
 def test_decode_row_equals_last_prefill_row():

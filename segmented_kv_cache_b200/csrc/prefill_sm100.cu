@@ -482,25 +482,10 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
         mbar_arrive(q_conv);
       }
     }
-    // Causal / tail mask of tile i, applied in place in tensor memory (-inf in
-    // the columns this row must not see).  Only tiles where some row of the warp
-    // needs it pay for it; the softmax itself never compares per element.
-    auto mask_tile = [&](int i) {
-      const int kb = (kt0 + i) * kTileKeys;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t a[32];
-        tmem_ld32(tS + 32 * c, a);
-        tmem_wait_ld(a);
-#pragma unroll
-        for (int e = 0; e < 32; ++e)
-          if (kb + 32 * c + e >= vis) a[e] = 0xff800000u;  // -inf
-        tmem_st32(tS + 32 * c, a);
-      }
-      tmem_wait_st();
-    };
-    // One tile of the online softmax (S already masked where needed).
-    auto softmax_tile = [&](int i) -> bool {
+    // One tile of the online softmax.  `masked`: some row of the warp must not
+    // see some key of the tile (causal diagonal, end of the request); the mask
+    // is applied to the registers, so other tiles never compare per element.
+    auto softmax_tile = [&](int i, bool masked) -> bool {
       auto f = [](uint32_t bits) { return __uint_as_float(bits); };
       // the whole S row in registers: one round trip to tensor memory
       uint32_t sv[4][32];
@@ -508,6 +493,14 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
       for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, sv[c]);
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_wait_ld(sv[c]);
+      if (masked) {
+        const int kb = (kt0 + i) * kTileKeys;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (kb + 32 * c + e >= vis) sv[c][e] = 0xff800000u;  // -inf
+      }
       float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
       for (int c = 0; c < 4; ++c)
@@ -572,8 +565,7 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
       }
       tc_fence_after();
       const bool masked = __any_sync(0xffffffffu, (kt0 + i + 1) * kTileKeys > vis);
-      if (masked) mask_tile(i);
-      if (!softmax_tile(i)) return false;
+      if (!softmax_tile(i, masked)) return false;
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(p_full + sb);
@@ -590,6 +582,21 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
       for (int i = 0; ok && i < n_tiles; ++i) ok = run_tile(i, t, i & 1);
     }
     if (!warp_live) ok = false;  // nothing to write
+    // this row's O (fp32, D columns) in registers: every load issued, one wait
+    auto load_o = [&](uint32_t (&o)[D / 32][32]) {
+      if (n_tiles > 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) tmem_ld32(tO + 32 * c, o[c]);
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) tmem_wait_ld(o[c]);
+      } else {
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c)
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[c][e] = 0u;
+      }
+    };
     if (ok && n_tiles > 0)
       ok = __all_sync(0xffffffffu,
                       mbar_wait(o_full + t, (n_tiles - 1) & 1, abort_flag, kWaitLimitNs));
@@ -599,48 +606,34 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
       const float inv = l > 0.f ? (FP8 ? __ldg(p.v_scale + g) : 1.f) / l : 0.f;
       const int64_t prow = (int64_t)slot * kItemRows + t * kTileRows + row;
       float* po = p.part_o + prow * D;
-      if (n_tiles > 0) tc_fence_after();
+      uint32_t o[D / 32][32];
+      load_o(o);
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
-        if (n_tiles > 0) {
-          tmem_ld32(tO + 32 * c, o);
-          tmem_wait_ld(o);
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = 0u;
-        }
         if (row_valid) {
 #pragma unroll
           for (int e = 0; e < 32; e += 4)
             *reinterpret_cast<float4*>(po + 32 * c + e) =
-                make_float4(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv,
-                            __uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
+                make_float4(__uint_as_float(o[c][e]) * inv, __uint_as_float(o[c][e + 1]) * inv,
+                            __uint_as_float(o[c][e + 2]) * inv, __uint_as_float(o[c][e + 3]) * inv);
         }
       }
       if (row_valid) p.part_lse[prow] = l > 0.f ? m_ref * sl2 + log2f(l) : -INFINITY;
     } else if (ok) {
       const float inv = l > 0.f ? (FP8 ? __ldg(p.v_scale + g) : 1.f) / l : 0.f;
       __nv_bfloat16* orow = p.out + ((int64_t)(tok0 + qi) * p.q_heads + head) * D;
-      if (n_tiles > 0) tc_fence_after();
+      uint32_t o[D / 32][32];
+      load_o(o);
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
-        if (n_tiles > 0) {
-          tmem_ld32(tO + 32 * c, o);
-          tmem_wait_ld(o);
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = 0u;
-        }
         if (row_valid) {
 #pragma unroll
           for (int e = 0; e < 32; e += 8) {
             uint4 v;
-            v.x = pack_bf16(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv);
-            v.y = pack_bf16(__uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
-            v.z = pack_bf16(__uint_as_float(o[e + 4]) * inv, __uint_as_float(o[e + 5]) * inv);
-            v.w = pack_bf16(__uint_as_float(o[e + 6]) * inv, __uint_as_float(o[e + 7]) * inv);
+            v.x = pack_bf16(__uint_as_float(o[c][e]) * inv, __uint_as_float(o[c][e + 1]) * inv);
+            v.y = pack_bf16(__uint_as_float(o[c][e + 2]) * inv, __uint_as_float(o[c][e + 3]) * inv);
+            v.z = pack_bf16(__uint_as_float(o[c][e + 4]) * inv, __uint_as_float(o[c][e + 5]) * inv);
+            v.w = pack_bf16(__uint_as_float(o[c][e + 6]) * inv, __uint_as_float(o[c][e + 7]) * inv);
             *reinterpret_cast<uint4*>(orow + 32 * c + e) = v;
           }
         }

@@ -466,14 +466,16 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
     bool ok = true;
     if (FP8 && n_tiles > 0) {
       // this thread's query row of tile t: bf16 -> f16 in place (elementwise, so
-      // the swizzled order of the 16-byte chunks within the row does not matter)
+      // the order of the row's 16-byte chunks does not matter; visiting chunk
+      // c ^ (row & 7) spreads a warp's 32 rows over all shared-memory banks)
       ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, abort_flag, kWaitLimitNs));
       if (ok) {
 #pragma unroll
         for (int h = 0; h < HALVES; ++h)
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
-            uint4* chunk = reinterpret_cast<uint4*>(sQ + t * TILE + h * kHalfBytes + row * 128 + c * 16);
+            uint4* chunk = reinterpret_cast<uint4*>(sQ + t * TILE + h * kHalfBytes + row * 128 +
+                                                    ((c ^ (row & 7)) << 4));
             uint4 v = *chunk;
             bf16x8_to_f16x8(v);
             *chunk = v;
@@ -597,6 +599,12 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
           for (int e = 0; e < 32; ++e) o[c][e] = 0u;
       }
     };
+    // S of the last tile ready proves PV complete up to tile n - 2, or only up to
+    // n - 3 with the two S buffers of one query tile: then wait for O phase n - 2
+    // first, since a parity wait tells apart just two consecutive phases
+    if (ok && single && n_tiles > 1)
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait(o_full + t, (n_tiles - 2) & 1, abort_flag, kWaitLimitNs));
     if (ok && n_tiles > 0)
       ok = __all_sync(0xffffffffu,
                       mbar_wait(o_full + t, (n_tiles - 1) & 1, abort_flag, kWaitLimitNs));

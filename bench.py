@@ -455,7 +455,8 @@ def run_ours(args):
         achieved = dominant[2] / (dominant[1] * 1e-3) / 1e12
         peak = peaks["bf16_tflops_sustained"]
         fp8 = args.kv_dtype == "fp8"
-        traffic = None if fp8 else profiled_traffic("prefill_sm100", f"cfg{wl.config}")
+        traffic = profiled_traffic("prefill_fp8_sm100" if fp8 else "prefill_sm100",
+                                   f"cfg{wl.config}")
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": traffic,
                 "kernel": "prefill_kernel<128> (E4M3 cache)" if fp8 else "prefill_kernel<128>",

@@ -359,7 +359,7 @@ extern "C" int seg_attn_build_table(int batch, const int32_t* q_lens, const int3
     plan_pieces(items, segattn::kMaxSplit, citems, main_pieces);
     main_citem = main_pieces.citem;
   } else {
-    int64_t L = 2048;
+    int64_t L = 4096;
     auto ctas = [&](int64_t len) {
       int64_t n = 0;
       for (int r = 0; r < batch; ++r) n += std::max<int64_t>(1, (okl[r] + len - 1) / len);

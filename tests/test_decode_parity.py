@@ -82,8 +82,8 @@ def test_decode_ragged_chunk_tails_and_tiny_segments():
 
 def test_decode_split_choice_does_not_change_result():
     # alone, the request is cut into 256-key chunks and merged; as one of 1200 copies
-    # sharing its (read-only) segments (1200 CTAs at 2048-key chunks, more than the
-    # planner's 8 x 148 target) the planner keeps 2048-key chunks, so the same
+    # sharing its (read-only) segments (1200 CTAs at 4096-key chunks, more than the
+    # planner's 8 x 148 target) the planner keeps 4096-key chunks, so the same
     # request takes the single-chunk path
     case = random_case(10, batch=1, hq=8, hkv=1, d=128, causal=True, max_k=2000, q_mode="decode")
     c = _dev(case)

@@ -97,6 +97,7 @@ __global__ void __launch_bounds__(kThreads) la_chunk_state_kernel(
   __shared__ volatile int abort_flag;
   __shared__ float g2[kChunk], warp_sum[4];
 
+  grid_launch_dependents();  // the scan may launch now; it waits for this grid's results
   const int c = blockIdx.x, h = blockIdx.y;
   const int4 ch = p.tab.chunks[c];
   const int row0 = ch.y, len = ch.z;
@@ -201,6 +202,10 @@ __global__ void __launch_bounds__(kThreads) la_chunk_state_kernel(
 // One CTA per (request, head, 1024-element slice of the state); each thread
 // carries 4 consecutive elements through the request's chunks in fp32.
 __global__ void __launch_bounds__(256) la_scan_kernel(const Params p) {
+  // the output pass may launch now (it waits for this grid before it reads the
+  // entering states); this pass needs every U of the state pass
+  grid_launch_dependents();
+  grid_dependency_wait();
   const int r = blockIdx.x / p.heads, h = blockIdx.x % p.heads;
   const int e = (blockIdx.y * 256 + threadIdx.x) * 4;
   const int in = __ldg(p.tab.in_slot + r), out = __ldg(p.tab.out_slot + r);
@@ -267,13 +272,11 @@ __global__ void __launch_bounds__(kThreads) la_chunk_out_kernel(
   if (warp == 0) {
     if (lane == 0) {
       mbar_expect_tx(&qk_full, 2 * kTile);
-      mbar_expect_tx(&s_full, kTile);
       mbar_expect_tx(&v_full, kTile);
       for (int hh = 0; hh < 2; ++hh) {
         tma_load_3d(sQ + hh * kHalf, &tm_q, &qk_full, 64 * hh, h, row0);
         tma_load_3d(sK + hh * kHalf, &tm_k, &qk_full, 64 * hh, h, row0);
       }
-      for (int hh = 0; hh < 2; ++hh) tma_load_3d(sS + hh * kHalf, &tm_s, &s_full, 64 * hh, 0, unit);
       for (int hh = 0; hh < 2; ++hh) tma_load_3d(sV + hh * kHalf, &tm_v, &v_full, 64 * hh, h, row0);
       const uint32_t qa = smem_u32(sQ), ka = smem_u32(sK), va = smem_u32(sV), sa = smem_u32(sS);
       constexpr uint32_t id_qk = idesc_bf16_f32(128, 128, false);  // B = K, K-major
@@ -289,6 +292,12 @@ __global__ void __launch_bounds__(kThreads) la_chunk_out_kernel(
         }
         mma_commit(&qk_done);
       }
+      // Only the entering state comes from the scan: everything above (and the
+      // math warps' P) runs while the scan is still going when this grid was
+      // launched as its programmatic dependent.
+      grid_dependency_wait();
+      mbar_expect_tx(&s_full, kTile);
+      for (int hh = 0; hh < 2; ++hh) tma_load_3d(sS + hh * kHalf, &tm_s, &s_full, 64 * hh, 0, unit);
       ok = ok && mbar_wait(&s_full, 0, &abort_flag, kWaitNs);
       if (ok) {
         tc_fence_after();
@@ -450,9 +459,25 @@ int launch_la_prefill(const Launch& a, cudaStream_t stream) {
     const dim3 grid(d.num_chunks, d.heads);
     la_chunk_state_kernel<<<grid, kThreads, smem1, stream>>>(tk, tv, p);
     if (cudaGetLastError() != cudaSuccess) return SEG_ATTN_ERR_CUDA;
-    la_scan_kernel<<<dim3(d.batch * d.heads, kDim * kDim / 1024), 256, 0, stream>>>(p);
-    if (cudaGetLastError() != cudaSuccess) return SEG_ATTN_ERR_CUDA;
-    la_chunk_out_kernel<<<grid, kThreads, smem3, stream>>>(tq, tk, tv, ts, p);
+    // the scan and the output pass are programmatic dependents of the pass before
+    // them: each launches while its predecessor still runs and waits for it only
+    // where it reads that predecessor's results
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.stream = stream;
+    cfg.attrs = pdl;
+    cfg.numAttrs = 1;
+    cfg.gridDim = dim3(d.batch * d.heads, kDim * kDim / 1024);
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = 0;
+    if (cudaLaunchKernelEx(&cfg, la_scan_kernel, p) != cudaSuccess) return SEG_ATTN_ERR_CUDA;
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem3;
+    if (cudaLaunchKernelEx(&cfg, la_chunk_out_kernel, tq, tk, tv, ts, p) != cudaSuccess)
+      return SEG_ATTN_ERR_CUDA;
   } else if (d.batch > 0) {
     // no tokens: the scan still moves every state from its input to its output slot
     la_scan_kernel<<<dim3(d.batch * d.heads, kDim * kDim / 1024), 256, 0, stream>>>(p);

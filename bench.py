@@ -368,9 +368,6 @@ def run_ours(args):
     wl = synth.make_workload(args.config, device=str(device), seed=rank_seed(args.config, rank),
                              context_scale=args.context_scale)
     share = args.share_prefix if args.share_prefix is not None else wl.config in (6, 7)
-    if share and args.kv_dtype == "fp8":
-        raise SystemExit("shared-prefix tables run the bf16 tensor-core prefix pass; "
-                         "use --kv-dtype bf16 or --no-share-prefix")
     path = Path(wl, device, args.kv_dtype, share)
     stream = torch.cuda.current_stream(device)
 

@@ -324,8 +324,10 @@ int seg_attn_kv_append(const void* k_new, const void* v_new, const int32_t* slot
  *                   aligned); the cached value is code * k_scale[g] (v_scale[g])
  *   k_scale, v_scale  device fp32 [kv_heads], per-kv-head dequantisation scales
  * Queries stay bf16 (used as f16 in the products: |q| must stay below 65504);
- * out / lse / table / workspace exactly as seg_attn_decode.  Half the HBM
- * bytes of the bf16 cache.
+ * out / lse / table / workspace exactly as seg_attn_decode, shared-prefix
+ * tables included (their prefix pass runs the FP8 prefill kernel).  Half the
+ * HBM bytes of the bf16 cache.  Missing or misaligned scales return
+ * SEG_ATTN_ERR_INVALID_ARG.
  */
 int seg_attn_decode_fp8(const void* q, const void* k_pool, const void* v_pool, const float* k_scale,
                         const float* v_scale, void* out, float* lse, const void* dev_table,
@@ -342,9 +344,9 @@ int seg_attn_decode_fp8(const void* q, const void* k_pool, const void* v_pool, c
  * Computes exactly what seg_attn_prefill computes on the dequantised pools, up
  * to rounding: every product is f16 x f16 -> fp32 (codes widen exactly; queries
  * become f16, so |q| must stay below 65504 and values under 2^-14 lose bits;
- * P is f16).  out / lse / table / workspace exactly as seg_attn_prefill.  A
- * shared-prefix table (SEG_ATTN_SHARE_PREFIX) returns SEG_ATTN_ERR_UNSUPPORTED;
- * missing or misaligned scales return SEG_ATTN_ERR_INVALID_ARG.
+ * P is f16).  out / lse / table / workspace exactly as seg_attn_prefill,
+ * shared-prefix tables (SEG_ATTN_SHARE_PREFIX) included.  Missing or
+ * misaligned scales return SEG_ATTN_ERR_INVALID_ARG.
  */
 int seg_attn_prefill_fp8(const void* q, const void* k_pool, const void* v_pool,
                          const float* k_scale, const float* v_scale, void* out, float* lse,

@@ -32,8 +32,10 @@ int check_common(const void* q, const void* k_pool, const void* v_pool, const vo
 
 char* at(void* base, size_t off) { return static_cast<char*>(base) + off; }
 
-// The pass over the shared prefixes (prefill kernel, every piece a partial).
-int launch_group_pass(const void* q, const void* k_pool, const void* v_pool, const void* dev_table,
+// The pass over the shared prefixes (prefill kernel, every piece a partial; on
+// an FP8 cache the FP8 prefill kernel with the same scales as the rest).
+int launch_group_pass(const void* q, const void* k_pool, const void* v_pool, const float* k_scale,
+                      const float* v_scale, bool fp8, const void* dev_table,
                       const seg_attn_table_desc& desc, const segattn::WorkspaceLayout& ws_at,
                       void* workspace, float scale, cudaStream_t stream) {
   if (desc.num_group_work == 0) return SEG_ATTN_OK;
@@ -49,6 +51,9 @@ int launch_group_pass(const void* q, const void* k_pool, const void* v_pool, con
   a.scale = scale;
   a.part_o = reinterpret_cast<float*>(at(workspace, ws_at.group_o));
   a.part_lse = reinterpret_cast<float*>(at(workspace, ws_at.group_lse));
+  a.fp8 = fp8;
+  a.k_scale = k_scale;
+  a.v_scale = v_scale;
   return segattn::launch_prefill(a, stream);
 }
 
@@ -78,8 +83,6 @@ int prefill_common(const void* q, const void* k_pool, const void* v_pool, const 
   int rc = check_common(q, k_pool, v_pool, out, lse, dev_table, desc, softmax_scale,
                         SEG_ATTN_MODE_PREFILL);
   if (rc != SEG_ATTN_OK) return rc;
-  // shared-prefix plans run their prefix pass on the bf16 cache only
-  if (fp8 && desc->shared) return SEG_ATTN_ERR_UNSUPPORTED;
   if (fp8 && desc->total_k > 0 &&
       (!k_scale || !v_scale || (reinterpret_cast<uintptr_t>(k_scale) & 3) ||
        (reinterpret_cast<uintptr_t>(v_scale) & 3)))
@@ -91,7 +94,8 @@ int prefill_common(const void* q, const void* k_pool, const void* v_pool, const 
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   const segattn::WorkspaceLayout ws_at = segattn::workspace_layout(*desc, false);
   if (desc->shared) {
-    rc = launch_group_pass(q, k_pool, v_pool, dev_table, *desc, ws_at, workspace, softmax_scale, st);
+    rc = launch_group_pass(q, k_pool, v_pool, k_scale, v_scale, fp8, dev_table, *desc, ws_at,
+                           workspace, softmax_scale, st);
     if (rc != SEG_ATTN_OK) return rc;
   }
   if (desc->num_work > 0) {
@@ -145,8 +149,6 @@ int decode_common(const void* q, const void* k_pool, const void* v_pool, const f
   int rc = check_common(q, k_pool, v_pool, out, lse, dev_table, desc, softmax_scale,
                         SEG_ATTN_MODE_DECODE);
   if (rc != SEG_ATTN_OK) return rc;
-  // the pass over shared prefixes runs on the bf16 tensor-core prefill kernel
-  if (fp8 && desc->shared) return SEG_ATTN_ERR_UNSUPPORTED;
   if (fp8 && desc->total_k > 0 &&
       (!k_scale || !v_scale || (reinterpret_cast<uintptr_t>(k_scale) & 3) ||
        (reinterpret_cast<uintptr_t>(v_scale) & 3)))
@@ -159,7 +161,8 @@ int decode_common(const void* q, const void* k_pool, const void* v_pool, const f
   const segattn::WorkspaceLayout ws_at =
       segattn::workspace_layout(*desc, desc->workspace_bytes > 0);
   if (desc->shared) {
-    rc = launch_group_pass(q, k_pool, v_pool, dev_table, *desc, ws_at, workspace, softmax_scale, st);
+    rc = launch_group_pass(q, k_pool, v_pool, k_scale, v_scale, fp8, dev_table, *desc, ws_at,
+                           workspace, softmax_scale, st);
     if (rc != SEG_ATTN_OK) return rc;
   }
   segattn::DecodeLaunch a;

@@ -10,7 +10,7 @@ import oracle
 import segmented_kv_cache_b200 as sa
 from segmented_kv_cache_b200 import synth
 
-from helpers import compact_requests, compare, random_case, slots_of
+from helpers import compact_requests, compare, random_case, shared_case, shared_values, slots_of
 
 pytestmark = pytest.mark.gpu
 
@@ -259,3 +259,63 @@ def test_fp8_prefill_late_score_jump(boost):
     for j in (k_len // 2, (3 * k_len) // 4):
         case["k_pool"][slots[j], 0] = (boost * u).to(torch.bfloat16)
     _check_fp8_prefill(_fp8_case(case), f"fp8 late score jump x{boost}")
+
+
+# ----------------------------------------------------------------- shared prefixes, FP8 cache
+def _run_fp8_any(case, decode, share):
+    q = case["q"].cuda()
+    hq, d = q.shape[1], q.shape[2]
+    mode = (sa.MODE_DECODE if decode else sa.MODE_PREFILL) | (sa.SHARE_PREFIX if share else 0)
+    tab = sa.SegTable.build(None if decode else case["q_lens"], case["seg_starts"],
+                            case["seg_lens"], case["num_slots"], True, mode, hq,
+                            case["k8"].shape[1], d).to("cuda")
+    out = torch.full_like(q, float("nan"))
+    lse = torch.full(q.shape[:2], float("nan"), dtype=torch.float32, device="cuda")
+    ws = (torch.empty(tab.workspace_bytes, dtype=torch.uint8, device="cuda")
+          if tab.workspace_bytes else None)
+    fn = sa.seg_attn_decode_fp8 if decode else sa.seg_attn_prefill_fp8
+    fn(q, case["k8"].cuda(), case["v8"].cuda(), case["ks"].cuda(), case["vs"].cuda(), out, lse,
+       tab.device, tab.desc, case["scale"], ws)
+    torch.cuda.synchronize()
+    assert sa.seg_attn_take_device_error() == 0
+    return out, lse, tab
+
+
+def _check_fp8_shared(case, decode, what):
+    out, lse, tab = _run_fp8_any(case, decode, True)
+    assert tab.desc.shared == 1, what
+    ref_o, ref_l = oracle.attention_fp8(case["q_lens"], case["seg_starts"], case["seg_lens"],
+                                        case["q"], case["k8"], case["v8"], case["ks"], case["vs"],
+                                        case["scale"], True)
+    compare(out, lse, ref_o, ref_l, what)
+    # every row against the unshared FP8 path (same products, other partial sums)
+    out_u, lse_u, _ = _run_fp8_any(case, decode, False)
+    assert (out.float() - out_u.float()).abs().max() <= 2 ** -7, what
+    fin = torch.isfinite(lse_u)
+    assert torch.equal(torch.isfinite(lse), fin), what
+    assert (lse[fin] - lse_u[fin]).abs().max() <= 1e-4, what
+    return tab
+
+
+@pytest.mark.parametrize("seed", [0, 4])
+@pytest.mark.parametrize("decode", [True, False])
+def test_fp8_shared_prefix_random(seed, decode):
+    reqs, q, S = shared_case(seed, B=8, decode=decode, max_prefix=5000)
+    case = _fp8_case(shared_values(reqs, q, S, 64, 8, 128, seed=seed + 17))
+    _check_fp8_shared(case, decode, f"fp8 shared {'decode' if decode else 'prefill'} s{seed}")
+
+
+def test_fp8_shared_decode_group_wider_than_one_item():
+    # 40 members x 8 heads = 320 packed rows: the prefix pass has two 256-row items
+    rnd = np.random.default_rng(1)
+    prefix = 5000
+    pre = [(0, prefix // 3), (prefix // 3 + 50, prefix - prefix // 3)]
+    nxt = prefix + 100
+    reqs = []
+    for _ in range(40):
+        own = int(rnd.integers(1, 701))
+        reqs.append(([s for s, _ in pre] + [nxt], [l for _, l in pre] + [own]))
+        nxt += own + int(rnd.integers(0, 9))
+    case = _fp8_case(shared_values(reqs, [1] * 40, nxt + 10, 64, 8, 128, seed=3))
+    tab = _check_fp8_shared(case, True, "fp8 shared decode, 40 members")
+    assert tab.desc.num_group_work > 2 * tab.desc.kv_heads

@@ -234,6 +234,17 @@ int seg_attn_decode(const void* q, const void* k_pool, const void* v_pool, void*
 int seg_attn_take_device_error(int* value);
 
 /*
+ * seg_attn_wait_selftest -- diagnostic (no counterpart on the source pages):
+ * launches one warp on `stream` that waits, with the bounded wait every kernel
+ * of this library uses, on an mbarrier nothing ever arrives on.  The wait gives
+ * up after wait_us microseconds (1 .. 1000000) and sets bit 0 of the device
+ * error word, which seg_attn_take_device_error then reports; the GPU context
+ * stays usable.  For checking that a stalled kernel surfaces as an error
+ * status instead of a hang.  wait_us out of range: SEG_ATTN_ERR_INVALID_ARG.
+ */
+int seg_attn_wait_selftest(int wait_us, void* stream);
+
+/*
  * seg_attn_decode_noalloc -- seg_attn_decode for callers that cannot allocate
  * device memory (no counterpart on the source pages; this is a library
  * convenience).  Typical callers: a plugin inside another runtime that owns

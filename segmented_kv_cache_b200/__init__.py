@@ -21,7 +21,7 @@ from ._build import LIB as LIB_PATH
 __all__ = [
     "SegAttnError", "seg_attn_table_desc", "seg_attn_build_table", "seg_attn_workspace_size",
     "seg_attn_prefill", "seg_attn_decode", "seg_attn_status_string", "seg_attn_version",
-    "seg_attn_take_device_error", "SegTable", "load_library", "LIB_PATH",
+    "seg_attn_take_device_error", "seg_attn_wait_selftest", "SegTable", "load_library", "LIB_PATH",
     "MODE_PREFILL", "MODE_DECODE", "STATUS", "SegPool", "seg_attn_kv_append",
     "seg_attn_decode_fp8", "seg_attn_prefill_fp8", "seg_attn_kv_append_fp8", "SHARE_PREFIX",
     "seg_la_table_desc", "seg_la_build_table", "seg_la_workspace_size", "seg_la_prefill",
@@ -126,6 +126,8 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         lib.seg_attn_version.restype = I
         lib.seg_attn_take_device_error.argtypes = [ctypes.POINTER(ctypes.c_int)]
         lib.seg_attn_take_device_error.restype = I
+        lib.seg_attn_wait_selftest.argtypes = [I, P]
+        lib.seg_attn_wait_selftest.restype = I
         PP = ctypes.POINTER(ctypes.c_void_p)
         lib.seg_attn_pool_create.argtypes = [I64, PP]
         lib.seg_attn_pool_destroy.argtypes = [P]
@@ -233,6 +235,14 @@ def seg_attn_decode(q, k_pool, v_pool, out, lse, dev_table, desc, softmax_scale,
     """Launch split-K decode attention on ``stream`` (default: torch's current stream)."""
     _compute("seg_attn_decode", q, k_pool, v_pool, out, lse, dev_table, desc, softmax_scale,
              workspace, stream)
+
+
+def seg_attn_wait_selftest(wait_us: int, stream=None) -> None:
+    """Launch the bounded-wait diagnostic: a wait that nothing completes gives up after
+    ``wait_us`` and sets bit 0 of the device error word."""
+    rc = load_library().seg_attn_wait_selftest(int(wait_us), _stream_ptr(stream))
+    if rc != 0:
+        raise SegAttnError("seg_attn_wait_selftest", rc)
 
 
 def seg_attn_take_device_error() -> int:

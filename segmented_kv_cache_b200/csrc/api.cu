@@ -207,6 +207,11 @@ extern "C" int seg_attn_decode_fp8(const void* q, const void* k_pool, const void
                        softmax_scale, workspace, workspace_bytes, stream);
 }
 
+extern "C" int seg_attn_wait_selftest(int wait_us, void* stream) {
+  if (wait_us < 1 || wait_us > 1000000) return SEG_ATTN_ERR_INVALID_ARG;
+  return segattn::launch_wait_selftest(wait_us, static_cast<cudaStream_t>(stream));
+}
+
 extern "C" int seg_attn_take_device_error(int* value) {
   if (!value) return SEG_ATTN_ERR_INVALID_ARG;
   int wait_err = 0, append_err = 0;

@@ -822,6 +822,34 @@ int launch_prefill(const PrefillLaunch& a, cudaStream_t stream) {
                                  : launch_prefill_d<64, false>(a, stream);
 }
 
+namespace {
+
+// Diagnostic: one warp waits, with the same bounded wait every kernel of this
+// library uses, on an mbarrier that nothing ever arrives on.  The wait gives up
+// after limit_ns and the grid records it in the device error word, as a stalled
+// prefill or linear-attention kernel would.
+__global__ void __launch_bounds__(32) wait_selftest_kernel(uint64_t limit_ns) {
+  using namespace ptx;
+  __shared__ uint64_t bar;
+  __shared__ volatile int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncwarp();
+  const bool done = mbar_wait(&bar, 0, &abort_flag, limit_ns);
+  __syncwarp();
+  if (threadIdx.x == 0 && (!done || abort_flag)) atomicOr(&g_device_error, 1);
+}
+
+}  // namespace
+
+int launch_wait_selftest(int wait_us, cudaStream_t stream) {
+  wait_selftest_kernel<<<1, 32, 0, stream>>>((uint64_t)wait_us * 1000ull);
+  return cudaGetLastError() == cudaSuccess ? SEG_ATTN_OK : SEG_ATTN_ERR_CUDA;
+}
+
 int take_device_error(int* value) {
   int v = 0;
   if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int)) != cudaSuccess) return SEG_ATTN_ERR_CUDA;

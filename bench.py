@@ -319,6 +319,20 @@ def oracle_sample(wl, leg_batches, budget_rows, rng_seed=0):
 
 
 # ----------------------------------------------------------------------------- main arms
+def arm_config(wl, args, world, share):
+    """The `config` object of the JSON line, the same for both arms."""
+    pool_bytes = 2 * wl.k_pool.numel() * 2
+    return {"workload": workload_name(wl) + ("" if args.context_scale == 1.0 else
+                                             f" (context x{args.context_scale})"),
+            "seed": wl.config - 1,
+            "q_heads": wl.q_heads, "kv_heads": wl.kv_heads, "head_dim": wl.head_dim,
+            "num_slots": wl.num_slots,
+            "l2": ("inputs larger than L2 (pools %.1f GB), no flush" % (pool_bytes / 1e9))
+            if pool_bytes > L2_BYTES else "inputs fit in L2",
+            "parallelism": f"dp{world} (independent batches per GPU)",
+            "share_prefix": bool(share), "kv_cache": args.kv_dtype}
+
+
 def run_reference(args):
     """The oracle as it stands, timed on the host cores, on bounded samples of the workload."""
     rank = int(os.environ.get("RANK", "0"))
@@ -341,7 +355,9 @@ def run_reference(args):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * sec / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": workload_name(wl), "seed": wl.config - 1},
+            "config": arm_config(wl, args, int(os.environ.get("WORLD_SIZE", "1")),
+                                 args.share_prefix if args.share_prefix is not None
+                                 else wl.config in (6, 7)),
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                              "sample": f"per step: {sample_desc}"},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -474,16 +490,7 @@ def run_ours(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if args.kv_dtype == "bf16" else "e4m3 cache, f16 products",
             "data": "synthetic",
-            "config": {"workload": workload_name(wl) + ("" if args.context_scale == 1.0 else
-                                                       f" (context x{args.context_scale})"),
-                       "seed": wl.config - 1,
-                       "q_heads": wl.q_heads, "kv_heads": wl.kv_heads, "head_dim": wl.head_dim,
-                       "num_slots": wl.num_slots,
-                       "l2": ("inputs larger than L2 (pools %.1f GB), no flush" %
-                              (2 * wl.k_pool.numel() * 2 / 1e9))
-                       if 2 * wl.k_pool.numel() * 2 > L2_BYTES else "inputs fit in L2",
-                       "parallelism": f"dp{world} (independent batches per GPU)",
-                       "share_prefix": bool(share), "kv_cache": args.kv_dtype},
+            "config": arm_config(wl, args, world, share),
             "legs": legs, "roofline": roof,
             "gpu_launches": path.launches_per_step() * args.steps,
             "clocks": clocks}

@@ -447,15 +447,12 @@ int launch_la_prefill(const Launch& a, cudaStream_t stream) {
         !encode3(&tv, a.v, d.heads, d.total_q, false) || !encode3(&ts, p.s_in, kDim, units, true))
       return SEG_ATTN_ERR_CUDA;
     constexpr int smem1 = 2 * kTile + 1024, smem3 = 4 * kTile + 1024;
-    static std::once_flag attr_once;
-    static bool attr_ok = false;
-    std::call_once(attr_once, [] {
-      attr_ok = cudaFuncSetAttribute(la_chunk_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     smem1) == cudaSuccess &&
-                cudaFuncSetAttribute(la_chunk_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     smem3) == cudaSuccess;
-    });
-    if (!attr_ok) return SEG_ATTN_ERR_CUDA;
+    // function attributes are per device: set them for the current one on every call
+    if (cudaFuncSetAttribute(la_chunk_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem1) != cudaSuccess ||
+        cudaFuncSetAttribute(la_chunk_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem3) != cudaSuccess)
+      return SEG_ATTN_ERR_CUDA;
     const dim3 grid(d.num_chunks, d.heads);
     la_chunk_state_kernel<<<grid, kThreads, smem1, stream>>>(tk, tv, p);
     if (cudaGetLastError() != cudaSuccess) return SEG_ATTN_ERR_CUDA;

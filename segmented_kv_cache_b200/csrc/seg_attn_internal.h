@@ -14,7 +14,7 @@ constexpr int kTilesPerItem = 2; // M-tiles sharing each K/V tile in one prefill
 constexpr int kSmCount = 148;    // B200
 constexpr int kItemRows = kTileRows * kTilesPerItem;  // query rows of one prefill item
 constexpr int kMinPieceTiles = 8;       // shortest K range a split prefill piece gets
-constexpr int kPieceOverheadTiles = 2;  // per-piece cost (prologue, epilogue) in K tiles
+constexpr int kPieceOverheadTiles = 3;  // per-piece cost (prologue, epilogue) in K tiles (traced: ~12 k cycles)
 constexpr int kMaxSplit = 4;            // most pieces one prefill item is cut into
 constexpr int kMaxGroupSplit = 32;      // the same for a pass over a shared prefix
 constexpr int kMinSharedKeys = 256;     // shortest prefix worth a pass of its own

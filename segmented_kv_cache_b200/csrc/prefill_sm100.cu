@@ -75,11 +75,19 @@ struct PrefillParams {
 // Q (2 tiles) + K ring (2) + V ring (2) + barriers + alignment slack.  The
 // d = 64 variant asks for more than half the SM's shared memory as well, so
 // one CTA owns an SM and its 512 tensor-memory columns.
+// K/V ring depth: the one-tile bf16 kernel spends the second query tile's
+// space on a third K and V stage; every other variant keeps two.
+template <bool SINGLE, bool FP8>
+constexpr int ring_stages() {
+  return SINGLE && !FP8 ? 3 : 2;
+}
+
 // The FP8 variant adds one staging tile of raw codes each for K and V.
-template <int D, bool FP8>
+template <int D, bool SINGLE, bool FP8>
 constexpr size_t prefill_smem_bytes() {
-  constexpr size_t need =
-      6 * (D / 64) * (size_t)kHalfBytes + (FP8 ? 2 * kTileKeys * D : 0) + 256 + 1024;
+  constexpr size_t need = ((SINGLE ? 1 : 2) + 2 * ring_stages<SINGLE, FP8>()) * (D / 64) *
+                              (size_t)kHalfBytes +
+                          (FP8 ? 2 * kTileKeys * D : 0) + 256 + 1024;
   return need < 120 * 1024 ? 120 * 1024 : need;
 }
 
@@ -151,27 +159,28 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
+  constexpr int RING = ring_stages<SINGLE, FP8>();
   uint8_t* sQ = sm;
-  uint8_t* sK = sm + 2 * TILE;
-  uint8_t* sV = sm + 4 * TILE;
-  uint8_t* sStK = sm + 6 * TILE;            // FP8: raw code tile of K
+  uint8_t* sK = sm + (SINGLE ? 1 : 2) * TILE;
+  uint8_t* sV = sK + RING * TILE;
+  uint8_t* sStK = sV + RING * TILE;         // FP8: raw code tile of K
   uint8_t* sStV = sStK + kTileKeys * D;     // FP8: raw code tile of V
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + 6 * TILE + (FP8 ? 2 * kTileKeys * D : 0));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + RING * TILE + (FP8 ? 2 * kTileKeys * D : 0));
   uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;   // [2]
-  uint64_t* k_empty = bars + 3;  // [2]
-  uint64_t* v_full = bars + 5;   // [2]
-  uint64_t* v_empty = bars + 7;  // [2]
-  uint64_t* s_full = bars + 9;   // [2] per query tile
-  uint64_t* p_full = bars + 11;  // [2]
-  uint64_t* o_full = bars + 13;  // [2]
-  uint64_t* mma_done = bars + 15;
-  uint64_t* kst_full = bars + 16;   // FP8: code staging of K filled (TMA bytes)
-  uint64_t* kst_empty = bars + 17;  // FP8: code staging of K read by the converters
-  uint64_t* vst_full = bars + 18;
-  uint64_t* vst_empty = bars + 19;
-  uint64_t* q_conv = bars + 20;     // FP8: query tiles converted to f16
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 21);
+  uint64_t* k_full = bars + 1;    // [RING]
+  uint64_t* k_empty = bars + 4;   // [RING]
+  uint64_t* v_full = bars + 7;    // [RING]
+  uint64_t* v_empty = bars + 10;  // [RING]
+  uint64_t* s_full = bars + 13;   // [2] per query tile (S buffer)
+  uint64_t* p_full = bars + 15;   // [2]
+  uint64_t* o_full = bars + 17;   // [2]
+  uint64_t* mma_done = bars + 19;
+  uint64_t* kst_full = bars + 20;   // FP8: code staging of K filled (TMA bytes)
+  uint64_t* kst_empty = bars + 21;  // FP8: code staging of K read by the converters
+  uint64_t* vst_full = bars + 22;
+  uint64_t* vst_empty = bars + 23;
+  uint64_t* q_conv = bars + 24;     // FP8: query tiles converted to f16
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 25);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -192,12 +201,14 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < RING; ++s) {
       // FP8: the ring is filled by the converter threads, not by TMA
       mbar_init(k_full + s, FP8 ? kConvThreads : 1);
       mbar_init(k_empty + s, 1);
       mbar_init(v_full + s, FP8 ? kConvThreads : 1);
       mbar_init(v_empty + s, 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(s_full + s, 1);
       mbar_init(p_full + s, 128);
       mbar_init(o_full + s, 1);
@@ -241,8 +252,8 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
       int seg = __ldg(p.tab.seg_offsets + req);
       const int seg_end = __ldg(p.tab.seg_offsets + req + 1);
       for (int i = 0; i < n_tiles; ++i) {
-        const int st = i & 1;
-        const uint32_t ph = (i >> 1) & 1;
+        const int st = i % RING;
+        const uint32_t ph = (i / RING) & 1;
         int rows[4], slot_first = 0;
         bool run = true;
 #pragma unroll
@@ -308,14 +319,14 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
         if (k_issued > 0) mbar_wait(kst_full, (k_issued - 1) & 1, nullptr, kWaitLimitNs);
         if (v_issued > 0) mbar_wait(vst_full, (v_issued - 1) & 1, nullptr, kWaitLimitNs);
       }
-      for (int s = 0; !FP8 && s < 2; ++s) {
+      for (int s = 0; !FP8 && s < RING; ++s) {
         if (k_issued > s) {
-          const int last = s + 2 * ((k_issued - 1 - s) / 2);
-          mbar_wait(k_full + s, (last >> 1) & 1, nullptr, kWaitLimitNs);
+          const int last = s + RING * ((k_issued - 1 - s) / RING);
+          mbar_wait(k_full + s, (last / RING) & 1, nullptr, kWaitLimitNs);
         }
         if (v_issued > s) {
-          const int last = s + 2 * ((v_issued - 1 - s) / 2);
-          mbar_wait(v_full + s, (last >> 1) & 1, nullptr, kWaitLimitNs);
+          const int last = s + RING * ((v_issued - 1 - s) / RING);
+          mbar_wait(v_full + s, (last / RING) & 1, nullptr, kWaitLimitNs);
         }
       }
       if (lane == 0) mbar_wait(q_full, 0, nullptr, kWaitLimitNs);
@@ -363,21 +374,24 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
           mma_commit(s_full + 1);
           mma_commit(k_empty + 1);
         }
+        // S buffer of tile i: i & 1; its K/V ring stage: i % RING
         for (int i = 0; ok && i < n_tiles; ++i) {
-          const int b = i & 1;
+          const int b = i & 1, vs = i % RING;
           const uint32_t ph = (i >> 1) & 1;
-          if (!(ok = mbar_wait(v_full + b, ph, abort_flag, kWaitLimitNs))) break;
+          if (!(ok = mbar_wait(v_full + vs, (i / RING) & 1, abort_flag, kWaitLimitNs))) break;
           if (!(ok = mbar_wait(p_full + b, ph, abort_flag, kWaitLimitNs))) break;
           tc_fence_after();
-          issue_pv(0, b, b, i > 0);
+          issue_pv(0, b, vs, i > 0);
           mma_commit(o_full + 0);
-          mma_commit(v_empty + b);
+          mma_commit(v_empty + vs);
           if (i + 2 < n_tiles) {
-            if (!(ok = mbar_wait(k_full + b, ph ^ 1, abort_flag, kWaitLimitNs))) break;
+            const int ks = (i + 2) % RING;
+            if (!(ok = mbar_wait(k_full + ks, ((i + 2) / RING) & 1, abort_flag, kWaitLimitNs)))
+              break;
             tc_fence_after();
-            issue_qk(0, b, b);
+            issue_qk(0, b, ks);
             mma_commit(s_full + b);
-            mma_commit(k_empty + b);
+            mma_commit(k_empty + ks);
           }
         }
       } else {
@@ -737,7 +751,7 @@ template <int D, bool SINGLE, bool FP8>
 int launch_items(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                  const CUtensorMap& tk3, const CUtensorMap& tv3, const PrefillParams& p, int n,
                  cudaStream_t stream) {
-  constexpr size_t smem = prefill_smem_bytes<D, FP8>();
+  constexpr size_t smem = prefill_smem_bytes<D, SINGLE, FP8>();
   if (cudaFuncSetAttribute(prefill_kernel<D, SINGLE, FP8>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return SEG_ATTN_ERR_CUDA;

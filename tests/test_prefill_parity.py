@@ -145,6 +145,23 @@ def test_prefill_late_score_jump(boost):
     _check(case, f"late score jump x{boost}")
 
 
+@pytest.mark.parametrize("d,hq,hkv,q_max", [(128, 64, 8, 16), (64, 16, 4, 32), (128, 8, 8, 128)])
+def test_prefill_short_chunks_run_the_one_tile_kernel(d, hq, hkv, q_max):
+    # every request's chunk fits one 128-row query tile, so the whole pass runs the
+    # one-tile kernel (double-buffered S, three-stage K/V ring); long prior contexts
+    # give each item many K tiles through the ring, some of them gathered
+    g = torch.Generator().manual_seed(47 + d + hq)
+    case = random_case(416 + d + hq, batch=6, hq=hq, hkv=hkv, d=d, causal=True, max_k=5000,
+                       nseg_max=6)
+    # at most 128 / G queries per request (one query tile), never more than its keys
+    case["q_lens"] = [min(sum(l), int(torch.randint(1, q_max + 1, (1,), generator=g)))
+                      for l in case["seg_lens"]]
+    case["q"] = torch.randn(sum(case["q_lens"]), hq, d, generator=g).to(torch.bfloat16)
+    _, _, tab = _run(case)
+    assert tab.desc.num_single == tab.desc.num_work > 0
+    _check(case, f"one-tile kernel d{d} {hq}/{hkv}")
+
+
 def test_decode_row_equals_last_prefill_row():
     case = random_case(25, batch=2, hq=8, hkv=1, d=128, causal=True, max_k=600, q_mode="full")
     out, lse, _ = _run(case)

@@ -16,9 +16,10 @@
 // loaded as two tiled boxes, which the TMA engine moves far faster than 64
 // four-row gathers.
 //
-// Warp roles (10 warps):
-//   warp 0       TMA producer: Q tiles once, then a 2-stage K ring and a
-//                2-stage V ring.
+// Warp roles (10 warps; 12 over an FP8 cache, see below):
+//   warp 0       TMA producer: Q tiles once, then a K ring and a V ring of
+//                2 stages (3 in the one-tile bf16 kernel, which has the second
+//                query tile's space to spare).
 //   warp 1       TMEM allocator; lane 0 issues every tcgen05.mma:
 //                  S_t = Q_t K^T   (SS, 128x128xD, fp32 in TMEM)
 //                  O_t += P_t V    (TS: P from TMEM as bf16, V MN-major)

@@ -20,19 +20,27 @@
 //   warp 0       TMA producer: Q tiles once, then a K ring and a V ring of
 //                2 stages (3 in the one-tile bf16 kernel, which has the second
 //                query tile's space to spare).
-//   warp 1       TMEM allocator; lane 0 issues every tcgen05.mma:
-//                  S_t = Q_t K^T   (SS, 128x128xD, fp32 in TMEM)
-//                  O_t += P_t V    (TS: P from TMEM as bf16, V MN-major)
-//                in ping-pong order so one tile's softmax overlaps the other
-//                tile's MMAs.
+//   warp 1       TMEM allocator; lane 0 issues every tcgen05.mma.
 //   warps 2-5    softmax for query tile 0, warps 6-9 for tile 1: one thread
 //                per row (its TMEM lane); online softmax (running max m and
 //                normaliser l, as in the Ascend FlashAttention article,
-//                "bottleneck 2") in registers, P written back to TMEM over S,
-//                O rescaled in TMEM only when the max grows by more than 2^8
-//                (the final O / l uses the same reference max, so the result
-//                is unchanged), epilogue O / l -> bf16 and lse.
-// TMEM columns: O0 [0,128) O1 [128,256) S0/P0 [256,384) S1/P1 [384,512).
+//                "bottleneck 2") in registers, O rescaled in TMEM only when
+//                the max grows by more than 2^8 (the final O / l uses the same
+//                reference max, so the result is unchanged), epilogue O / l ->
+//                bf16 and lse.
+// Two query tiles (the usual item): the softmax threads copy their query rows
+// into tensor memory once, so
+//                  S   = Q_t K^T   (TS: Q from TMEM, K from the ring)
+//                  O_t += P_t V    (SS: P from shared memory, V MN-major)
+// and the two tiles take turns on one S buffer.  A softmax thread loads its
+// whole S row, releases the buffer (the other tile's QK can go), and writes P
+// to shared memory, so the next K tile's S of a query tile is computed while
+// this tile's softmax still runs: each tile's chain is its softmax alone, not
+// softmax + PV + QK.
+// TMEM columns: O0 [0,128) O1 [128,256) S [256,384) Q0 [384,448) Q1 [448,512).
+// One query tile (SINGLE): Q stays in shared memory (SS QK), P is written over
+// S in TMEM (TS PV) and S is double-buffered instead:
+// TMEM columns: O [0,128) S0/P0 [256,384) S1/P1 [384,512).
 // Every mbarrier wait is bounded (1 s); a timeout stops all roles of the CTA,
 // drains in-flight copies and MMAs, frees TMEM and flags a device error.
 #include <cuda.h>
@@ -58,7 +66,12 @@ constexpr int kThreadsFp8 = 384;
 constexpr int kConvThreads = 64;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
 constexpr float kRescaleLog2 = 8.0f;
+// Two tiles: a tile's softmax signals after this many 32-key chunks of its
+// current K tile that its next S may be computed; the chunks left take about
+// as long as that S takes to arrive.
+constexpr int kSoonChunks = 2;
 constexpr uint32_t kHalfBytes = 128 * 128;  // 128 rows x 64 bf16 (one swizzle-128B panel)
+constexpr uint32_t kPTile = 2 * kHalfBytes;   // P of one query tile: 128 rows x 128 keys
 
 struct PrefillParams {
   __nv_bfloat16* out;
@@ -73,23 +86,67 @@ struct PrefillParams {
   const float* v_scale;
 };
 
-// Q (2 tiles) + K ring (2) + V ring (2) + barriers + alignment slack.  The
-// d = 64 variant asks for more than half the SM's shared memory as well, so
-// one CTA owns an SM and its 512 tensor-memory columns.
-// K/V ring depth: the one-tile bf16 kernel spends the second query tile's
-// space on a third K and V stage; every other variant keeps two.
+// Query region + K ring + V ring + barriers + alignment slack.  The query
+// region is one Q tile (SINGLE) or the two P tiles, which hold the two Q tiles
+// until the softmax threads have moved them to tensor memory.  The d = 64
+// variant asks for more than half the SM's shared memory as well, so one CTA
+// owns an SM and its 512 tensor-memory columns.
+// K/V ring depths (stages of K, of V).  Over a bf16 cache the one-tile kernel
+// spends the second query tile's space on a third K and V stage, and the
+// two-tile kernel, whose query tiles live in tensor memory, on a third K
+// stage: its QK of a K tile runs a softmax ahead of the PV of the previous
+// one, so K tiles are wanted earlier than V tiles.  FP8 keeps two of each.
 template <bool SINGLE, bool FP8>
-constexpr int ring_stages() {
+constexpr int ring_k() {
+  return FP8 ? 2 : 3;
+}
+template <bool SINGLE, bool FP8>
+constexpr int ring_v() {
   return SINGLE && !FP8 ? 3 : 2;
+}
+
+template <int D, bool SINGLE>
+constexpr size_t query_region_bytes() {
+  return SINGLE ? (D / 64) * (size_t)kHalfBytes : 2 * (size_t)kPTile;
 }
 
 // The FP8 variant adds one staging tile of raw codes each for K and V.
 template <int D, bool SINGLE, bool FP8>
 constexpr size_t prefill_smem_bytes() {
-  constexpr size_t need = ((SINGLE ? 1 : 2) + 2 * ring_stages<SINGLE, FP8>()) * (D / 64) *
+  constexpr size_t need = query_region_bytes<D, SINGLE>() +
+                          (ring_k<SINGLE, FP8>() + ring_v<SINGLE, FP8>()) * (D / 64) *
                               (size_t)kHalfBytes +
                           (FP8 ? 2 * kTileKeys * D : 0) + 256 + 1024;
+  static_assert(need <= 227 * 1024, "shared memory per CTA");
   return need < 120 * 1024 ? 120 * 1024 : need;
+}
+
+// Three-input maximum (one instruction on sm_100).
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Packed fp32 pairs: one instruction does two fmaf / two adds, each rounded as
+// the scalar one would be.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -160,18 +217,21 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
-  constexpr int RING = ring_stages<SINGLE, FP8>();
+  constexpr int RK = ring_k<SINGLE, FP8>(), RV = ring_v<SINGLE, FP8>();
+  // SINGLE: the one Q tile.  Two tiles: P_t at sQ + t * kPTile, which holds Q
+  // tile t until its softmax threads have copied it to tensor memory.
+  constexpr uint32_t QSTRIDE = SINGLE ? TILE : kPTile;
   uint8_t* sQ = sm;
-  uint8_t* sK = sm + (SINGLE ? 1 : 2) * TILE;
-  uint8_t* sV = sK + RING * TILE;
-  uint8_t* sStK = sV + RING * TILE;         // FP8: raw code tile of K
+  uint8_t* sK = sm + query_region_bytes<D, SINGLE>();
+  uint8_t* sV = sK + RK * TILE;
+  uint8_t* sStK = sV + RV * TILE;           // FP8: raw code tile of K
   uint8_t* sStV = sStK + kTileKeys * D;     // FP8: raw code tile of V
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + RING * TILE + (FP8 ? 2 * kTileKeys * D : 0));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + RV * TILE + (FP8 ? 2 * kTileKeys * D : 0));
   uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;    // [RING]
-  uint64_t* k_empty = bars + 4;   // [RING]
-  uint64_t* v_full = bars + 7;    // [RING]
-  uint64_t* v_empty = bars + 10;  // [RING]
+  uint64_t* k_full = bars + 1;    // [RK]
+  uint64_t* k_empty = bars + 4;   // [RK]
+  uint64_t* v_full = bars + 7;    // [RV]
+  uint64_t* v_empty = bars + 10;  // [RV]
   uint64_t* s_full = bars + 13;   // [2] per query tile (S buffer)
   uint64_t* p_full = bars + 15;   // [2]
   uint64_t* o_full = bars + 17;   // [2]
@@ -180,8 +240,10 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
   uint64_t* kst_empty = bars + 21;  // FP8: code staging of K read by the converters
   uint64_t* vst_full = bars + 22;
   uint64_t* vst_empty = bars + 23;
-  uint64_t* q_conv = bars + 24;     // FP8: query tiles converted to f16
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 25);
+  uint64_t* q_conv = bars + 24;     // queries ready: in TMEM (two tiles), converted (FP8)
+  uint64_t* s_free = bars + 25;     // two tiles: the shared S buffer read by its softmax
+  uint64_t* s_soon = bars + 26;     // [2] two tiles: the tile's softmax is near the end of a K tile
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 28);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -202,10 +264,12 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < RING; ++s) {
-      // FP8: the ring is filled by the converter threads, not by TMA
+    // FP8: the rings are filled by the converter threads, not by TMA
+    for (int s = 0; s < RK; ++s) {
       mbar_init(k_full + s, FP8 ? kConvThreads : 1);
       mbar_init(k_empty + s, 1);
+    }
+    for (int s = 0; s < RV; ++s) {
       mbar_init(v_full + s, FP8 ? kConvThreads : 1);
       mbar_init(v_empty + s, 1);
     }
@@ -215,12 +279,15 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
       mbar_init(o_full + s, 1);
     }
     mbar_init(mma_done, 1);
+    mbar_init(s_free, 4);  // one arrival per softmax warp of the tile that read S
+    mbar_init(s_soon + 0, 128);
+    mbar_init(s_soon + 1, 128);
+    mbar_init(q_conv, (SINGLE ? 1 : 2) * 128);
     if (FP8) {
       mbar_init(kst_full, 1);
       mbar_init(kst_empty, kConvThreads);
       mbar_init(vst_full, 1);
       mbar_init(vst_empty, kConvThreads);
-      mbar_init(q_conv, (SINGLE ? 1 : 2) * 128);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -247,117 +314,181 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
         mbar_expect_tx(q_full, q_tiles * TILE);
         for (int t = 0; t < q_tiles; ++t)
           for (int h = 0; h < HALVES; ++h)
-            tma_load_3d(sQ + t * TILE + h * kHalfBytes, &tm_q, q_full, 64 * h, g * p.group,
+            tma_load_3d(sQ + t * QSTRIDE + h * kHalfBytes, &tm_q, q_full, 64 * h, g * p.group,
                         tok0 + q0 + t * p.qpt);
       }
       int seg = __ldg(p.tab.seg_offsets + req);
       const int seg_end = __ldg(p.tab.seg_offsets + req + 1);
-      for (int i = 0; i < n_tiles; ++i) {
-        const int st = i % RING;
-        const uint32_t ph = (i / RING) & 1;
-        int rows[4], slot_first = 0;
+      // Pool rows of K tile i: lane l holds logical keys 4l .. 4l + 3 (keys past the
+      // request are clamped to its last key).  Most tiles are 128 consecutive pool
+      // slots (segments are long): one tiled box per 64-column half; tiles that
+      // straddle a segment boundary or the end of the request are gathered row by
+      // row.  Tiles are visited in increasing order (the segment cursor only moves on).
+      struct TileRows {
+        int rows[4];
+        int slot0;
+        bool contiguous;
+      };
+      auto tile_rows = [&](int i, TileRows& tr) {
+        int slot_first = 0;
         bool run = true;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int j = min((kt0 + i) * kTileKeys + 4 * lane + e, k_len - 1);
           while (seg + 1 < seg_end && __ldg(p.tab.seg_kstart + seg + 1) <= j) ++seg;
           const int slot = __ldg(p.tab.seg_start + seg) + (j - __ldg(p.tab.seg_kstart + seg));
-          rows[e] = slot * p.kv_heads + g;
+          tr.rows[e] = slot * p.kv_heads + g;
           if (e == 0) slot_first = slot;
         }
-        // Most tiles are 128 consecutive pool slots (segments are long): one tiled
-        // box per 64-column half.  Tiles that straddle a segment boundary or the end
-        // of the request are gathered row by row.
-        const int slot0 = __shfl_sync(0xffffffffu, slot_first, 0);
+        tr.slot0 = __shfl_sync(0xffffffffu, slot_first, 0);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) run &= rows[e] == (slot0 + 4 * lane + e) * p.kv_heads + g;
-        const bool contiguous = __all_sync(0xffffffffu, run);
-        auto load_tile = [&](uint8_t* dst, const CUtensorMap* tiled, const CUtensorMap* rowmap,
-                             uint64_t* bar) {
-          if (lane == 0) mbar_expect_tx(bar, TILE);
-          __syncwarp();
-          if (contiguous) {
-            if (lane == 0)
-              for (int h = 0; h < HALVES; ++h)
-                tma_load_3d(dst + h * kHalfBytes, tiled, bar, 64 * h, g, slot0);
-          } else {
-#pragma unroll
+        for (int e = 0; e < 4; ++e) run &= tr.rows[e] == (tr.slot0 + 4 * lane + e) * p.kv_heads + g;
+        tr.contiguous = __all_sync(0xffffffffu, run);
+      };
+      auto load_tile = [&](const TileRows& tr, uint8_t* dst, const CUtensorMap* tiled,
+                           const CUtensorMap* rowmap, uint64_t* bar) {
+        if (lane == 0) mbar_expect_tx(bar, TILE);
+        __syncwarp();
+        if (tr.contiguous) {
+          if (lane == 0)
             for (int h = 0; h < HALVES; ++h)
-              tma_gather4(dst + h * kHalfBytes + lane * 512, rowmap, bar, 64 * h, rows[0], rows[1],
-                          rows[2], rows[3]);
-          }
-        };
-        // FP8: raw code rows (D bytes each) into the staging tile, no swizzle
-        auto load_codes = [&](uint8_t* dst, const CUtensorMap* tiled, const CUtensorMap* rowmap,
-                              uint64_t* bar) {
-          if (lane == 0) mbar_expect_tx(bar, kTileKeys * D);
-          __syncwarp();
-          if (contiguous) {
-            if (lane == 0) tma_load_3d(dst, tiled, bar, 0, g, slot0);
-          } else {
-            tma_gather4(dst + lane * 4 * D, rowmap, bar, 0, rows[0], rows[1], rows[2], rows[3]);
-          }
-        };
-        if (FP8) {
+              tma_load_3d(dst + h * kHalfBytes, tiled, bar, 64 * h, g, tr.slot0);
+        } else {
+#pragma unroll
+          for (int h = 0; h < HALVES; ++h)
+            tma_gather4(dst + h * kHalfBytes + lane * 512, rowmap, bar, 64 * h, tr.rows[0],
+                        tr.rows[1], tr.rows[2], tr.rows[3]);
+        }
+      };
+      // FP8: raw code rows (D bytes each) into the staging tile, no swizzle
+      auto load_codes = [&](const TileRows& tr, uint8_t* dst, const CUtensorMap* tiled,
+                            const CUtensorMap* rowmap, uint64_t* bar) {
+        if (lane == 0) mbar_expect_tx(bar, kTileKeys * D);
+        __syncwarp();
+        if (tr.contiguous) {
+          if (lane == 0) tma_load_3d(dst, tiled, bar, 0, g, tr.slot0);
+        } else {
+          tma_gather4(dst + lane * 4 * D, rowmap, bar, 0, tr.rows[0], tr.rows[1], tr.rows[2],
+                      tr.rows[3]);
+        }
+      };
+      auto load_k = [&](int i, const TileRows& tr) -> bool {
+        const int st = i % RK;
+        if (!__all_sync(0xffffffffu, mbar_wait(k_empty + st, ((i / RK) & 1) ^ 1, abort_flag,
+                                               kWaitLimitNs, true)))
+          return false;
+        load_tile(tr, sK + st * TILE, &tm_k3, &tm_k, k_full + st);
+        ++k_issued;
+        return true;
+      };
+      auto load_v = [&](int i, const TileRows& tr) -> bool {
+        const int st = i % RV;
+        if (!__all_sync(0xffffffffu, mbar_wait(v_empty + st, ((i / RV) & 1) ^ 1, abort_flag,
+                                               kWaitLimitNs, true)))
+          return false;
+        load_tile(tr, sV + st * TILE, &tm_v3, &tm_v, v_full + st);
+        ++v_issued;
+        return true;
+      };
+      if (FP8) {
+        // codes of K tile i, then of V tile i, through one staging tile each
+        for (int i = 0; i < n_tiles; ++i) {
+          TileRows tr;
+          tile_rows(i, tr);
           if (!__all_sync(0xffffffffu, mbar_wait(kst_empty, (i & 1) ^ 1, abort_flag, kWaitLimitNs, true))) break;
-          load_codes(sStK, &tm_k3, &tm_k, kst_full);
+          load_codes(tr, sStK, &tm_k3, &tm_k, kst_full);
           ++k_issued;
           if (!__all_sync(0xffffffffu, mbar_wait(vst_empty, (i & 1) ^ 1, abort_flag, kWaitLimitNs, true))) break;
-          load_codes(sStV, &tm_v3, &tm_v, vst_full);
+          load_codes(tr, sStV, &tm_v3, &tm_v, vst_full);
           ++v_issued;
-          continue;
         }
-        if (!__all_sync(0xffffffffu, mbar_wait(k_empty + st, ph ^ 1, abort_flag, kWaitLimitNs, true))) break;
-        load_tile(sK + st * TILE, &tm_k3, &tm_k, k_full + st);
-        ++k_issued;
-        if (!__all_sync(0xffffffffu, mbar_wait(v_empty + st, ph ^ 1, abort_flag, kWaitLimitNs, true))) break;
-        load_tile(sV + st * TILE, &tm_v3, &tm_v, v_full + st);
-        ++v_issued;
-      }
-      // never leave the CTA with copies in flight (FP8: a staged copy is issued
-      // only after the converters read the previous one, so the last is enough)
-      if (FP8) {
+        // never leave the CTA with copies in flight (a staged copy is issued only
+        // after the converters read the previous one, so the last is enough)
         if (k_issued > 0) mbar_wait(kst_full, (k_issued - 1) & 1, nullptr, kWaitLimitNs);
         if (v_issued > 0) mbar_wait(vst_full, (v_issued - 1) & 1, nullptr, kWaitLimitNs);
-      }
-      for (int s = 0; !FP8 && s < RING; ++s) {
-        if (k_issued > s) {
-          const int last = s + RING * ((k_issued - 1 - s) / RING);
-          mbar_wait(k_full + s, (last / RING) & 1, nullptr, kWaitLimitNs);
+      } else {
+        // K tile i + 1 before V tile i: the MMA warp takes them in that order
+        TileRows cur, nxt;
+        tile_rows(0, cur);
+        bool run = load_k(0, cur);
+        for (int i = 0; run && i < n_tiles; ++i) {
+          if (i + 1 < n_tiles) {
+            tile_rows(i + 1, nxt);
+            if (!(run = load_k(i + 1, nxt))) break;
+          }
+          if (!(run = load_v(i, cur))) break;
+          cur = nxt;
         }
-        if (v_issued > s) {
-          const int last = s + RING * ((v_issued - 1 - s) / RING);
-          mbar_wait(v_full + s, (last / RING) & 1, nullptr, kWaitLimitNs);
-        }
+        // never leave the CTA with copies in flight
+        for (int s = 0; s < RK; ++s)
+          if (k_issued > s) {
+            const int last = s + RK * ((k_issued - 1 - s) / RK);
+            mbar_wait(k_full + s, (last / RK) & 1, nullptr, kWaitLimitNs);
+          }
+        for (int s = 0; s < RV; ++s)
+          if (v_issued > s) {
+            const int last = s + RV * ((v_issued - 1 - s) / RV);
+            mbar_wait(v_full + s, (last / RV) & 1, nullptr, kWaitLimitNs);
+          }
       }
       if (lane == 0) mbar_wait(q_full, 0, nullptr, kWaitLimitNs);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && n_tiles > 0) {
+    // The whole warp runs the issue loop on warp-uniform values; one elected lane
+    // executes each tcgen05.mma / commit.
+    if (n_tiles > 0) {
+      auto wait_all = [&](uint64_t* bar, uint32_t parity) {
+        return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, kWaitLimitNs));
+      };
       const uint32_t idesc_qk =
           FP8 ? idesc_f16_f32(128, 128, false) : idesc_bf16_f32(128, 128, false);
       const uint32_t idesc_pv = FP8 ? idesc_f16_f32(128, D, true) : idesc_bf16_f32(128, D, true);
       const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
-      const uint32_t tS0 = tmem + 256, tO0 = tmem;
+      const uint32_t tS0 = tmem + 256, tO0 = tmem, tQ0 = tmem + 384;
+      // S buffer `sb` = Q tile `qt` . K stage `st`^T;  O tile `ot` += P (in S buffer `sb`) . V stage `st`
+      // Shared-memory descriptors are built once: a ring stage or P tile moves the
+      // start address (16-byte units, the low 14 bits) by a multiple of its size,
+      // and each 16-deep K step by a constant.  Building them per MMA inside the
+      // issue loop measured ~1.8x slower MMA issue than the tensor core's rate.
+      const uint64_t dq = sdesc_sw128(q_addr, 16, 1024), dk = sdesc_sw128(k_addr, 16, 1024);
+      const uint64_t dv = sdesc_sw128(v_addr, kHalfBytes, 1024);
+      constexpr uint32_t kTileU = TILE >> 4, kPTileU = kPTile >> 4;
+      // K-step k of a K-major operand: panel k / 4, 32 bytes per step inside it
+      auto kstep = [](int k) -> uint32_t { return ((k >> 2) * kHalfBytes + (k & 3) * 32) >> 4; };
       // S buffer `sb` = Q tile `qt` . K stage `st`^T;  O tile `ot` += P (in S buffer `sb`) . V stage `st`
       auto issue_qk = [&](int qt, int sb, int st) {
+        const uint64_t a0 = dq + qt * kTileU, b0 = dk + st * kTileU;
+        const uint32_t d = tS0 + 128 * sb;
 #pragma unroll
-        for (int k = 0; k < KSTEPS; ++k) {
-          const uint32_t off = (k >> 2) * kHalfBytes + (k & 3) * 32;
-          mma_ss(tS0 + 128 * sb, sdesc_sw128(q_addr + qt * TILE + off, 16, 1024),
-                 sdesc_sw128(k_addr + st * TILE + off, 16, 1024), idesc_qk, k > 0 ? 1u : 0u);
-        }
+        for (int k = 0; k < KSTEPS; ++k)
+          mma_ss_warp(d, a0 + kstep(k), b0 + kstep(k), idesc_qk, k > 0 ? 1u : 0u);
       };
       auto issue_pv = [&](int ot, int sb, int st, bool acc) {
+        const uint64_t b0 = dv + st * kTileU;
+        const uint32_t d = tO0 + 128 * ot, a = tS0 + 128 * sb;
 #pragma unroll
         for (int k = 0; k < kTileKeys / 16; ++k)
-          mma_ts(tO0 + 128 * ot, tS0 + 128 * sb + 8 * k,
-                 sdesc_sw128(v_addr + st * TILE + k * 2048, kHalfBytes, 1024), idesc_pv,
-                 (acc || k > 0) ? 1u : 0u);
+          mma_ts_warp(d, a + 8 * k, b0 + ((k * 2048) >> 4), idesc_pv, (acc || k > 0) ? 1u : 0u);
       };
-      bool ok = mbar_wait(FP8 ? q_conv : q_full, 0, abort_flag, kWaitLimitNs) &&
-                mbar_wait(k_full + 0, 0, abort_flag, kWaitLimitNs);
+      // two tiles: S = Q tile `qt` (in TMEM) . K stage `st`^T into the shared S buffer;
+      // O tile `ot` += P tile `ot` (shared memory) . V stage `st`
+      auto issue_qk_t = [&](int qt, int st) {
+        const uint64_t b0 = dk + st * kTileU;
+        const uint32_t a = tQ0 + 64 * qt;
+#pragma unroll
+        for (int k = 0; k < KSTEPS; ++k)
+          mma_ts_warp(tS0, a + 8 * k, b0 + kstep(k), idesc_qk, k > 0 ? 1u : 0u);
+      };
+      auto issue_pv_s = [&](int ot, int st, bool acc) {
+        const uint64_t a0 = dq + ot * kPTileU, b0 = dv + st * kTileU;
+        const uint32_t d = tO0 + 128 * ot;
+#pragma unroll
+        for (int k = 0; k < kTileKeys / 16; ++k)
+          mma_ss_warp(d, a0 + kstep(k), b0 + ((k * 2048) >> 4), idesc_pv, (acc || k > 0) ? 1u : 0u);
+      };
+      bool ok = wait_all((FP8 || !single) ? q_conv : q_full, 0) &&
+                wait_all(k_full + 0, 0);
       if (single) {
         // one query tile, S double-buffered: K tile i uses S buffer i & 1.  While the
         // softmax works on buffer i & 1, S of tile i + 1 is already in the other one;
@@ -366,75 +497,96 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
         if (ok) {
           tc_fence_after();
           issue_qk(0, 0, 0);
-          mma_commit(s_full + 0);
-          mma_commit(k_empty + 0);
+          mma_commit_warp(s_full + 0);
+          mma_commit_warp(k_empty + 0);
         }
-        if (ok && n_tiles > 1 && (ok = mbar_wait(k_full + 1, 0, abort_flag, kWaitLimitNs))) {
+        if (ok && n_tiles > 1 && (ok = wait_all(k_full + 1, 0))) {
           tc_fence_after();
           issue_qk(0, 1, 1);
-          mma_commit(s_full + 1);
-          mma_commit(k_empty + 1);
+          mma_commit_warp(s_full + 1);
+          mma_commit_warp(k_empty + 1);
         }
-        // S buffer of tile i: i & 1; its K/V ring stage: i % RING
+        // S buffer of tile i: i & 1; its ring stages: i % RK, i % RV
         for (int i = 0; ok && i < n_tiles; ++i) {
-          const int b = i & 1, vs = i % RING;
+          const int b = i & 1, vs = i % RV;
           const uint32_t ph = (i >> 1) & 1;
-          if (!(ok = mbar_wait(v_full + vs, (i / RING) & 1, abort_flag, kWaitLimitNs))) break;
-          if (!(ok = mbar_wait(p_full + b, ph, abort_flag, kWaitLimitNs))) break;
+          if (!(ok = wait_all(v_full + vs, (i / RV) & 1))) break;
+          if (!(ok = wait_all(p_full + b, ph))) break;
           tc_fence_after();
           issue_pv(0, b, vs, i > 0);
-          mma_commit(o_full + 0);
-          mma_commit(v_empty + vs);
+          mma_commit_warp(o_full + 0);
+          mma_commit_warp(v_empty + vs);
           if (i + 2 < n_tiles) {
-            const int ks = (i + 2) % RING;
-            if (!(ok = mbar_wait(k_full + ks, ((i + 2) / RING) & 1, abort_flag, kWaitLimitNs)))
+            const int ks = (i + 2) % RK;
+            if (!(ok = wait_all(k_full + ks, ((i + 2) / RK) & 1)))
               break;
             tc_fence_after();
             issue_qk(0, b, ks);
-            mma_commit(s_full + b);
-            mma_commit(k_empty + ks);
+            mma_commit_warp(s_full + b);
+            mma_commit_warp(k_empty + ks);
           }
         }
       } else {
+        // Two tiles, one S buffer.  Use u of the buffer is QK of K tile u / 2 for
+        // query tile u % 2; it may start once the softmax has read use u - 1
+        // (completion u - 1 of s_free).  Per K tile i the order is
+        //   QK_0(i + 1), PV_0(i), QK_1(i + 1), PV_1(i)
+        // so the S of a query tile's next K tile is ready when its softmax
+        // finishes the current one.
         if (ok) {
           tc_fence_after();
-          issue_qk(0, 0, 0);
-          mma_commit(s_full + 0);
-          issue_qk(1, 1, 0);
-          mma_commit(s_full + 1);
-          mma_commit(k_empty + 0);
+          issue_qk_t(0, 0);
+          mma_commit_warp(s_full + 0);
+        }
+        if (ok && (ok = wait_all(s_free, 0))) {
+          tc_fence_after();
+          issue_qk_t(1, 0);
+          mma_commit_warp(s_full + 1);
+          mma_commit_warp(k_empty + 0);
         }
         for (int i = 0; ok && i < n_tiles; ++i) {
-          const int st = i & 1;
-          const uint32_t ph = (i >> 1) & 1;
+          const int st = i % RV;  // V stage of K tile i
+          const uint32_t ph = (i / RV) & 1;
           const bool more = i + 1 < n_tiles;
-          const int st1 = (i + 1) & 1;
-          const uint32_t ph1 = ((i + 1) >> 1) & 1;
-          if (!(ok = mbar_wait(v_full + st, ph, abort_flag, kWaitLimitNs))) break;
-          if (!(ok = mbar_wait(p_full + 0, i & 1, abort_flag, kWaitLimitNs))) break;
-          tc_fence_after();
-          issue_pv(0, 0, st, i > 0);
-          mma_commit(o_full + 0);
+          const int st1 = (i + 1) % RK;  // K stage of K tile i + 1
+          const uint32_t ph1 = ((i + 1) / RK) & 1;
           if (more) {
-            if (!(ok = mbar_wait(k_full + st1, ph1, abort_flag, kWaitLimitNs))) break;
+            // use 2i + 2 waits for completion 2i + 1 (tile 1 read S of K tile i), and
+            // for tile 0 to near the end of K tile i: S waiting in the shared buffer
+            // for a busy softmax would hold up the other tile
+            if (!(ok = wait_all(k_full + st1, ph1) &&
+                       wait_all(s_free, 1) &&
+                       wait_all(s_soon + 0, i & 1)))
+              break;
             tc_fence_after();
-            issue_qk(0, 0, st1);
-            mma_commit(s_full + 0);
+            issue_qk_t(0, st1);
+            mma_commit_warp(s_full + 0);
           }
-          if (!(ok = mbar_wait(p_full + 1, i & 1, abort_flag, kWaitLimitNs))) break;
+          if (!(ok = wait_all(v_full + st, ph) &&
+                     wait_all(p_full + 0, i & 1)))
+            break;
           tc_fence_after();
-          issue_pv(1, 1, st, i > 0);
-          mma_commit(o_full + 1);
-          mma_commit(v_empty + st);
+          issue_pv_s(0, st, i > 0);
+          mma_commit_warp(o_full + 0);
           if (more) {
-            issue_qk(1, 1, st1);
-            mma_commit(s_full + 1);
-            mma_commit(k_empty + st1);
+            // use 2i + 3 waits for completion 2i + 2 (tile 0 read S of K tile i + 1)
+            if (!(ok = wait_all(s_free, 0) &&
+                       wait_all(s_soon + 1, i & 1)))
+              break;
+            tc_fence_after();
+            issue_qk_t(1, st1);
+            mma_commit_warp(s_full + 1);
+            mma_commit_warp(k_empty + st1);
           }
+          if (!(ok = wait_all(p_full + 1, i & 1))) break;
+          tc_fence_after();
+          issue_pv_s(1, st, i > 0);
+          mma_commit_warp(o_full + 1);
+          mma_commit_warp(v_empty + st);
         }
       }
       // all MMAs finished before tensor memory is released
-      mma_commit(mma_done);
+      mma_commit_warp(mma_done);
       mbar_wait(mma_done, 0, nullptr, kWaitLimitNs);
     }
     __syncwarp();
@@ -445,21 +597,20 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
     const int ct = threadIdx.x - 10 * 32;
     bool ok = true;
     for (int i = 0; ok && i < n_tiles; ++i) {
-      const int st = i & 1;
-      const uint32_t ph = (i >> 1) & 1;
+      const int sk = i % RK, sv = i % RV;
       if (!(ok = mbar_wait(kst_full, i & 1, abort_flag, kWaitLimitNs) &&
-                 mbar_wait(k_empty + st, ph ^ 1, abort_flag, kWaitLimitNs)))
+                 mbar_wait(k_empty + sk, ((i / RK) & 1) ^ 1, abort_flag, kWaitLimitNs)))
         break;
-      widen_tile<D>(sStK, sK + st * TILE, ct);
+      widen_tile<D>(sStK, sK + sk * TILE, ct);
       fence_proxy_async_smem();
-      mbar_arrive(k_full + st);
+      mbar_arrive(k_full + sk);
       mbar_arrive(kst_empty);
       if (!(ok = mbar_wait(vst_full, i & 1, abort_flag, kWaitLimitNs) &&
-                 mbar_wait(v_empty + st, ph ^ 1, abort_flag, kWaitLimitNs)))
+                 mbar_wait(v_empty + sv, ((i / RV) & 1) ^ 1, abort_flag, kWaitLimitNs)))
         break;
-      widen_tile<D>(sStV, sV + st * TILE, ct);
+      widen_tile<D>(sStV, sV + sv * TILE, ct);
       fence_proxy_async_smem();
-      mbar_arrive(v_full + st);
+      mbar_arrive(v_full + sv);
       mbar_arrive(vst_empty);
     }
   } else if (!single || warp < 6) {
@@ -472,30 +623,53 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
     const bool row_valid = qi < q_len;
     const int vis = p.causal ? min(k_len, k_len - q_len + qi + 1) : k_len;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-    uint32_t tS = lane_base + 256 + 128 * t;  // S buffer of the current K tile
+    uint32_t tS = lane_base + 256 + 128 * t;  // S buffer of the current K tile (SINGLE)
+    if (!single) tS = lane_base + 256;        // two tiles: the shared S buffer
     const uint32_t tO = lane_base + 128 * t;
     // FP8: scores are q . code * k_scale, so the K scale joins the softmax scale
     const float sl2 = FP8 ? p.scale_log2 * __ldg(p.k_scale + g) : p.scale_log2;
     float m_ref = -INFINITY;  // raw score units
     float l = 0.f;
     bool ok = true;
-    if (FP8 && n_tiles > 0) {
-      // this thread's query row of tile t: bf16 -> f16 in place (elementwise, so
-      // the order of the row's 16-byte chunks does not matter; visiting chunk
-      // c ^ (row & 7) spreads a warp's 32 rows over all shared-memory banks)
+    if (n_tiles > 0 && (FP8 || !single)) {
+      // This thread's query row of tile t (visiting chunk c ^ (row & 7), the
+      // place of the row's logical chunk c, spreads a warp's 32 rows over all
+      // shared-memory banks).  One tile: bf16 -> f16 in place (FP8 cache).  Two
+      // tiles: into this row's TMEM lane, 2 elements per column (f16 over an
+      // FP8 cache), the layout of a tensor-memory A operand.
       ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, abort_flag, kWaitLimitNs));
-      if (ok) {
+      if (ok && single) {
 #pragma unroll
         for (int h = 0; h < HALVES; ++h)
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
-            uint4* chunk = reinterpret_cast<uint4*>(sQ + t * TILE + h * kHalfBytes + row * 128 +
+            uint4* chunk = reinterpret_cast<uint4*>(sQ + t * QSTRIDE + h * kHalfBytes + row * 128 +
                                                     ((c ^ (row & 7)) << 4));
             uint4 v = *chunk;
             bf16x8_to_f16x8(v);
             *chunk = v;
           }
         fence_proxy_async_smem();
+        mbar_arrive(q_conv);
+      } else if (ok) {
+        const uint32_t tQ = lane_base + 384 + 64 * t;
+#pragma unroll
+        for (int h = 0; h < HALVES; ++h) {
+          uint32_t qv[32];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            uint4 v = *reinterpret_cast<const uint4*>(sQ + t * QSTRIDE + h * kHalfBytes +
+                                                      row * 128 + ((c ^ (row & 7)) << 4));
+            if (FP8) bf16x8_to_f16x8(v);
+            qv[4 * c] = v.x;
+            qv[4 * c + 1] = v.y;
+            qv[4 * c + 2] = v.z;
+            qv[4 * c + 3] = v.w;
+          }
+          tmem_st32(tQ + 32 * h, qv);
+        }
+        tmem_wait_st();
+        tc_fence_before();
         mbar_arrive(q_conv);
       }
     }
@@ -510,6 +684,12 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
       for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, sv[c]);
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_wait_ld(sv[c]);
+      if (!single) {
+        // two tiles: the shared S buffer is free for the other tile's QK
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_free);
+      }
       if (masked) {
         const int kb = (kt0 + i) * kTileKeys;
 #pragma unroll
@@ -522,8 +702,8 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
 #pragma unroll
       for (int c = 0; c < 4; ++c)
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) mx[c] = fmaxf(mx[c], fmaxf(f(sv[c][e]), f(sv[c][e + 1])));
-      const float row_max = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+        for (int e = 0; e < 32; e += 2) mx[c] = max3(mx[c], f(sv[c][e]), f(sv[c][e + 1]));
+      const float row_max = max3(mx[0], mx[1], fmaxf(mx[2], mx[3]));
       const float m_new = fmaxf(m_ref, row_max);
       float alpha = 1.f;
       bool rescale = false;
@@ -535,25 +715,64 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
         rescale = true;
       }
       const float base = m_ref == -INFINITY ? 0.f : m_ref * sl2;
-      // P = 2^(s*scale*log2e - base) as bf16 pairs over the first 64 S columns
-      float ls[2] = {0.f, 0.f};
+      // P = 2^(s*scale*log2e - base), packed in pairs (bf16, or f16 over an FP8 cache)
+      // two tiles: packed pairs (fewer instructions per score; the one-tile
+      // kernel keeps scalar arithmetic, whose register allocation does not spill)
+      uint64_t ls = f2_pack(0.f, 0.f);
+      float ls0 = 0.f, ls1 = 0.f;
+      const uint64_t sl2x2 = f2_pack(sl2, sl2), nbase2 = f2_pack(-base, -base);
+      uint32_t pk[4][16];
+      // two tiles: P row into the K-major 128-byte-swizzled A-operand layout of
+      // P_t in shared memory (keys [64h, 64h + 64) in panel h, logical 16-byte
+      // chunk c at c ^ (row & 7)); 32 keys (4 chunks) per call
+      auto store_p = [&](int c) {
+        uint8_t* prow = sQ + t * kPTile + (c >> 1) * kHalfBytes + row * 128;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          *reinterpret_cast<uint4*>(prow + (((4 * (c & 1) + j) ^ (row & 7)) << 4)) =
+              make_uint4(pk[c][4 * j], pk[c][4 * j + 1], pk[c][4 * j + 2], pk[c][4 * j + 3]);
+      };
+      // two tiles: P(i) replaces P(i - 1) in shared memory once PV(i - 1) has read it
+      // (complete by now as a rule: it was issued when this tile's S was)
+      bool waited = false;
+      if (!single && i > 0) {
+        if (!__all_sync(0xffffffffu, mbar_wait(o_full + t, (i - 1) & 1, abort_flag, kWaitLimitNs)))
+          return false;
+        tc_fence_after();
+        waited = true;
+      }
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const float pa = ex2(fmaf(f(sv[c][2 * e]), sl2, -base));
-          const float pb = ex2(fmaf(f(sv[c][2 * e + 1]), sl2, -base));
-          ls[0] += pa;
-          ls[1] += pb;
-          pk[e] = FP8 ? pack_f16x2(pa, pb) : pack_bf16(pa, pb);
+          float pa, pb;
+          if constexpr (SINGLE) {
+            pa = ex2(fmaf(f(sv[c][2 * e]), sl2, -base));
+            pb = ex2(fmaf(f(sv[c][2 * e + 1]), sl2, -base));
+            ls0 += pa;
+            ls1 += pb;
+          } else {
+            float xa, xb;
+            f2_unpack(f2_fma(f2_pack(f(sv[c][2 * e]), f(sv[c][2 * e + 1])), sl2x2, nbase2), xa, xb);
+            pa = ex2(xa);
+            pb = ex2(xb);
+            ls = f2_add(ls, f2_pack(pa, pb));
+          }
+          pk[c][e] = FP8 ? pack_f16x2(pa, pb) : pack_bf16(pa, pb);
         }
-        tmem_st16(tS + 16 * c, pk);
+        if (single) {
+          tmem_st16(tS + 16 * c, pk[c]);  // one tile: P over the first 64 columns of this S buffer
+        } else {
+          store_p(c);
+          if (c == kSoonChunks - 1) mbar_arrive(s_soon + t);
+        }
       }
-      l = l * alpha + (ls[0] + ls[1]);
+      if constexpr (!SINGLE) f2_unpack(ls, ls0, ls1);
+      l = l * alpha + (ls0 + ls1);
       if (__any_sync(0xffffffffu, rescale)) {
-        // O_t holds PV of the previous tile (S_t of this tile completed after it); rescale in place
-        if (!__all_sync(0xffffffffu, mbar_wait(o_full + t, (i - 1) & 1, abort_flag, kWaitLimitNs)))
+        // O_t holds PV up to K tile i - 1; rescale it in place once that is complete
+        if (!waited &&
+            !__all_sync(0xffffffffu, mbar_wait(o_full + t, (i - 1) & 1, abort_flag, kWaitLimitNs)))
           return false;
         tc_fence_after();
 #pragma unroll
@@ -566,6 +785,7 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
           tmem_st32(tO + 32 * c, o);
         }
       }
+      if (!single) fence_proxy_async_smem();
       return true;
     };
     // A warp whose 32 rows hold no query (past the end of the chunk) only keeps
@@ -573,10 +793,20 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
     const bool warp_live = __any_sync(0xffffffffu, row_valid);
     // one K tile of softmax on S buffer sb (phase sph of its barriers)
     auto run_tile = [&](int i, int sb, uint32_t sph) -> bool {
-      tS = lane_base + 256 + 128 * sb;
+      if (single) tS = lane_base + 256 + 128 * sb;
       if (!__all_sync(0xffffffffu, mbar_wait(s_full + sb, sph, abort_flag, kWaitLimitNs)))
         return false;
       if (!warp_live) {
+        if (!single) {
+          // release S; arrive for P(i) only after PV(i - 1), so that these
+          // arrivals never count towards the previous P
+          __syncwarp();
+          if (lane == 0) mbar_arrive(s_free);
+          if (i > 0 &&
+              !__all_sync(0xffffffffu, mbar_wait(o_full + t, (i - 1) & 1, abort_flag, kWaitLimitNs)))
+            return false;
+          mbar_arrive(s_soon + t);
+        }
         mbar_arrive(p_full + sb);
         return true;
       }

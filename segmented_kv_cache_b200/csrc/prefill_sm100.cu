@@ -439,7 +439,7 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
     // executes each tcgen05.mma / commit.
     if (n_tiles > 0) {
       auto wait_all = [&](uint64_t* bar, uint32_t parity) {
-        return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, kWaitLimitNs));
+        return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, kWaitLimitNs, true));
       };
       const uint32_t idesc_qk =
           FP8 ? idesc_f16_f32(128, 128, false) : idesc_bf16_f32(128, 128, false);
@@ -736,7 +736,8 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
       // (complete by now as a rule: it was issued when this tile's S was)
       bool waited = false;
       if (!single && i > 0) {
-        if (!__all_sync(0xffffffffu, mbar_wait(o_full + t, (i - 1) & 1, abort_flag, kWaitLimitNs)))
+        if (!__all_sync(0xffffffffu,
+                        mbar_wait(o_full + t, (i - 1) & 1, abort_flag, kWaitLimitNs, true)))
           return false;
         tc_fence_after();
         waited = true;
@@ -794,7 +795,7 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
     // one K tile of softmax on S buffer sb (phase sph of its barriers)
     auto run_tile = [&](int i, int sb, uint32_t sph) -> bool {
       if (single) tS = lane_base + 256 + 128 * sb;
-      if (!__all_sync(0xffffffffu, mbar_wait(s_full + sb, sph, abort_flag, kWaitLimitNs)))
+      if (!__all_sync(0xffffffffu, mbar_wait(s_full + sb, sph, abort_flag, kWaitLimitNs, true)))
         return false;
       if (!warp_live) {
         if (!single) {

@@ -28,19 +28,21 @@
 //                the max grows by more than 2^8 (the final O / l uses the same
 //                reference max, so the result is unchanged), epilogue O / l ->
 //                bf16 and lse.
-// Two query tiles (the usual item): the softmax threads copy their query rows
-// into tensor memory once, so
+// Two query tiles over a bf16 cache (the usual item): the softmax threads copy
+// their query rows into tensor memory once, so
 //                  S   = Q_t K^T   (TS: Q from TMEM, K from the ring)
 //                  O_t += P_t V    (SS: P from shared memory, V MN-major)
 // and the two tiles take turns on one S buffer.  A softmax thread loads its
 // whole S row, releases the buffer (the other tile's QK can go), and writes P
 // to shared memory, so the next K tile's S of a query tile is computed while
-// this tile's softmax still runs: each tile's chain is its softmax alone, not
-// softmax + PV + QK.
+// this tile's softmax still runs, and no MMA writes tensor memory that the MMA
+// before it reads (such a write waits for the tensor pipe to drain).
 // TMEM columns: O0 [0,128) O1 [128,256) S [256,384) Q0 [384,448) Q1 [448,512).
-// One query tile (SINGLE): Q stays in shared memory (SS QK), P is written over
-// S in TMEM (TS PV) and S is double-buffered instead:
-// TMEM columns: O [0,128) S0/P0 [256,384) S1/P1 [384,512).
+// One query tile, or two over an FP8 cache (whose code staging leaves no
+// shared memory for P): Q stays in shared memory (SS QK) and P is written over
+// S in TMEM (TS PV); one tile double-buffers S, two tiles have one S each and
+// issue PV_0, QK_0, PV_1, QK_1 so one tile's softmax overlaps the other's MMAs.
+// TMEM columns: O0 [0,128) (O1 [128,256)) S0/P0 [256,384) S1/P1 [384,512).
 // Every mbarrier wait is bounded (1 s); a timeout stops all roles of the CTA,
 // drains in-flight copies and MMAs, frees TMEM and flags a device error.
 #include <cuda.h>
@@ -105,15 +107,25 @@ constexpr int ring_v() {
   return SINGLE && !FP8 ? 3 : 2;
 }
 
-template <int D, bool SINGLE>
+// Two query tiles over a bf16 cache: queries in tensor memory, P in shared
+// memory, one S buffer the two tiles take turns on.  Every other variant (one
+// query tile; the FP8 cache, whose code staging leaves no shared memory for P)
+// keeps its queries in shared memory and writes P over S in tensor memory.
+template <bool SINGLE, bool FP8>
+constexpr bool queries_in_tmem() {
+  return !SINGLE && !FP8;
+}
+
+template <int D, bool SINGLE, bool FP8>
 constexpr size_t query_region_bytes() {
-  return SINGLE ? (D / 64) * (size_t)kHalfBytes : 2 * (size_t)kPTile;
+  return queries_in_tmem<SINGLE, FP8>() ? 2 * (size_t)kPTile
+                                        : (SINGLE ? 1 : 2) * (D / 64) * (size_t)kHalfBytes;
 }
 
 // The FP8 variant adds one staging tile of raw codes each for K and V.
 template <int D, bool SINGLE, bool FP8>
 constexpr size_t prefill_smem_bytes() {
-  constexpr size_t need = query_region_bytes<D, SINGLE>() +
+  constexpr size_t need = query_region_bytes<D, SINGLE, FP8>() +
                           (ring_k<SINGLE, FP8>() + ring_v<SINGLE, FP8>()) * (D / 64) *
                               (size_t)kHalfBytes +
                           (FP8 ? 2 * kTileKeys * D : 0) + 256 + 1024;
@@ -218,11 +230,12 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
   constexpr int RK = ring_k<SINGLE, FP8>(), RV = ring_v<SINGLE, FP8>();
-  // SINGLE: the one Q tile.  Two tiles: P_t at sQ + t * kPTile, which holds Q
-  // tile t until its softmax threads have copied it to tensor memory.
-  constexpr uint32_t QSTRIDE = SINGLE ? TILE : kPTile;
+  // Q tiles at sQ + t * TILE; with queries in tensor memory, P_t at sQ + t * kPTile,
+  // which holds Q tile t until its softmax threads have copied it there.
+  constexpr bool QT = queries_in_tmem<SINGLE, FP8>();
+  constexpr uint32_t QSTRIDE = QT ? kPTile : TILE;
   uint8_t* sQ = sm;
-  uint8_t* sK = sm + query_region_bytes<D, SINGLE>();
+  uint8_t* sK = sm + query_region_bytes<D, SINGLE, FP8>();
   uint8_t* sV = sK + RK * TILE;
   uint8_t* sStK = sV + RV * TILE;           // FP8: raw code tile of K
   uint8_t* sStV = sStK + kTileKeys * D;     // FP8: raw code tile of V
@@ -487,7 +500,7 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
         for (int k = 0; k < kTileKeys / 16; ++k)
           mma_ss_warp(d, a0 + kstep(k), b0 + ((k * 2048) >> 4), idesc_pv, (acc || k > 0) ? 1u : 0u);
       };
-      bool ok = wait_all((FP8 || !single) ? q_conv : q_full, 0) &&
+      bool ok = wait_all((FP8 || QT) ? q_conv : q_full, 0) &&
                 wait_all(k_full + 0, 0);
       if (single) {
         // one query tile, S double-buffered: K tile i uses S buffer i & 1.  While the
@@ -524,6 +537,45 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
             issue_qk(0, b, ks);
             mma_commit_warp(s_full + b);
             mma_commit_warp(k_empty + ks);
+          }
+        }
+      } else if (!QT) {
+        // Two tiles, P over S (FP8 cache): per K tile i the order is
+        //   PV_0(i), QK_0(i + 1), PV_1(i), QK_1(i + 1)
+        // so one tile's softmax overlaps the other tile's MMAs.
+        if (ok) {
+          tc_fence_after();
+          issue_qk(0, 0, 0);
+          mma_commit_warp(s_full + 0);
+          issue_qk(1, 1, 0);
+          mma_commit_warp(s_full + 1);
+          mma_commit_warp(k_empty + 0);
+        }
+        for (int i = 0; ok && i < n_tiles; ++i) {
+          const int st = i % RV;  // V stage of K tile i
+          const uint32_t ph = (i / RV) & 1;
+          const bool more = i + 1 < n_tiles;
+          const int st1 = (i + 1) % RK;  // K stage of K tile i + 1
+          const uint32_t ph1 = ((i + 1) / RK) & 1;
+          if (!(ok = wait_all(v_full + st, ph) && wait_all(p_full + 0, i & 1))) break;
+          tc_fence_after();
+          issue_pv(0, 0, st, i > 0);
+          mma_commit_warp(o_full + 0);
+          if (more) {
+            if (!(ok = wait_all(k_full + st1, ph1))) break;
+            tc_fence_after();
+            issue_qk(0, 0, st1);
+            mma_commit_warp(s_full + 0);
+          }
+          if (!(ok = wait_all(p_full + 1, i & 1))) break;
+          tc_fence_after();
+          issue_pv(1, 1, st, i > 0);
+          mma_commit_warp(o_full + 1);
+          mma_commit_warp(v_empty + st);
+          if (more) {
+            issue_qk(1, 1, st1);
+            mma_commit_warp(s_full + 1);
+            mma_commit_warp(k_empty + st1);
           }
         }
       } else {
@@ -624,21 +676,21 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
     const int vis = p.causal ? min(k_len, k_len - q_len + qi + 1) : k_len;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     uint32_t tS = lane_base + 256 + 128 * t;  // S buffer of the current K tile (SINGLE)
-    if (!single) tS = lane_base + 256;        // two tiles: the shared S buffer
+    if (QT) tS = lane_base + 256;             // queries in TMEM: the shared S buffer
     const uint32_t tO = lane_base + 128 * t;
     // FP8: scores are q . code * k_scale, so the K scale joins the softmax scale
     const float sl2 = FP8 ? p.scale_log2 * __ldg(p.k_scale + g) : p.scale_log2;
     float m_ref = -INFINITY;  // raw score units
     float l = 0.f;
     bool ok = true;
-    if (n_tiles > 0 && (FP8 || !single)) {
+    if (n_tiles > 0 && (FP8 || QT)) {
       // This thread's query row of tile t (visiting chunk c ^ (row & 7), the
       // place of the row's logical chunk c, spreads a warp's 32 rows over all
       // shared-memory banks).  One tile: bf16 -> f16 in place (FP8 cache).  Two
       // tiles: into this row's TMEM lane, 2 elements per column (f16 over an
       // FP8 cache), the layout of a tensor-memory A operand.
       ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, abort_flag, kWaitLimitNs));
-      if (ok && single) {
+      if (ok && !QT) {
 #pragma unroll
         for (int h = 0; h < HALVES; ++h)
 #pragma unroll
@@ -684,8 +736,8 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
       for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, sv[c]);
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_wait_ld(sv[c]);
-      if (!single) {
-        // two tiles: the shared S buffer is free for the other tile's QK
+      if (QT) {
+        // the shared S buffer is free for the other tile's QK
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(s_free);
@@ -735,7 +787,7 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
       // two tiles: P(i) replaces P(i - 1) in shared memory once PV(i - 1) has read it
       // (complete by now as a rule: it was issued when this tile's S was)
       bool waited = false;
-      if (!single && i > 0) {
+      if (QT && i > 0) {
         if (!__all_sync(0xffffffffu,
                         mbar_wait(o_full + t, (i - 1) & 1, abort_flag, kWaitLimitNs, true)))
           return false;
@@ -747,7 +799,7 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           float pa, pb;
-          if constexpr (SINGLE) {
+          if constexpr (!QT) {
             pa = ex2(fmaf(f(sv[c][2 * e]), sl2, -base));
             pb = ex2(fmaf(f(sv[c][2 * e + 1]), sl2, -base));
             ls0 += pa;
@@ -761,14 +813,14 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
           }
           pk[c][e] = FP8 ? pack_f16x2(pa, pb) : pack_bf16(pa, pb);
         }
-        if (single) {
-          tmem_st16(tS + 16 * c, pk[c]);  // one tile: P over the first 64 columns of this S buffer
+        if (!QT) {
+          tmem_st16(tS + 16 * c, pk[c]);  // P over the first 64 columns of this S buffer
         } else {
           store_p(c);
           if (c == kSoonChunks - 1) mbar_arrive(s_soon + t);
         }
       }
-      if constexpr (!SINGLE) f2_unpack(ls, ls0, ls1);
+      if constexpr (QT) f2_unpack(ls, ls0, ls1);
       l = l * alpha + (ls0 + ls1);
       if (__any_sync(0xffffffffu, rescale)) {
         // O_t holds PV up to K tile i - 1; rescale it in place once that is complete
@@ -786,7 +838,7 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
           tmem_st32(tO + 32 * c, o);
         }
       }
-      if (!single) fence_proxy_async_smem();
+      if (QT) fence_proxy_async_smem();
       return true;
     };
     // A warp whose 32 rows hold no query (past the end of the chunk) only keeps
@@ -798,7 +850,7 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
       if (!__all_sync(0xffffffffu, mbar_wait(s_full + sb, sph, abort_flag, kWaitLimitNs, true)))
         return false;
       if (!warp_live) {
-        if (!single) {
+        if (QT) {
           // release S; arrive for P(i) only after PV(i - 1), so that these
           // arrivals never count towards the previous P
           __syncwarp();

@@ -17,10 +17,10 @@
 // four-row gathers.
 //
 // Warp roles (10 warps; 12 over an FP8 cache, see below):
-//   warp 0       TMA producer: Q tiles once, then a K ring and a V ring of
-//                2 stages (3 in the one-tile bf16 kernel, which has the second
-//                query tile's space to spare).
-//   warp 1       TMEM allocator; lane 0 issues every tcgen05.mma.
+//   warp 0       TMA producer: Q tiles once, then a K ring and a V ring
+//                (stages per variant below), K tile i + 1 before V tile i.
+//   warp 1       TMEM allocator and MMA issuer: the whole warp runs the issue
+//                loop, one elected lane executes each tcgen05.mma / commit.
 //   warps 2-5    softmax for query tile 0, warps 6-9 for tile 1: one thread
 //                per row (its TMEM lane); online softmax (running max m and
 //                normaliser l, as in the Ascend FlashAttention article,

@@ -767,14 +767,15 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
         rescale = true;
       }
       const float base = m_ref == -INFINITY ? 0.f : m_ref * sl2;
-      // P = 2^(s*scale*log2e - base), packed in pairs (bf16, or f16 over an FP8 cache)
-      // two tiles: packed pairs (fewer instructions per score; the one-tile
-      // kernel keeps scalar arithmetic, whose register allocation does not spill)
+      // P = 2^(s*scale*log2e - base), packed in pairs (bf16, or f16 over an FP8 cache).
+      // Queries in TMEM: f32x2 pairs for the scale-and-subtract and the sums (fewer
+      // instructions per score); the P-over-S variants keep scalar arithmetic, whose
+      // register allocation does not spill.
       uint64_t ls = f2_pack(0.f, 0.f);
       float ls0 = 0.f, ls1 = 0.f;
       const uint64_t sl2x2 = f2_pack(sl2, sl2), nbase2 = f2_pack(-base, -base);
       uint32_t pk[4][16];
-      // two tiles: P row into the K-major 128-byte-swizzled A-operand layout of
+      // queries in TMEM: P row into the K-major 128-byte-swizzled A-operand layout of
       // P_t in shared memory (keys [64h, 64h + 64) in panel h, logical 16-byte
       // chunk c at c ^ (row & 7)); 32 keys (4 chunks) per call
       auto store_p = [&](int c) {
@@ -784,7 +785,7 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
           *reinterpret_cast<uint4*>(prow + (((4 * (c & 1) + j) ^ (row & 7)) << 4)) =
               make_uint4(pk[c][4 * j], pk[c][4 * j + 1], pk[c][4 * j + 2], pk[c][4 * j + 3]);
       };
-      // two tiles: P(i) replaces P(i - 1) in shared memory once PV(i - 1) has read it
+      // queries in TMEM: P(i) replaces P(i - 1) in shared memory once PV(i - 1) has read it
       // (complete by now as a rule: it was issued when this tile's S was)
       bool waited = false;
       if (QT && i > 0) {

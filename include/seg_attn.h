@@ -192,11 +192,15 @@ int seg_attn_build_table(int batch, const int32_t* q_lens, const int32_t* seg_co
 size_t seg_attn_workspace_size(const seg_attn_table_desc* desc);
 
 /*
- * seg_attn_prefill -- chunked-prefill attention (mode PREFILL table).
- * One persistent-tile sm_100a kernel: K/V tiles of 128 logical keys are
- * gathered row by row from the pool with TMA, S = QK^T and O += PV run on the
- * tcgen05 tensor cores with accumulators in tensor memory, the online softmax
- * runs in registers.  Writes out (and lse if non-NULL) for every row.
+ * seg_attn_prefill -- chunked-prefill attention (mode PREFILL table): a chunk
+ * of new queries per request over its prior context plus itself (Flood README,
+ * feature list: chunked prefill; the Q_len = K_len = 1024 rows of its
+ * "Kernels > Seg-attn" table are the one-chunk case).  One sm_100a kernel
+ * launch per pass (plus a merge kernel when long items are split): K/V tiles
+ * of 128 logical keys are gathered from the pool with TMA, S = QK^T and
+ * O += PV run on the tcgen05 tensor cores with accumulators in tensor memory,
+ * the online softmax runs in registers.  Writes out (and lse if non-NULL) for
+ * every row.
  *   softmax_scale  > 0 and finite (typically 1/sqrt(head_dim))
  *   workspace      device memory of at least seg_attn_workspace_size(desc)
  *                  bytes, 16-byte aligned, when that size is non-zero: the
@@ -210,12 +214,15 @@ int seg_attn_prefill(const void* q, const void* k_pool, const void* v_pool, void
 
 /*
  * seg_attn_decode -- one query per request over its whole context (mode
- * DECODE table).  Split-K over chunks of logical keys: one CTA per
- * (chunk, kv head) streams K/V with 128-bit loads, packs the group's query
- * heads so each K/V byte is read once per kv head, and keeps the softmax state
- * in registers; a second kernel merges the per-chunk partials by their
- * log-sum-exp.  workspace: device memory of at least
- * seg_attn_workspace_size(desc) bytes, 16-byte aligned (contents are scratch).
+ * DECODE table; the Q_len = 1 rows of the Flood README "Kernels > Seg-attn"
+ * table).  Split-K over chunks of logical keys, each chunk a partial attention
+ * reduced per request afterwards (FlashAccel article, "data layout
+ * optimisation"): one CTA per (chunk, kv head, slice of up to 8 query heads)
+ * streams K/V with 128-bit loads, packs the slice's query heads so each K/V
+ * byte fetched serves all of them, and keeps the softmax state in registers;
+ * a second kernel merges the per-chunk partials by their log-sum-exp.
+ * workspace: device memory of at least seg_attn_workspace_size(desc) bytes,
+ * 16-byte aligned (contents are scratch).
  */
 int seg_attn_decode(const void* q, const void* k_pool, const void* v_pool, void* out, float* lse,
                     const void* dev_table, const seg_attn_table_desc* desc, float softmax_scale,
@@ -261,7 +268,11 @@ int seg_attn_wait_selftest(int wait_us, void* stream);
  *     streams or host threads) race on it: order them, e.g. on one stream.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current); make that first call
- *     before starting any stream capture.
+ *     before starting any stream capture.  The address is remembered for the
+ *     life of the process: after cudaDeviceReset (or anything else that
+ *     destroys the device's primary context) the library's module is loaded
+ *     again and the array may sit elsewhere, so do not call this entry point
+ *     on that device again in the same process.
  *   - Calls no cudaMalloc, cudaFree or other allocating routine.
  */
 int seg_attn_decode_noalloc(const void* q, const void* k_pool, const void* v_pool, void* out,

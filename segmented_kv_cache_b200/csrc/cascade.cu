@@ -85,13 +85,13 @@ __global__ void __launch_bounds__(128) cascade_merge_kernel(const CascadeParams 
     const float w = exp2f(lse_of(j) - Mb);
     L += w;
     const float* po = o_of(j) + lane * PER;
+    // PER is 2 (d = 64) or 4 (d = 128): 8-byte pairs fit both, and a lane's
+    // columns start 8-byte aligned in either case
 #pragma unroll
-    for (int c = 0; c < PER; c += 4) {
-      const float4 x = *reinterpret_cast<const float4*>(po + c);
+    for (int c = 0; c < PER; c += 2) {
+      const float2 x = *reinterpret_cast<const float2*>(po + c);
       acc[c] += w * x.x;
       acc[c + 1] += w * x.y;
-      acc[c + 2] += w * x.z;
-      acc[c + 3] += w * x.w;
     }
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;

@@ -20,7 +20,10 @@
 //     caller must order them, e.g. by issuing them on one stream.
 //   - The first call on each device asks the runtime for the array's device
 //     address (cudaGetSymbolAddress) with that device current and remembers
-//     it.  Make that first call before any stream capture is started.
+//     it.  Make that first call before any stream capture is started.  The
+//     remembered address is only valid while the device's primary context
+//     lives: a cudaDeviceReset reloads the module, possibly elsewhere, so the
+//     entry point must not be used on that device again in the process.
 //   - Nothing here calls cudaMalloc, cudaFree or an allocating library routine.
 #include <cuda_runtime.h>
 #include <stdint.h>

@@ -118,12 +118,12 @@ def test_config4_sampled_requests(cfg):
     compare(out[rows], lse[rows], ref_o, ref_l, "config 4")
 
 
-def test_config5_decode_sampled():
+def test_config5_decode_all_requests():
     wl = synth.make_workload(5, device="cuda")
     b = wl.batches[0]
     out, lse, _ = run_batch(wl, b)
     torch.cuda.synchronize()
-    sub = compact_requests(wl, b, [0, 5])
+    sub = compact_requests(wl, b, list(range(b.batch)))
     ref_o, ref_l = oracle.attention(sub["q_lens"], sub["seg_starts"], sub["seg_lens"], sub["q"],
                                     sub["k_pool"], sub["v_pool"], wl.scale, True)
     rows = sub["q_rows"].cuda()

@@ -175,13 +175,16 @@ def test_decode_row_equals_last_prefill_row():
     assert (lse_d - lse[last]).abs().max() <= 1e-4
 
 
-def test_config3_sampled_requests():
+def test_config3_all_requests():
+    # every row of all 16 requests of the chunked varlen batch (about 2.8e11 flop in the
+    # oracle), in the launch configuration the benchmark times
     wl = synth.make_workload(3, device="cuda")
     b = wl.batches[0]
     out, lse, _ = run_batch(wl, b)
     torch.cuda.synchronize()
     assert torch.isfinite(out.float()).all()
-    reqs = [r for r in range(b.batch) if b.q_lens[r] > 0][:3]
+    reqs = [r for r in range(b.batch) if b.q_lens[r] > 0]
+    assert sum(b.q_lens[r] for r in reqs) == b.total_q
     sub = compact_requests(wl, b, reqs)
     ref_o, ref_l = oracle.attention(sub["q_lens"], sub["seg_starts"], sub["seg_lens"], sub["q"],
                                     sub["k_pool"], sub["v_pool"], wl.scale, True)
@@ -189,16 +192,40 @@ def test_config3_sampled_requests():
     compare(out[rows], lse[rows], ref_o, ref_l, "config 3")
 
 
-def test_config5_prefill_sampled_rows():
+def config5_prefill_rows(qpt, span, q_len, q_heads, kv_heads, seed=5):
+    """(token, head) rows of the 2048-query chunk that reach every work item of the plan:
+    for each 2-tile item (span queries) one query in each of its two query tiles and, for
+    each kv head, one query head of its group; plus every head of the first and last
+    query.  Each row attends to all key tiles, so every split piece of every item (first
+    and last key tile included) contributes to some checked row."""
+    g = torch.Generator().manual_seed(seed)
+    group = q_heads // kv_heads
+    toks, heads = [], []
+    for q0 in range(0, q_len, span):
+        for t in range(2):
+            lo = q0 + t * qpt
+            if lo >= q_len:
+                continue
+            for kv in range(kv_heads):
+                toks.append(lo + int(torch.randint(0, min(qpt, q_len - lo), (1,), generator=g)))
+                heads.append(kv * group + int(torch.randint(0, group, (1,), generator=g)))
+    for tok in (0, q_len - 1):
+        toks += [tok] * q_heads
+        heads += list(range(q_heads))
+    return torch.tensor(toks), torch.tensor(heads)
+
+
+def test_config5_prefill_rows_of_every_item():
     wl = synth.make_workload(5, device="cuda")
     b = wl.batches[1]
-    out, lse, _ = run_batch(wl, b)
+    out, lse, tab = run_batch(wl, b)
     torch.cuda.synchronize()
     assert torch.isfinite(out.float()).all()
+    assert tab.desc.num_merge > 0  # the items are split along their keys at this size
+    qpt = tab.desc.queries_per_tile
+    toks, heads = config5_prefill_rows(qpt, 2 * qpt, b.q_lens[0], wl.q_heads, wl.kv_heads)
+    assert toks.numel() >= 1024
     sub = compact_requests(wl, b, [0])
-    g = torch.Generator().manual_seed(5)
-    toks = torch.cat([torch.tensor([0, 2047]), torch.randint(0, 2048, (14,), generator=g)])
-    heads = torch.randint(0, wl.q_heads, (toks.numel(),), generator=g)
     ref_o, ref_l = oracle.attention(sub["q_lens"], sub["seg_starts"], sub["seg_lens"], sub["q"],
                                     sub["k_pool"], sub["v_pool"], wl.scale, True,
                                     rows=(toks.numpy(), heads.numpy()))

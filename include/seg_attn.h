@@ -38,8 +38,7 @@
  *   - The new tokens' K/V rows are already written into the pool: they are
  *     the last q_len logical keys of each request's segment list.
  *   - Supported shapes: head_dim in {64, 128}; q_heads % kv_heads == 0;
- *     prefill: group size q_heads/kv_heads a power of two <= 128;
- *     decode:  group size a power of two <= 8.
+ *     group size q_heads/kv_heads a power of two <= 128 (prefill and decode).
  *   - Errors are returned synchronously as a negative seg_attn_status before
  *     anything is launched; nothing is launched on error.  A launch failure
  *     is reported as SEG_ATTN_ERR_CUDA.  Device code never traps.
@@ -250,6 +249,25 @@ int seg_attn_take_device_error(int* value);
  * status instead of a hang.  wait_us out of range: SEG_ATTN_ERR_INVALID_ARG.
  */
 int seg_attn_wait_selftest(int wait_us, void* stream);
+
+/*
+ * seg_attn_stall_test -- diagnostic (no counterpart on the source pages):
+ * makes later prefill launches stall the way a copy that never lands would,
+ * so that the kernel's give-up path can be exercised without a GPU fault.
+ *   withhold_k_tile >= 0: the producer warp of every CTA whose piece has more
+ *                  K tiles than that stops loading before that K tile; the
+ *                  tensor-core and softmax warps then wait for it, give up
+ *                  after wait_us, drain the copies and MMAs already issued,
+ *                  free tensor memory and set bit 0 of the device error word
+ *                  (the CTA's output rows are left unwritten).
+ *   withhold_k_tile < 0: off (the default).
+ *   wait_us        limit of every bounded wait of later prefill launches,
+ *                  1 .. 1000000 (default 1000000, i.e. one second).
+ * Host-side settings read at each launch (process-wide, not thread-safe with
+ * concurrent prefill calls).  seg_attn_stall_test(-1, 1000000) restores the
+ * defaults.  wait_us out of range: SEG_ATTN_ERR_INVALID_ARG.
+ */
+int seg_attn_stall_test(int withhold_k_tile, int wait_us);
 
 /*
  * seg_attn_decode_noalloc -- seg_attn_decode for callers that cannot allocate

@@ -21,7 +21,7 @@ from ._build import LIB as LIB_PATH
 __all__ = [
     "SegAttnError", "seg_attn_table_desc", "seg_attn_build_table", "seg_attn_workspace_size",
     "seg_attn_prefill", "seg_attn_decode", "seg_attn_status_string", "seg_attn_version",
-    "seg_attn_take_device_error", "seg_attn_wait_selftest", "SegTable", "load_library", "LIB_PATH",
+    "seg_attn_take_device_error", "seg_attn_wait_selftest", "seg_attn_stall_test", "SegTable", "load_library", "LIB_PATH",
     "MODE_PREFILL", "MODE_DECODE", "STATUS", "SegPool", "seg_attn_kv_append",
     "seg_attn_decode_fp8", "seg_attn_prefill_fp8", "seg_attn_kv_append_fp8", "SHARE_PREFIX",
     "seg_la_table_desc", "seg_la_build_table", "seg_la_workspace_size", "seg_la_prefill",
@@ -128,6 +128,8 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         lib.seg_attn_take_device_error.restype = I
         lib.seg_attn_wait_selftest.argtypes = [I, P]
         lib.seg_attn_wait_selftest.restype = I
+        lib.seg_attn_stall_test.argtypes = [I, I]
+        lib.seg_attn_stall_test.restype = I
         PP = ctypes.POINTER(ctypes.c_void_p)
         lib.seg_attn_pool_create.argtypes = [I64, PP]
         lib.seg_attn_pool_destroy.argtypes = [P]
@@ -243,6 +245,14 @@ def seg_attn_wait_selftest(wait_us: int, stream=None) -> None:
     rc = load_library().seg_attn_wait_selftest(int(wait_us), _stream_ptr(stream))
     if rc != 0:
         raise SegAttnError("seg_attn_wait_selftest", rc)
+
+
+def seg_attn_stall_test(withhold_k_tile: int, wait_us: int = 1000000) -> None:
+    """Stall test switch of later prefill launches: the producer stops before K tile
+    ``withhold_k_tile`` (< 0: off) and every bounded wait gives up after ``wait_us``."""
+    rc = load_library().seg_attn_stall_test(int(withhold_k_tile), int(wait_us))
+    if rc != 0:
+        raise SegAttnError("seg_attn_stall_test", rc)
 
 
 def seg_attn_take_device_error() -> int:

@@ -212,6 +212,11 @@ extern "C" int seg_attn_wait_selftest(int wait_us, void* stream) {
   return segattn::launch_wait_selftest(wait_us, static_cast<cudaStream_t>(stream));
 }
 
+extern "C" int seg_attn_stall_test(int withhold_k_tile, int wait_us) {
+  if (wait_us < 1 || wait_us > 1000000) return SEG_ATTN_ERR_INVALID_ARG;
+  return segattn::set_stall_test(withhold_k_tile, wait_us);
+}
+
 extern "C" int seg_attn_take_device_error(int* value) {
   if (!value) return SEG_ATTN_ERR_INVALID_ARG;
   int wait_err = 0, append_err = 0;

@@ -119,6 +119,10 @@ struct DecodeParams {
   float* part_lse;
   float scale_log2;
   int q_heads, kv_heads, group;
+  // query heads per CTA: hs = min(group, 8) packed heads (the mma's N = 8 side);
+  // a group larger than 8 is covered by `slices` = group / 8 CTAs per (chunk, kv
+  // head), adjacent in the grid so the siblings' K/V reads hit L2
+  int hs, slices;
 };
 
 // Merge the four warps' (m, l, O) of this chunk through shared memory and write
@@ -126,12 +130,12 @@ struct DecodeParams {
 template <int D>
 __device__ __forceinline__ void write_chunk_result(const DecodeParams& p, float (&sm_o)[kDecodeWarps][8][D],
                                                    float (&sm_m)[kDecodeWarps][8],
-                                                   float (&sm_l)[kDecodeWarps][8], int req, int g,
-                                                   int n_chunks, float out_scale) {
+                                                   float (&sm_l)[kDecodeWarps][8], int req, int chunk,
+                                                   int h0, int n_chunks, float out_scale) {
   constexpr int PER_THREAD = 8 * D / kDecodeThreads;  // outputs per thread
   const int hh = threadIdx.x / (D / PER_THREAD);
   const int d0 = (threadIdx.x % (D / PER_THREAD)) * PER_THREAD;
-  if (hh >= p.group) return;
+  if (hh >= p.hs) return;
   float mw[kDecodeWarps], M = -INFINITY;
 #pragma unroll
   for (int w = 0; w < kDecodeWarps; ++w) {
@@ -150,7 +154,7 @@ __device__ __forceinline__ void write_chunk_result(const DecodeParams& p, float 
     for (int e = 0; e < PER_THREAD; ++e) acc[e] += a * sm_o[w][hh][d0 + e];
   }
   const float inv = L > 0.f ? out_scale / L : 0.f;
-  const int head = g * p.group + hh;
+  const int head = h0 + hh;
   const float lse2 = L > 0.f ? Mb + log2f(L) : -INFINITY;
   if (n_chunks == 1) {
     const int tok = __ldg(p.tab.q_offsets + req);
@@ -164,12 +168,12 @@ __device__ __forceinline__ void write_chunk_result(const DecodeParams& p, float 
     }
     if (p.lse && d0 == 0) p.lse[(int64_t)tok * p.q_heads + head] = lse2 * 0.69314718055994531f;
   } else {
-    float* prow = p.part_o + ((int64_t)blockIdx.x * p.q_heads + head) * D + d0;
+    float* prow = p.part_o + ((int64_t)chunk * p.q_heads + head) * D + d0;
 #pragma unroll
     for (int e = 0; e < PER_THREAD; e += 4)
       *reinterpret_cast<float4*>(prow + e) =
           make_float4(acc[e] * inv, acc[e + 1] * inv, acc[e + 2] * inv, acc[e + 3] * inv);
-    if (d0 == 0) p.part_lse[(int64_t)blockIdx.x * p.q_heads + head] = lse2;
+    if (d0 == 0) p.part_lse[(int64_t)chunk * p.q_heads + head] = lse2;
   }
 }
 
@@ -183,22 +187,24 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_chunk_kernel(const D
   __shared__ float sm_m[kDecodeWarps][8];
   __shared__ float sm_l[kDecodeWarps][8];
 
-  const int4 item = p.tab.work[blockIdx.x];
+  const int chunk = blockIdx.x / p.slices;
+  const int4 item = p.tab.work[chunk];
   const int req = item.x, k_begin = item.y, k_end = item.z, n_chunks = item.w;
   const int g = blockIdx.y;
+  const int h0 = g * p.group + (blockIdx.x - chunk * p.slices) * 8;  // first query head here
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = lane >> 2, qd = lane & 3;
   const int64_t kv_stride = (int64_t)p.kv_heads * D;  // elements between consecutive slots
 
-  // Q^T operand fragments of the packed heads (head r of this group; zero pad past G).
+  // Q^T operand fragments of the packed heads (head h0 + r; zero pad past hs).
   uint32_t qf[KSTEPS][2];
   {
     const int tok = __ldg(p.tab.q_offsets + req);
-    const __nv_bfloat16* qrow = p.q + ((int64_t)tok * p.q_heads + (int64_t)g * p.group + r) * D;
+    const __nv_bfloat16* qrow = p.q + ((int64_t)tok * p.q_heads + h0 + r) * D;
 #pragma unroll
     for (int t = 0; t < KCH; ++t) {
       uint4 w = make_uint4(0, 0, 0, 0);
-      if (r < p.group) w = *reinterpret_cast<const uint4*>(qrow + 8 * (qd + 4 * t));
+      if (r < p.hs) w = *reinterpret_cast<const uint4*>(qrow + 8 * (qd + 4 * t));
       qf[2 * t][0] = w.x;
       qf[2 * t][1] = w.y;
       qf[2 * t + 1][0] = w.z;
@@ -347,7 +353,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_chunk_kernel(const D
   }
   __syncthreads();
 
-  write_chunk_result<D>(p, sm_o, sm_m, sm_l, req, g, n_chunks, 1.f);
+  write_chunk_result<D>(p, sm_o, sm_m, sm_l, req, chunk, h0, n_chunks, 1.f);
 }
 
 // FP8 (E4M3) KV cache: same split-K structure, half the bytes.  The E4M3
@@ -370,23 +376,25 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_chunk_fp8_kernel(con
   __shared__ float sm_m[kDecodeWarps][8];
   __shared__ float sm_l[kDecodeWarps][8];
 
-  const int4 item = p.tab.work[blockIdx.x];
+  const int chunk = blockIdx.x / p.slices;
+  const int4 item = p.tab.work[chunk];
   const int req = item.x, k_begin = item.y, k_end = item.z, n_chunks = item.w;
   const int g = blockIdx.y;
+  const int h0 = g * p.group + (blockIdx.x - chunk * p.slices) * 8;  // first query head here
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = lane >> 2, qd = lane & 3;
   const int64_t kv_stride = (int64_t)p.kv_heads * D;  // bytes between consecutive slots
   const float sl2 = p.scale_log2 * __ldg(p.k_scale + g);
   const float v_scale = __ldg(p.v_scale + g);
 
-  uint32_t qf[KSTEPS][2];  // f16 Q^T fragments of head r of the group
+  uint32_t qf[KSTEPS][2];  // f16 Q^T fragments of head h0 + r (zero past hs)
   {
     const int tok = __ldg(p.tab.q_offsets + req);
-    const __nv_bfloat16* qrow = p.q + ((int64_t)tok * p.q_heads + (int64_t)g * p.group + r) * D;
+    const __nv_bfloat16* qrow = p.q + ((int64_t)tok * p.q_heads + h0 + r) * D;
 #pragma unroll
     for (int t = 0; t < KCH; ++t) {
       uint4 w0 = make_uint4(0, 0, 0, 0), w1 = make_uint4(0, 0, 0, 0);
-      if (r < p.group) {
+      if (r < p.hs) {
         w0 = *reinterpret_cast<const uint4*>(qrow + 16 * (qd + 4 * t));
         w1 = *reinterpret_cast<const uint4*>(qrow + 16 * (qd + 4 * t) + 8);
       }
@@ -542,7 +550,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_chunk_fp8_kernel(con
     sm_o[warp][2 * qd + 1][d0 + 1] = o[i][3];
   }
   __syncthreads();
-  write_chunk_result<D>(p, sm_o, sm_m, sm_l, req, g, n_chunks, v_scale);
+  write_chunk_result<D>(p, sm_o, sm_m, sm_l, req, chunk, h0, n_chunks, v_scale);
 }
 
 // Merge the chunk partials of each multi-chunk request (one warp per head).
@@ -605,10 +613,13 @@ int launch_decode_d(const DecodeLaunch& a, cudaStream_t stream) {
   p.q_heads = d.q_heads;
   p.kv_heads = d.kv_heads;
   p.group = d.q_heads / d.kv_heads;
+  p.hs = p.group < 8 ? p.group : 8;
+  p.slices = p.group / p.hs;
+  const dim3 grid(d.num_work * p.slices, d.kv_heads);
   if (a.fp8)
-    decode_chunk_fp8_kernel<D><<<dim3(d.num_work, d.kv_heads), kDecodeThreads, 0, stream>>>(p);
+    decode_chunk_fp8_kernel<D><<<grid, kDecodeThreads, 0, stream>>>(p);
   else
-    decode_chunk_kernel<D><<<dim3(d.num_work, d.kv_heads), kDecodeThreads, 0, stream>>>(p);
+    decode_chunk_kernel<D><<<grid, kDecodeThreads, 0, stream>>>(p);
   if (cudaGetLastError() != cudaSuccess) return SEG_ATTN_ERR_CUDA;
   // a shared-prefix table leaves every merge to the cascade merge
   if (d.workspace_bytes > 0 && !d.shared) {

@@ -51,6 +51,7 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "ptx_sm100.cuh"
@@ -66,7 +67,11 @@ constexpr int kThreads = 320;
 // FP8 cache: two more warps (10, 11) widen E4M3 code tiles to f16 in shared memory
 constexpr int kThreadsFp8 = 384;
 constexpr int kConvThreads = 64;
-constexpr uint64_t kWaitLimitNs = 1000000000ull;
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // default limit of a bounded wait
+// Stall test (off by default): the K tile at which every later prefill CTA's
+// producer stops loading (-1: none), and the limit of its bounded waits.
+std::atomic<int> g_stall_tile{-1};
+std::atomic<uint64_t> g_stall_wait_ns{kWaitLimitNs};
 constexpr float kRescaleLog2 = 8.0f;
 // Two tiles: a tile's softmax signals after this many 32-key chunks of its
 // current K tile that its next S may be computed; the chunks left take about
@@ -86,6 +91,8 @@ struct PrefillParams {
   int work_base;    // first work item of this launch
   const float* k_scale;  // FP8 cache: [kv_heads] dequantisation scales (value = code * scale)
   const float* v_scale;
+  uint64_t wait_ns;      // limit of every bounded wait (1 s unless a stall test shortens it)
+  int withhold_tile;     // stall test: the producer stops before loading this K tile (-1: off)
 };
 
 // Query region + K ring + V ring + barriers + alignment slack.  The query
@@ -258,6 +265,8 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
   uint64_t* s_soon = bars + 26;     // [2] two tiles: the tile's softmax is near the end of a K tile
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 28);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  // limit of every bounded wait, read only when a wait checks it
+  volatile uint64_t* wait_limit = reinterpret_cast<volatile uint64_t*>(bars + 29);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // piece: keys tiles [kt0, kt1) of item (request, kv head g, query tiles from q0);
@@ -303,6 +312,7 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
       mbar_init(vst_empty, kConvThreads);
     }
     *abort_flag = 0;
+    *wait_limit = p.wait_ns;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -386,9 +396,12 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
         }
       };
       auto load_k = [&](int i, const TileRows& tr) -> bool {
+        // stall test: stop loading here, as a copy that never lands would; the
+        // consumers' bounded waits then give up and the CTA drains and exits
+        if (i == p.withhold_tile) return false;
         const int st = i % RK;
         if (!__all_sync(0xffffffffu, mbar_wait(k_empty + st, ((i / RK) & 1) ^ 1, abort_flag,
-                                               kWaitLimitNs, true)))
+                                               wait_limit, true)))
           return false;
         load_tile(tr, sK + st * TILE, &tm_k3, &tm_k, k_full + st);
         ++k_issued;
@@ -397,7 +410,7 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
       auto load_v = [&](int i, const TileRows& tr) -> bool {
         const int st = i % RV;
         if (!__all_sync(0xffffffffu, mbar_wait(v_empty + st, ((i / RV) & 1) ^ 1, abort_flag,
-                                               kWaitLimitNs, true)))
+                                               wait_limit, true)))
           return false;
         load_tile(tr, sV + st * TILE, &tm_v3, &tm_v, v_full + st);
         ++v_issued;
@@ -408,17 +421,18 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
         for (int i = 0; i < n_tiles; ++i) {
           TileRows tr;
           tile_rows(i, tr);
-          if (!__all_sync(0xffffffffu, mbar_wait(kst_empty, (i & 1) ^ 1, abort_flag, kWaitLimitNs, true))) break;
+          if (i == p.withhold_tile) break;  // stall test (see load_k)
+          if (!__all_sync(0xffffffffu, mbar_wait(kst_empty, (i & 1) ^ 1, abort_flag, wait_limit, true))) break;
           load_codes(tr, sStK, &tm_k3, &tm_k, kst_full);
           ++k_issued;
-          if (!__all_sync(0xffffffffu, mbar_wait(vst_empty, (i & 1) ^ 1, abort_flag, kWaitLimitNs, true))) break;
+          if (!__all_sync(0xffffffffu, mbar_wait(vst_empty, (i & 1) ^ 1, abort_flag, wait_limit, true))) break;
           load_codes(tr, sStV, &tm_v3, &tm_v, vst_full);
           ++v_issued;
         }
         // never leave the CTA with copies in flight (a staged copy is issued only
         // after the converters read the previous one, so the last is enough)
-        if (k_issued > 0) mbar_wait(kst_full, (k_issued - 1) & 1, nullptr, kWaitLimitNs);
-        if (v_issued > 0) mbar_wait(vst_full, (v_issued - 1) & 1, nullptr, kWaitLimitNs);
+        if (k_issued > 0) mbar_wait(kst_full, (k_issued - 1) & 1, nullptr, wait_limit);
+        if (v_issued > 0) mbar_wait(vst_full, (v_issued - 1) & 1, nullptr, wait_limit);
       } else {
         // K tile i + 1 before V tile i: the MMA warp takes them in that order
         TileRows cur, nxt;
@@ -436,15 +450,15 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
         for (int s = 0; s < RK; ++s)
           if (k_issued > s) {
             const int last = s + RK * ((k_issued - 1 - s) / RK);
-            mbar_wait(k_full + s, (last / RK) & 1, nullptr, kWaitLimitNs);
+            mbar_wait(k_full + s, (last / RK) & 1, nullptr, wait_limit);
           }
         for (int s = 0; s < RV; ++s)
           if (v_issued > s) {
             const int last = s + RV * ((v_issued - 1 - s) / RV);
-            mbar_wait(v_full + s, (last / RV) & 1, nullptr, kWaitLimitNs);
+            mbar_wait(v_full + s, (last / RV) & 1, nullptr, wait_limit);
           }
       }
-      if (lane == 0) mbar_wait(q_full, 0, nullptr, kWaitLimitNs);
+      if (lane == 0) mbar_wait(q_full, 0, nullptr, wait_limit);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -452,7 +466,7 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
     // executes each tcgen05.mma / commit.
     if (n_tiles > 0) {
       auto wait_all = [&](uint64_t* bar, uint32_t parity) {
-        return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, kWaitLimitNs, true));
+        return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, wait_limit, true));
       };
       const uint32_t idesc_qk =
           FP8 ? idesc_f16_f32(128, 128, false) : idesc_bf16_f32(128, 128, false);
@@ -639,7 +653,7 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
       }
       // all MMAs finished before tensor memory is released
       mma_commit_warp(mma_done);
-      mbar_wait(mma_done, 0, nullptr, kWaitLimitNs);
+      mbar_wait(mma_done, 0, nullptr, wait_limit);
     }
     __syncwarp();
   } else if (FP8 && warp >= 10) {
@@ -650,15 +664,15 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
     bool ok = true;
     for (int i = 0; ok && i < n_tiles; ++i) {
       const int sk = i % RK, sv = i % RV;
-      if (!(ok = mbar_wait(kst_full, i & 1, abort_flag, kWaitLimitNs) &&
-                 mbar_wait(k_empty + sk, ((i / RK) & 1) ^ 1, abort_flag, kWaitLimitNs)))
+      if (!(ok = mbar_wait(kst_full, i & 1, abort_flag, wait_limit) &&
+                 mbar_wait(k_empty + sk, ((i / RK) & 1) ^ 1, abort_flag, wait_limit)))
         break;
       widen_tile<D>(sStK, sK + sk * TILE, ct);
       fence_proxy_async_smem();
       mbar_arrive(k_full + sk);
       mbar_arrive(kst_empty);
-      if (!(ok = mbar_wait(vst_full, i & 1, abort_flag, kWaitLimitNs) &&
-                 mbar_wait(v_empty + sv, ((i / RV) & 1) ^ 1, abort_flag, kWaitLimitNs)))
+      if (!(ok = mbar_wait(vst_full, i & 1, abort_flag, wait_limit) &&
+                 mbar_wait(v_empty + sv, ((i / RV) & 1) ^ 1, abort_flag, wait_limit)))
         break;
       widen_tile<D>(sStV, sV + sv * TILE, ct);
       fence_proxy_async_smem();
@@ -689,7 +703,7 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
       // shared-memory banks).  One tile: bf16 -> f16 in place (FP8 cache).  Two
       // tiles: into this row's TMEM lane, 2 elements per column (f16 over an
       // FP8 cache), the layout of a tensor-memory A operand.
-      ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, abort_flag, kWaitLimitNs));
+      ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, abort_flag, wait_limit));
       if (ok && !QT) {
 #pragma unroll
         for (int h = 0; h < HALVES; ++h)
@@ -790,7 +804,7 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
       bool waited = false;
       if (QT && i > 0) {
         if (!__all_sync(0xffffffffu,
-                        mbar_wait(o_full + t, (i - 1) & 1, abort_flag, kWaitLimitNs, true)))
+                        mbar_wait(o_full + t, (i - 1) & 1, abort_flag, wait_limit, true)))
           return false;
         tc_fence_after();
         waited = true;
@@ -826,7 +840,7 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
       if (__any_sync(0xffffffffu, rescale)) {
         // O_t holds PV up to K tile i - 1; rescale it in place once that is complete
         if (!waited &&
-            !__all_sync(0xffffffffu, mbar_wait(o_full + t, (i - 1) & 1, abort_flag, kWaitLimitNs)))
+            !__all_sync(0xffffffffu, mbar_wait(o_full + t, (i - 1) & 1, abort_flag, wait_limit)))
           return false;
         tc_fence_after();
 #pragma unroll
@@ -848,7 +862,7 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
     // one K tile of softmax on S buffer sb (phase sph of its barriers)
     auto run_tile = [&](int i, int sb, uint32_t sph) -> bool {
       if (single) tS = lane_base + 256 + 128 * sb;
-      if (!__all_sync(0xffffffffu, mbar_wait(s_full + sb, sph, abort_flag, kWaitLimitNs, true)))
+      if (!__all_sync(0xffffffffu, mbar_wait(s_full + sb, sph, abort_flag, wait_limit, true)))
         return false;
       if (!warp_live) {
         if (QT) {
@@ -857,7 +871,7 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(s_free);
           if (i > 0 &&
-              !__all_sync(0xffffffffu, mbar_wait(o_full + t, (i - 1) & 1, abort_flag, kWaitLimitNs)))
+              !__all_sync(0xffffffffu, mbar_wait(o_full + t, (i - 1) & 1, abort_flag, wait_limit)))
             return false;
           mbar_arrive(s_soon + t);
         }
@@ -903,10 +917,10 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
     // first, since a parity wait tells apart just two consecutive phases
     if (ok && single && n_tiles > 1)
       ok = __all_sync(0xffffffffu,
-                      mbar_wait(o_full + t, (n_tiles - 2) & 1, abort_flag, kWaitLimitNs));
+                      mbar_wait(o_full + t, (n_tiles - 2) & 1, abort_flag, wait_limit));
     if (ok && n_tiles > 0)
       ok = __all_sync(0xffffffffu,
-                      mbar_wait(o_full + t, (n_tiles - 1) & 1, abort_flag, kWaitLimitNs));
+                      mbar_wait(o_full + t, (n_tiles - 1) & 1, abort_flag, wait_limit));
     if (ok && slot >= 0) {
       // piece of a split item (or of a shared-prefix pass): O / l and log2(sum of exp)
       // of this key range, for every row that holds a query
@@ -1092,6 +1106,8 @@ int launch_prefill_d(const PrefillLaunch& a, cudaStream_t stream) {
   p.part_lse = a.part_lse;
   p.k_scale = a.k_scale;
   p.v_scale = a.v_scale;
+  p.wait_ns = g_stall_wait_ns.load();
+  p.withhold_tile = g_stall_tile.load();
   // two-tile items first, then the single-tile items listed at the end
   const int n_single = d.num_single, n_two = d.num_work - d.num_single;
   if (n_two > 0) {
@@ -1143,6 +1159,12 @@ __global__ void __launch_bounds__(32) wait_selftest_kernel(uint64_t limit_ns) {
 }
 
 }  // namespace
+
+int set_stall_test(int withhold_k_tile, int wait_us) {
+  g_stall_tile.store(withhold_k_tile < 0 ? -1 : withhold_k_tile);
+  g_stall_wait_ns.store((uint64_t)wait_us * 1000ull);
+  return SEG_ATTN_OK;
+}
 
 int launch_wait_selftest(int wait_us, cudaStream_t stream) {
   wait_selftest_kernel<<<1, 32, 0, stream>>>((uint64_t)wait_us * 1000ull);

@@ -83,6 +83,26 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// The same with the limit read from memory (shared memory, set once per CTA)
+// only when it is checked, so a run-time limit costs no register in the
+// loops around the wait.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          const volatile uint64_t* limit_ns, bool suspend = false) {
+  const uint32_t a = smem_u32(bar);
+  if (mbar_try_wait(a, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (suspend ? mbar_try_wait_suspend(a, parity, 200000u) : mbar_try_wait(a, parity)) return true;
+    if ((it & 15) == 0) {
+      if (abort && *abort) return false;
+      if (globaltimer_ns() - t0 > *limit_ns) {
+        if (abort) *abort = 1;
+        return false;
+      }
+    }
+  }
+}
+
 // ---------------------------------------------------------------- programmatic dependent launch
 // Let the grid launched after this one on the stream (as its programmatic
 // dependent) start now.

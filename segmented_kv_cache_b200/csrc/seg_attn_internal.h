@@ -116,6 +116,8 @@ int launch_decode(const DecodeLaunch& a, cudaStream_t stream);
 // Read and clear the device error words: a bounded wait that gave up (prefill)
 // and a KV-append slot out of range.
 int launch_wait_selftest(int wait_us, cudaStream_t stream);
+// Stall test of the prefill kernel (seg_attn_stall_test).
+int set_stall_test(int withhold_k_tile, int wait_us);
 int take_device_error(int* value);
 int take_append_error(int* value);
 

@@ -252,8 +252,10 @@ extern "C" int seg_attn_build_table(int batch, const int32_t* q_lens, const int3
   const int group = q_heads / kv_heads;
   if (head_dim != 64 && head_dim != 128) return SEG_ATTN_ERR_UNSUPPORTED;
   if (!is_pow2(group)) return SEG_ATTN_ERR_UNSUPPORTED;
-  if (mode == SEG_ATTN_MODE_PREFILL && group > segattn::kTileRows) return SEG_ATTN_ERR_UNSUPPORTED;
-  if (mode == SEG_ATTN_MODE_DECODE && group > 8) return SEG_ATTN_ERR_UNSUPPORTED;
+  // a prefill query tile packs whole groups; decode packs up to 8 heads per CTA and
+  // covers a larger group with group / 8 sibling CTAs (and a shared-prefix decode
+  // runs its prefix pass on the prefill kernel)
+  if (group > segattn::kTileRows) return SEG_ATTN_ERR_UNSUPPORTED;
   // the K/V gather addresses pool rows (slot * kv_heads + head) with int32
   if (num_slots * (int64_t)kv_heads > (int64_t)std::numeric_limits<int32_t>::max())
     return SEG_ATTN_ERR_UNSUPPORTED;
@@ -360,10 +362,11 @@ extern "C" int seg_attn_build_table(int batch, const int32_t* q_lens, const int3
     main_citem = main_pieces.citem;
   } else {
     int64_t L = 4096;
+    const int64_t slices = group > 8 ? group / 8 : 1;  // CTAs per (chunk, kv head)
     auto ctas = [&](int64_t len) {
       int64_t n = 0;
       for (int r = 0; r < batch; ++r) n += std::max<int64_t>(1, (okl[r] + len - 1) / len);
-      return n * kv_heads;
+      return n * kv_heads * slices;
     };
     while (L > 256 && ctas(L) < segattn::kDecodeTargetCtas) L /= 2;
     chunk_len = (int32_t)L;
@@ -381,7 +384,9 @@ extern "C" int seg_attn_build_table(int batch, const int32_t* q_lens, const int3
     }
   }
   const size_t n_work = mode == SEG_ATTN_MODE_PREFILL ? main_pieces.work.size() : work.size();
-  if (n_work > (size_t)kI32Max) return SEG_ATTN_ERR_UNSUPPORTED;
+  // decode launches n_work * (group / 8) CTAs along the grid's x dimension
+  const size_t grid_x = n_work * (mode == SEG_ATTN_MODE_DECODE && group > 8 ? group / 8 : 1);
+  if (grid_x > (size_t)kI32Max) return SEG_ATTN_ERR_UNSUPPORTED;
 
   // ---- shared-prefix pass and cascade rows
   std::vector<int32_t> gq_off, greq;      // per group: first query row, first request

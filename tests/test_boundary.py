@@ -72,7 +72,11 @@ def test_validation_errors():
     assert code_of(lambda: build([1], [[(10, 4)]], hq=6, hkv=4)) == S["INVALID_ARG"]
     assert code_of(lambda: build([1], [[(10, 4)]], d=96)) == S["UNSUPPORTED"]
     assert code_of(lambda: build([1], [[(10, 4)]], hq=6, hkv=2)) == S["UNSUPPORTED"]  # G=3
-    assert code_of(lambda: build([1], [[(10, 4)]], hq=32, hkv=2, mode=sa.MODE_DECODE)) == S["UNSUPPORTED"]
+    # decode covers groups above 8 with sibling CTAs of 8 heads each; 256 is past the limit
+    build([1], [[(10, 4)]], hq=32, hkv=2, mode=sa.MODE_DECODE)
+    build([1], [[(10, 4)]], hq=128, hkv=1, mode=sa.MODE_DECODE)
+    assert code_of(lambda: build([1], [[(10, 4)]], hq=256, hkv=1, mode=sa.MODE_DECODE)) == S["UNSUPPORTED"]
+    assert code_of(lambda: build([1], [[(10, 4)]], hq=256, hkv=1)) == S["UNSUPPORTED"]
     assert code_of(lambda: build([2], [[(10, 4)]], mode=sa.MODE_DECODE)) == S["INVALID_ARG"]
     # the same slots in two requests are legal (shared read-only prefix)
     build([1, 1], [[(10, 4)], [(10, 4)]])

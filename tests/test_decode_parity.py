@@ -100,6 +100,21 @@ def test_decode_split_choice_does_not_change_result():
     assert (lse2 - lse1).abs().max() <= 1e-5
 
 
+@pytest.mark.parametrize("d,hq,hkv", [(128, 32, 2), (64, 64, 1), (128, 128, 1), (64, 32, 4)])
+def test_decode_groups_above_eight(d, hq, hkv):
+    # G = 16, 64, 128, 8 x 4: the group's heads are split over sibling CTAs of 8 heads;
+    # long requests make several chunks (merged), short ones a single chunk (final output)
+    case = random_case(70 + hq + d, batch=5, hq=hq, hkv=hkv, d=d, causal=True, max_k=9000,
+                       nseg_max=5, q_mode="decode")
+    # one request of a single short segment (a prefix of its first segment's slots)
+    case["seg_lens"][0] = [min(7, case["seg_lens"][0][0])]
+    case["seg_starts"][0] = case["seg_starts"][0][:1]
+    _, tab = _check_case(case, f"decode d{d} {hq}/{hkv}")
+    rc = tab.host[tab.desc.off_req_chunks: tab.desc.off_req_chunks + 6].tolist()
+    n = np.diff(rc)
+    assert n.max() > 1 and n.min() == 1
+
+
 @pytest.mark.parametrize("cfg", [4])
 def test_config4_sampled_requests(cfg):
     wl = synth.make_workload(cfg, device="cuda")

@@ -1,5 +1,8 @@
 """Failure detection without a GPU fault: a wait that nothing completes must give up
-after its limit, surface as the device error word, and leave the context usable."""
+after its limit, surface as the device error word, and leave the context usable --
+for a lone diagnostic warp, and for the prefill kernel itself when its producer
+withholds a K tile (the stall test switch), which exercises the kernel's drain of
+the copies and MMAs already in flight and its release of tensor memory."""
 import pytest
 import torch
 
@@ -16,6 +19,80 @@ def test_wait_selftest_rejects_out_of_range_limits():
     lib = sa.load_library()
     for bad in (0, -5, 1000001):
         assert lib.seg_attn_wait_selftest(bad, None) == S["INVALID_ARG"]
+        assert lib.seg_attn_stall_test(-1, bad) == S["INVALID_ARG"]
+    assert lib.seg_attn_stall_test(-1, 1000000) == 0  # the defaults
+
+
+def _stall_case(q_per_req, hq=8, hkv=2, d=128):
+    """Request 0 has 200 keys (2 K tiles), request 1 has 1000 (8 K tiles); non-causal, so
+    every item of request 1 reaches K tile 2 and every item of request 0 stops short."""
+    case = random_case(62, batch=2, hq=hq, hkv=hkv, d=d, causal=False, max_k=4)
+    g = torch.Generator().manual_seed(63)
+    S_ = 1700
+    k = torch.full((S_, hkv, d), float("nan"))
+    v = torch.full((S_, hkv, d), float("nan"))
+    starts = [[10, 230], [600, 1300]]  # two segments per request, free (NaN) slots between
+    lens = [[120, 80], [650, 350]]
+    for ss, ll in zip(starts, lens):
+        for s0, l in zip(ss, ll):
+            k[s0:s0 + l] = torch.randn(l, hkv, d, generator=g)
+            v[s0:s0 + l] = torch.randn(l, hkv, d, generator=g)
+    case.update(q_lens=[q_per_req, q_per_req], seg_starts=starts, seg_lens=lens, num_slots=S_,
+                k_pool=k.to(torch.bfloat16), v_pool=v.to(torch.bfloat16),
+                q=torch.randn(2 * q_per_req, hq, d, generator=g).to(torch.bfloat16))
+    return case
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("variant", ["two-tile", "one-tile", "e4m3"])
+def test_prefill_gives_up_on_a_withheld_tile_and_recovers(variant):
+    """The producer stops before K tile 2: CTAs of request 1 (8 tiles) wait, give up after
+    1 ms, drain and exit without writing their rows; CTAs of request 0 (2 tiles) finish.
+    Afterwards the same process computes a normal prefill correctly."""
+    from segmented_kv_cache_b200 import synth
+    q_per_req = 20 if variant == "one-tile" else 50  # qpt = 128 / 4 = 32 queries per tile
+    case = _stall_case(q_per_req)
+    c = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in case.items()}
+    tab = sa.SegTable.build(case["q_lens"], case["seg_starts"], case["seg_lens"],
+                            case["num_slots"], False, sa.MODE_PREFILL, 8, 2, 128).to("cuda")
+    assert (tab.desc.num_single == tab.desc.num_work) == (variant == "one-tile")
+    assert tab.workspace_bytes == 0  # no split pieces: each item is one CTA
+    out = torch.full_like(c["q"], float("nan"))
+    lse = torch.full(c["q"].shape[:2], float("nan"), dtype=torch.float32, device="cuda")
+    if variant == "e4m3":
+        k8, v8, ks, vs = synth.fp8_pools(case["k_pool"], case["v_pool"])
+        k8, v8, ks, vs = k8.cuda(), v8.cuda(), ks.cuda(), vs.cuda()
+        call = lambda: sa.seg_attn_prefill_fp8(c["q"], k8, v8, ks, vs, out, lse, tab.device,
+                                               tab.desc, case["scale"], None)
+        ref_o, ref_l = oracle.attention_fp8(case["q_lens"], case["seg_starts"], case["seg_lens"],
+                                            case["q"], k8.cpu(), v8.cpu(), ks.cpu(), vs.cpu(),
+                                            case["scale"], False)
+    else:
+        call = lambda: sa.seg_attn_prefill(c["q"], c["k_pool"], c["v_pool"], out, lse, tab.device,
+                                           tab.desc, case["scale"], None)
+        ref_o, ref_l = oracle.attention(case["q_lens"], case["seg_starts"], case["seg_lens"],
+                                        case["q"], case["k_pool"], case["v_pool"], case["scale"],
+                                        False)
+    assert sa.seg_attn_take_device_error() == 0
+    try:
+        sa.seg_attn_stall_test(2, 1000)
+        call()
+        torch.cuda.synchronize()
+    finally:
+        sa.seg_attn_stall_test(-1, 1000000)
+    assert sa.seg_attn_take_device_error() == 1
+    assert sa.seg_attn_take_device_error() == 0
+    n0 = q_per_req
+    # request 0 finished normally; request 1's CTAs gave up and wrote nothing
+    compare(out[:n0], lse[:n0], ref_o[:n0], ref_l[:n0], f"stall test {variant}: finished CTAs")
+    assert torch.isnan(out[n0:].float()).all() and torch.isnan(lse[n0:]).all()
+    # the context is intact: the same call without the stall matches the oracle everywhere
+    out.fill_(float("nan"))
+    lse.fill_(float("nan"))
+    call()
+    torch.cuda.synchronize()
+    compare(out, lse, ref_o, ref_l, f"after the stall test ({variant})")
+    assert sa.seg_attn_take_device_error() == 0
 
 
 @pytest.mark.gpu

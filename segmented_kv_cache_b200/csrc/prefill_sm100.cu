@@ -270,14 +270,15 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // piece: keys tiles [kt0, kt1) of item (request, kv head g, query tiles from q0);
-  // slot >= 0 when the item is split and this piece writes a partial result
+  // slot >= 0 when the item is split and this piece writes a partial result.  The
+  // row also carries the request's first query row, queries, keys and the segment
+  // of the piece's first key, so no dependent table load precedes the first copies.
   const int item = p.work_base + blockIdx.x;
-  const int4 w0 = p.tab.work[2 * item], w1 = p.tab.work[2 * item + 1];
-  const int req = w0.x, g = w0.y, q0 = w0.z, kt0 = w0.w, slot = w1.y;
+  const int4 w0 = p.tab.work[3 * item], w1 = p.tab.work[3 * item + 1];
+  const int4 w2 = p.tab.work[3 * item + 2];
+  const int g = w0.y, q0 = w0.z, kt0 = w0.w, slot = w1.y;
   const int n_tiles = w1.x - kt0;
-  const int tok0 = __ldg(p.tab.q_offsets + req);
-  const int q_len = __ldg(p.tab.q_offsets + req + 1) - tok0;
-  const int k_len = __ldg(p.tab.k_lens + req);
+  const int tok0 = w2.x, q_len = w2.y, k_len = w2.z;
   // Only query tile 0 holds queries (a short chunk, or the packed queries of a
   // small shared-prefix group): tile 1 is skipped and its S columns become a
   // second S buffer of tile 0, so the next tile's S = QK^T overlaps this tile's
@@ -340,8 +341,8 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
             tma_load_3d(sQ + t * QSTRIDE + h * kHalfBytes, &tm_q, q_full, 64 * h, g * p.group,
                         tok0 + q0 + t * p.qpt);
       }
-      int seg = __ldg(p.tab.seg_offsets + req);
-      const int seg_end = __ldg(p.tab.seg_offsets + req + 1);
+      int seg = w2.w;
+      const int seg_end = w1.w;
       // Pool rows of K tile i: lane l holds logical keys 4l .. 4l + 3 (keys past the
       // request are clamped to its last key).  Most tiles are 128 consecutive pool
       // slots (segments are long): one tiled box per 64-column half; tiles that
@@ -921,43 +922,76 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
     if (ok && n_tiles > 0)
       ok = __all_sync(0xffffffffu,
                       mbar_wait(o_full + t, (n_tiles - 1) & 1, abort_flag, wait_limit));
+    // Results leave through shared memory so that a warp stores whole rows: a thread
+    // owns one row, and its own 16-byte pieces of it would put every warp store on 32
+    // different lines.  Each warp stages its 32 rows in a quarter of the tile's query
+    // / P region (free: the commit of the tile's last PV covers every earlier MMA),
+    // 16-byte chunk c of row-local r at ((c & ~7) | ((c ^ r) & 7)), then copies rows
+    // out with consecutive lanes on consecutive chunks.
+    uint8_t* stage_w = sQ + t * QSTRIDE + quad * (QSTRIDE / 4);
+    auto swz = [](int c, int r) { return (c & ~7) | ((c ^ r) & 7); };
     if (ok && slot >= 0) {
       // piece of a split item (or of a shared-prefix pass): O / l and log2(sum of exp)
-      // of this key range, for every row that holds a query
+      // of this key range, for every row that holds a query; fp32 rows go out in
+      // passes of PCOLS columns (the staging quarter holds 32 rows of PCOLS floats)
+      constexpr int PCOLS = (int)(QSTRIDE / 512) < D ? (int)(QSTRIDE / 512) : D;
+      constexpr int PCH = PCOLS / 4;        // 16-byte chunks per row per pass
+      constexpr int RPI = 32 / PCH;         // rows per warp instruction of the copy
       const float inv = l > 0.f ? (FP8 ? __ldg(p.v_scale + g) : 1.f) / l : 0.f;
-      const int64_t prow = (int64_t)slot * kItemRows + t * kTileRows + row;
-      float* po = p.part_o + prow * D;
+      const int64_t prow0 = (int64_t)slot * kItemRows + t * kTileRows + quad * 32;
+      uint32_t o[D / 32][32];
+      load_o(o);
+#pragma unroll
+      for (int pass = 0; pass < D / PCOLS; ++pass) {
+#pragma unroll
+        for (int c = 0; c < PCH; ++c) {
+          const int col = pass * PCOLS + 4 * c;
+          const float4 v = make_float4(__uint_as_float(o[col / 32][col % 32]) * inv,
+                                       __uint_as_float(o[col / 32][col % 32 + 1]) * inv,
+                                       __uint_as_float(o[col / 32][col % 32 + 2]) * inv,
+                                       __uint_as_float(o[col / 32][col % 32 + 3]) * inv);
+          *reinterpret_cast<float4*>(stage_w + lane * (PCOLS * 4) + swz(c, lane) * 16) = v;
+        }
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < 32; k += RPI) {
+          const int lr = k + lane / PCH, c = lane % PCH;
+          const int qi_r = q0 + t * p.qpt + (quad * 32 + lr) / p.group;
+          if (qi_r < q_len)
+            *reinterpret_cast<float4*>(p.part_o + (prow0 + lr) * D + pass * PCOLS + 4 * c) =
+                *reinterpret_cast<const float4*>(stage_w + lr * (PCOLS * 4) + swz(c, lr) * 16);
+        }
+        __syncwarp();
+      }
+      if (row_valid) p.part_lse[prow0 + lane] = l > 0.f ? m_ref * sl2 + log2f(l) : -INFINITY;
+    } else if (ok) {
+      constexpr int CH = D / 8;    // 16-byte chunks of a bf16 row
+      constexpr int RPI = 32 / CH; // rows per warp instruction of the copy
+      const float inv = l > 0.f ? (FP8 ? __ldg(p.v_scale + g) : 1.f) / l : 0.f;
       uint32_t o[D / 32][32];
       load_o(o);
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
-        if (row_valid) {
 #pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4*>(po + 32 * c + e) =
-                make_float4(__uint_as_float(o[c][e]) * inv, __uint_as_float(o[c][e + 1]) * inv,
-                            __uint_as_float(o[c][e + 2]) * inv, __uint_as_float(o[c][e + 3]) * inv);
+        for (int e = 0; e < 32; e += 8) {
+          uint4 v;
+          v.x = pack_bf16(__uint_as_float(o[c][e]) * inv, __uint_as_float(o[c][e + 1]) * inv);
+          v.y = pack_bf16(__uint_as_float(o[c][e + 2]) * inv, __uint_as_float(o[c][e + 3]) * inv);
+          v.z = pack_bf16(__uint_as_float(o[c][e + 4]) * inv, __uint_as_float(o[c][e + 5]) * inv);
+          v.w = pack_bf16(__uint_as_float(o[c][e + 6]) * inv, __uint_as_float(o[c][e + 7]) * inv);
+          *reinterpret_cast<uint4*>(stage_w + lane * (D * 2) + swz((32 * c + e) / 8, lane) * 16) = v;
         }
       }
-      if (row_valid) p.part_lse[prow] = l > 0.f ? m_ref * sl2 + log2f(l) : -INFINITY;
-    } else if (ok) {
-      const float inv = l > 0.f ? (FP8 ? __ldg(p.v_scale + g) : 1.f) / l : 0.f;
-      __nv_bfloat16* orow = p.out + ((int64_t)(tok0 + qi) * p.q_heads + head) * D;
-      uint32_t o[D / 32][32];
-      load_o(o);
+      __syncwarp();
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        if (row_valid) {
-#pragma unroll
-          for (int e = 0; e < 32; e += 8) {
-            uint4 v;
-            v.x = pack_bf16(__uint_as_float(o[c][e]) * inv, __uint_as_float(o[c][e + 1]) * inv);
-            v.y = pack_bf16(__uint_as_float(o[c][e + 2]) * inv, __uint_as_float(o[c][e + 3]) * inv);
-            v.z = pack_bf16(__uint_as_float(o[c][e + 4]) * inv, __uint_as_float(o[c][e + 5]) * inv);
-            v.w = pack_bf16(__uint_as_float(o[c][e + 6]) * inv, __uint_as_float(o[c][e + 7]) * inv);
-            *reinterpret_cast<uint4*>(orow + 32 * c + e) = v;
-          }
-        }
+      for (int k = 0; k < 32; k += RPI) {
+        const int lr = k + lane / CH, c = lane % CH;
+        const int rr = quad * 32 + lr;
+        const int qi_r = q0 + t * p.qpt + rr / p.group;
+        if (qi_r < q_len)
+          *reinterpret_cast<uint4*>(p.out + ((int64_t)(tok0 + qi_r) * p.q_heads + g * p.group +
+                                             rr % p.group) * D + 8 * c) =
+              *reinterpret_cast<const uint4*>(stage_w + lr * (D * 2) + swz(c, lr) * 16);
       }
       if (row_valid && p.lse)
         p.lse[(int64_t)(tok0 + qi) * p.q_heads + head] =

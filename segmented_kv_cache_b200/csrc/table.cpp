@@ -36,6 +36,11 @@ namespace {
 using segattn::align_up;
 using Row8 = std::array<int32_t, 8>;
 using Row4 = std::array<int32_t, 4>;
+// prefill piece: request, kv head, first query, first K tile | end K tile, partial
+// slot (-1: none), one-tile flag, end of the request's segments | first packed query
+// row, queries and keys of the request, segment holding the piece's first key
+constexpr int kWorkInts = 12;
+using Row12 = std::array<int32_t, kWorkInts>;
 
 bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 
@@ -102,7 +107,7 @@ struct PItem {
 };
 
 struct Pieces {
-  std::vector<Row8> work;       // two-tile pieces longest first, then single-tile ones
+  std::vector<Row12> work;      // two-tile pieces longest first, then single-tile ones
   std::vector<Row8> merge;      // split items that are not cascade items
   std::vector<int32_t> citem;   // per item: its index in `citems`, or -1
   int32_t slots = 0;            // partial-result slots
@@ -172,16 +177,42 @@ void plan_pieces(const std::vector<PItem>& items, int max_split, std::vector<Row
       const int32_t kt0 = (int32_t)((int64_t)it.tiles * j / p);
       const int32_t kt1 = (int32_t)((int64_t)it.tiles * (j + 1) / p);
       out.work.push_back({it.r, it.g, it.q0, kt0, kt1, slotted ? slot0 + j : -1,
-                          it.single ? 1 : 0, 0});
+                          it.single ? 1 : 0, 0, 0, 0, 0, 0});
       out.single += it.single ? 1 : 0;
     }
   }
   // two-tile pieces, then single-tile pieces (word 6), each longest first; stable
   // keeps (request, query tile, head, piece) order among equals
-  std::stable_sort(out.work.begin(), out.work.end(), [](const Row8& a, const Row8& b) {
+  std::stable_sort(out.work.begin(), out.work.end(), [](const Row12& a, const Row12& b) {
     if (a[6] != b[6]) return a[6] < b[6];
     return a[4] - a[3] > b[4] - b[3];
   });
+}
+
+// Fill the per-request words of each piece from the arrays the kernel would
+// otherwise read first (saves the dependent table loads at CTA start): end of
+// the request's segments, first packed query row, queries, keys, and the
+// segment that holds the piece's first key (the last segment whose logical
+// start is <= that key, as the device's segment walk finds it).
+void fill_request_words(std::vector<Row12>& work, const std::vector<int32_t>& q_off,
+                        const std::vector<int32_t>& k_len, const std::vector<Segs>& lists,
+                        const std::vector<int32_t>& seg_off) {
+  for (Row12& w : work) {
+    const int r = w[0];
+    const int64_t first_key = (int64_t)w[3] * segattn::kTileKeys;
+    int32_t seg = seg_off[r];
+    const int32_t seg_end = seg_off[r + 1];
+    int64_t kstart_next = seg < seg_end ? lists[r].len[0] : 0;  // logical start of seg + 1
+    for (size_t i = 0; seg + 1 < seg_end && kstart_next <= first_key; ++i) {
+      ++seg;
+      kstart_next += lists[r].len[i + 1];
+    }
+    w[7] = seg_end;
+    w[8] = q_off[r];
+    w[9] = q_off[r + 1] - q_off[r];
+    w[10] = k_len[r];
+    w[11] = seg;
+  }
 }
 
 // Cut the batch into groups of consecutive requests that share a prefix.
@@ -453,7 +484,7 @@ extern "C" int seg_attn_build_table(int batch, const int32_t* q_lens, const int3
   desc->off_seg_start = lay.take(nseg);
   desc->off_seg_kstart = lay.take(nseg);
   desc->off_seg_len = lay.take(nseg);
-  desc->off_work = lay.take((mode == SEG_ATTN_MODE_PREFILL ? 8 : 4) * (int64_t)n_work);
+  desc->off_work = lay.take((mode == SEG_ATTN_MODE_PREFILL ? kWorkInts : 4) * (int64_t)n_work);
   desc->off_req_chunks = lay.take(mode == SEG_ATTN_MODE_DECODE ? batch + 1 : 0);
   desc->off_merge = lay.take(8 * (int64_t)main_pieces.merge.size());
   const int ng = shared ? (int)gstart.size() - 1 : 0;
@@ -464,7 +495,7 @@ extern "C" int seg_attn_build_table(int batch, const int32_t* q_lens, const int3
   desc->off_group_seg_start = lay.take(ngseg);
   desc->off_group_seg_kstart = lay.take(ngseg);
   desc->off_group_seg_len = lay.take(ngseg);
-  desc->off_group_work = lay.take(8 * (int64_t)group_pieces.work.size());
+  desc->off_group_work = lay.take(kWorkInts * (int64_t)group_pieces.work.size());
   desc->off_citem = lay.take(4 * (int64_t)citems.size());
   desc->off_cascade = lay.take(8 * (int64_t)cascade.size());
 
@@ -538,7 +569,15 @@ extern "C" int seg_attn_build_table(int batch, const int32_t* q_lens, const int3
     for (size_t i = 0; i < rows.size(); ++i)
       memcpy(t + off + rows[i].size() * i, rows[i].data(), rows[i].size() * sizeof(int32_t));
   };
+  auto csr_offsets = [](const std::vector<Segs>& lists) {
+    std::vector<int32_t> off(lists.size() + 1, 0);
+    for (size_t r = 0; r < lists.size(); ++r) off[r + 1] = off[r] + (int32_t)lists[r].len.size();
+    return off;
+  };
   if (mode == SEG_ATTN_MODE_PREFILL) {
+    std::vector<int32_t> qo(batch + 1, 0);
+    for (int r = 0; r < batch; ++r) qo[r + 1] = qo[r] + ql[r];
+    fill_request_words(main_pieces.work, qo, okl, own, csr_offsets(own));
     put_rows(desc->off_work, main_pieces.work);
     put_rows(desc->off_merge, main_pieces.merge);
   } else {
@@ -551,6 +590,9 @@ extern "C" int seg_attn_build_table(int batch, const int32_t* q_lens, const int3
     for (int p = 0; p < ng; ++p) t[desc->off_group_k_lens + p] = (int32_t)gkeys[p];
     write_csr(gsegs, t + desc->off_group_seg_offsets, t + desc->off_group_seg_start,
               t + desc->off_group_seg_kstart, t + desc->off_group_seg_len);
+    std::vector<int32_t> gk(ng);
+    for (int p = 0; p < ng; ++p) gk[p] = (int32_t)gkeys[p];
+    fill_request_words(group_pieces.work, gq_off, gk, gsegs, csr_offsets(gsegs));
     put_rows(desc->off_group_work, group_pieces.work);
     put_rows(desc->off_citem, citems);
     put_rows(desc->off_cascade, cascade);

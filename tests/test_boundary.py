@@ -119,11 +119,34 @@ def test_prefill_table_contents():
     assert view(tab, d.off_seg_kstart, 5) == [0, 2, 0, 0, 20]
     assert view(tab, d.off_seg_len, 5) == [2, 5, 3, 20, 30]
     assert d.off_work % 4 == 0 and d.queries_per_tile == 32  # 128 rows / group 4
-    work = np.array(view(tab, d.off_work, 8 * d.num_work)).reshape(-1, 8)
+    work = np.array(view(tab, d.off_work, 12 * d.num_work)).reshape(-1, 12)
     # request 0: one pair x 2 kv heads; request 2: 40 queries -> 1 pair (64 per pair) x 2 heads
     assert len(work) == 4 and sorted(set(work[:, 0])) == [0, 2]
     # causal tile count: last query of request 2 sees all 50 keys -> tiles [0, 1), unsplit
     assert all(w[3] == 0 and w[4] == 1 and w[5] == -1 for w in work)
+    # request words of each row: end of its segments, first query row, queries, keys,
+    # segment of the first key
+    q_off, k_len, s_off = [0, 3, 3, 43], [7, 3, 50], [0, 2, 3, 5]
+    for w in work:
+        r = w[0]
+        assert list(w[7:12]) == [s_off[r + 1], q_off[r], q_off[r + 1] - q_off[r], k_len[r], s_off[r]]
+
+
+def test_prefill_first_segment_of_split_pieces():
+    # 4000 keys over segments with zero-length ones in between; the single item is cut
+    # into pieces along its 32 K tiles, each row names the segment of its first key as
+    # the device walk finds it: the last segment whose logical start is <= that key
+    lens = [0, 300, 0, 1200, 0, 0, 2500]
+    starts = [0, 10, 400, 500, 2000, 2000, 3000]
+    tab = build([1], [list(zip(starts, lens))], num_slots=6000, causal=False, hq=8, hkv=1)
+    d = tab.desc
+    work = np.array(view(tab, d.off_work, 12 * d.num_work)).reshape(-1, 12)
+    assert d.num_work > 1 and d.num_merge == 1  # split into several pieces
+    kstart = np.cumsum([0] + lens)[:-1]
+    for w in work:
+        j = w[3] * 128
+        want = max(i for i in range(len(lens)) if kstart[i] <= j)
+        assert w[11] == want and w[7] == len(lens) and list(w[8:11]) == [0, 1, 4000]
 
 
 def test_decode_chunks_cover_each_request():
@@ -182,7 +205,7 @@ def test_prefill_split_plan_covers_every_item_once():
     tab = build([64], [[(0, 20000)]], num_slots=20000, hq=16, hkv=2)
     d = tab.desc
     assert d.num_merge > 0 and d.num_parts > d.num_merge and d.workspace_bytes > 0
-    work = np.array(view(tab, d.off_work, 8 * d.num_work)).reshape(-1, 8)
+    work = np.array(view(tab, d.off_work, 12 * d.num_work)).reshape(-1, 12)
     merge = np.array(view(tab, d.off_merge, 8 * d.num_merge)).reshape(-1, 8)
     seen_slots = set()
     for r, g, q0, slot0, parts, *_ in merge:
@@ -207,7 +230,7 @@ def test_prefill_without_split_needs_no_workspace():
     tab = build([40, 3], [[(20, 20), (60, 30)], [(0, 7)]], num_slots=100, hq=8, hkv=2)
     d = tab.desc
     assert d.num_merge == 0 and d.num_parts == 0 and d.workspace_bytes == 0
-    work = np.array(view(tab, d.off_work, 8 * d.num_work)).reshape(-1, 8)
+    work = np.array(view(tab, d.off_work, 12 * d.num_work)).reshape(-1, 12)
     assert (work[:, 5] == -1).all() and (work[:, 3] == 0).all()
 
 
@@ -216,7 +239,7 @@ def test_prefill_one_tile_kernel_only_for_all_single_tile_passes():
     # Requests of 10 and 7 queries: every item holds queries in its first tile only.
     tab = build([10, 7], [[(0, 300)], [(400, 200)]], num_slots=900, hq=16, hkv=2)
     d = tab.desc
-    work = np.array(view(tab, d.off_work, 8 * d.num_work)).reshape(-1, 8)
+    work = np.array(view(tab, d.off_work, 12 * d.num_work)).reshape(-1, 12)
     assert d.num_single == d.num_work == 4 and (work[:, 6] == 1).all()
     lens = work[:, 4] - work[:, 3]
     assert list(lens) == sorted(lens, reverse=True)
@@ -224,7 +247,7 @@ def test_prefill_one_tile_kernel_only_for_all_single_tile_passes():
     tab = build([40, 10, 7], [[(0, 300)], [(400, 200)], [(700, 100)]], num_slots=900, hq=16,
                 hkv=2)
     d = tab.desc
-    work = np.array(view(tab, d.off_work, 8 * d.num_work)).reshape(-1, 8)
+    work = np.array(view(tab, d.off_work, 12 * d.num_work)).reshape(-1, 12)
     assert d.num_single == 0 and (work[:, 6] == 0).all()
 
 

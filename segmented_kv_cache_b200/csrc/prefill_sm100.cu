@@ -73,10 +73,6 @@ constexpr uint64_t kWaitLimitNs = 1000000000ull;  // default limit of a bounded 
 std::atomic<int> g_stall_tile{-1};
 std::atomic<uint64_t> g_stall_wait_ns{kWaitLimitNs};
 constexpr float kRescaleLog2 = 8.0f;
-// Two tiles: a tile's softmax signals after this many 32-key chunks of its
-// current K tile that its next S may be computed; the chunks left take about
-// as long as that S takes to arrive.
-constexpr int kSoonChunks = 2;
 constexpr uint32_t kHalfBytes = 128 * 128;  // 128 rows x 64 bf16 (one swizzle-128B panel)
 constexpr uint32_t kPTile = 2 * kHalfBytes;   // P of one query tile: 128 rows x 128 keys
 
@@ -262,7 +258,6 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
   uint64_t* vst_empty = bars + 23;
   uint64_t* q_conv = bars + 24;     // queries ready: in TMEM (two tiles), converted (FP8)
   uint64_t* s_free = bars + 25;     // two tiles: the shared S buffer read by its softmax
-  uint64_t* s_soon = bars + 26;     // [2] two tiles: the tile's softmax is near the end of a K tile
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 28);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   // limit of every bounded wait, read only when a wait checks it
@@ -303,8 +298,6 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
     }
     mbar_init(mma_done, 1);
     mbar_init(s_free, 4);  // one arrival per softmax warp of the tile that read S
-    mbar_init(s_soon + 0, 128);
-    mbar_init(s_soon + 1, 128);
     mbar_init(q_conv, (SINGLE ? 1 : 2) * 128);
     if (FP8) {
       mbar_init(kst_full, 1);
@@ -354,6 +347,18 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
         bool contiguous;
       };
       auto tile_rows = [&](int i, TileRows& tr) {
+        // the usual case: all 128 keys inside the segment of the first one, i.e. 128
+        // consecutive pool slots -- one lookup, the same on every lane
+        {
+          const int j0 = (kt0 + i) * kTileKeys;
+          while (seg + 1 < seg_end && __ldg(p.tab.seg_kstart + seg + 1) <= j0) ++seg;
+          const int ks = __ldg(p.tab.seg_kstart + seg);
+          if (j0 + kTileKeys <= ks + __ldg(p.tab.seg_len + seg)) {
+            tr.slot0 = __ldg(p.tab.seg_start + seg) + (j0 - ks);
+            tr.contiguous = true;
+            return;
+          }
+        }
         int slot_first = 0;
         bool run = true;
 #pragma unroll
@@ -466,9 +471,16 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
     // The whole warp runs the issue loop on warp-uniform values; one elected lane
     // executes each tcgen05.mma / commit.
     if (n_tiles > 0) {
-      auto wait_all = [&](uint64_t* bar, uint32_t parity) {
-        return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, wait_limit, true));
+      // The issue loop is one warp sharing its sub-partition with two softmax warps,
+      // so every instruction on it adds latency to the period: a complete phase is
+      // taken on the first try (uniform across the warp, no vote), and several
+      // barriers get independent first tries whose latencies overlap; the bounded
+      // wait runs only when a phase is not complete yet.
+      auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
+        if (mbar_try_wait(smem_u32(bar), parity)) return true;
+        return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, wait_limit, true)) != 0;
       };
+      auto ready = [&](uint64_t* bar, uint32_t parity) { return mbar_try_wait(smem_u32(bar), parity); };
       const uint32_t idesc_qk =
           FP8 ? idesc_f16_f32(128, 128, false) : idesc_bf16_f32(128, 128, false);
       const uint32_t idesc_pv = FP8 ? idesc_f16_f32(128, D, true) : idesc_bf16_f32(128, D, true);
@@ -618,27 +630,23 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
           const int st1 = (i + 1) % RK;  // K stage of K tile i + 1
           const uint32_t ph1 = ((i + 1) / RK) & 1;
           if (more) {
-            // use 2i + 2 waits for completion 2i + 1 (tile 1 read S of K tile i), and
-            // for tile 0 to near the end of K tile i: S waiting in the shared buffer
-            // for a busy softmax would hold up the other tile
-            if (!(ok = wait_all(k_full + st1, ph1) &&
-                       wait_all(s_free, 1) &&
-                       wait_all(s_soon + 0, i & 1)))
+            // use 2i + 2 waits for completion 2i + 1 (tile 1 read S of K tile i)
+            if (!(ready(k_full + st1, ph1) & ready(s_free, 1)) &&
+                !(ok = wait_all(k_full + st1, ph1) && wait_all(s_free, 1)))
               break;
             tc_fence_after();
             issue_qk_t(0, st1);
             mma_commit_warp(s_full + 0);
           }
-          if (!(ok = wait_all(v_full + st, ph) &&
-                     wait_all(p_full + 0, i & 1)))
+          if (!(ready(v_full + st, ph) & ready(p_full + 0, i & 1)) &&
+              !(ok = wait_all(v_full + st, ph) && wait_all(p_full + 0, i & 1)))
             break;
           tc_fence_after();
           issue_pv_s(0, st, i > 0);
           mma_commit_warp(o_full + 0);
           if (more) {
             // use 2i + 3 waits for completion 2i + 2 (tile 0 read S of K tile i + 1)
-            if (!(ok = wait_all(s_free, 0) &&
-                       wait_all(s_soon + 1, i & 1)))
+            if (!(ok = wait_all(s_free, 0)))
               break;
             tc_fence_after();
             issue_qk_t(1, st1);
@@ -833,7 +841,6 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
           tmem_st16(tS + 16 * c, pk[c]);  // P over the first 64 columns of this S buffer
         } else {
           store_p(c);
-          if (c == kSoonChunks - 1) mbar_arrive(s_soon + t);
         }
       }
       if constexpr (QT) f2_unpack(ls, ls0, ls1);
@@ -874,7 +881,6 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
           if (i > 0 &&
               !__all_sync(0xffffffffu, mbar_wait(o_full + t, (i - 1) & 1, abort_flag, wait_limit)))
             return false;
-          mbar_arrive(s_soon + t);
         }
         mbar_arrive(p_full + sb);
         return true;

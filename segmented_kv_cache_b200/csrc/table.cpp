@@ -181,11 +181,21 @@ void plan_pieces(const std::vector<PItem>& items, int max_split, std::vector<Row
       out.single += it.single ? 1 : 0;
     }
   }
-  // two-tile pieces, then single-tile pieces (word 6), each longest first; stable
-  // keeps (request, query tile, head, piece) order among equals
-  std::stable_sort(out.work.begin(), out.work.end(), [](const Row12& a, const Row12& b) {
+  // Two-tile pieces, then single-tile pieces (word 6), each longest first in 16
+  // length classes of the longest piece's 1/16; inside a class the pieces that read
+  // the same keys (request, kv head, piece of the key range) are adjacent, ordered by
+  // query block, so the CTAs running at one time share their K/V tiles through L2
+  // instead of each streaming its own range from HBM.
+  int32_t max_len = 1;
+  for (const Row12& w : out.work) max_len = std::max(max_len, w[4] - w[3]);
+  auto cls = [&](const Row12& w) { return (int64_t)(w[4] - w[3]) * 16 / max_len; };
+  std::stable_sort(out.work.begin(), out.work.end(), [&](const Row12& a, const Row12& b) {
     if (a[6] != b[6]) return a[6] < b[6];
-    return a[4] - a[3] > b[4] - b[3];
+    if (cls(a) != cls(b)) return cls(a) > cls(b);
+    if (a[0] != b[0]) return a[0] < b[0];  // request
+    if (a[1] != b[1]) return a[1] < b[1];  // kv head
+    if (a[3] != b[3]) return a[3] < b[3];  // first K tile of the piece
+    return a[2] < b[2];                    // query block
   });
 }
 

@@ -28,8 +28,8 @@
 //                the max grows by more than 2^8 (the final O / l uses the same
 //                reference max, so the result is unchanged), epilogue O / l ->
 //                bf16 and lse.
-// Two query tiles over a bf16 cache (the usual item): the softmax threads copy
-// their query rows into tensor memory once, so
+// Two query tiles (the usual item): the softmax threads copy their query rows
+// into tensor memory once, so
 //                  S   = Q_t K^T   (TS: Q from TMEM, K from the ring)
 //                  O_t += P_t V    (SS: P from shared memory, V MN-major)
 // and the two tiles take turns on one S buffer.  A softmax thread loads its
@@ -38,11 +38,12 @@
 // this tile's softmax still runs, and no MMA writes tensor memory that the MMA
 // before it reads (such a write waits for the tensor pipe to drain).
 // TMEM columns: O0 [0,128) O1 [128,256) S [256,384) Q0 [384,448) Q1 [448,512).
-// One query tile, or two over an FP8 cache (whose code staging leaves no
-// shared memory for P): Q stays in shared memory (SS QK) and P is written over
-// S in TMEM (TS PV); one tile double-buffers S, two tiles have one S each and
-// issue PV_0, QK_0, PV_1, QK_1 so one tile's softmax overlaps the other's MMAs.
-// TMEM columns: O0 [0,128) (O1 [128,256)) S0/P0 [256,384) S1/P1 [384,512).
+// One query tile: Q stays in shared memory (SS QK) and P is written over S in
+// TMEM (TS PV), with S double-buffered.
+// TMEM columns: O [0,128) S0/P0 [256,384) S1/P1 [384,512).
+// Over an FP8 cache two more warps widen the E4M3 codes to f16: with two query
+// tiles in place, inside the ring slot whose second half the codes were loaded
+// into; with one, from staging tiles of their own.
 // Every mbarrier wait is bounded (1 s); a timeout stops all roles of the CTA,
 // drains in-flight copies and MMAs, frees TMEM and flags a device error.
 #include <cuda.h>
@@ -98,25 +99,38 @@ struct PrefillParams {
 // owns an SM and its 512 tensor-memory columns.
 // K/V ring depths (stages of K, of V).  Over a bf16 cache the one-tile kernel
 // spends the second query tile's space on a third K and V stage, and the
-// two-tile kernel, whose query tiles live in tensor memory, on a third K
+// two-tile kernels, whose query tiles live in tensor memory, on a third K
 // stage: its QK of a K tile runs a softmax ahead of the PV of the previous
-// one, so K tiles are wanted earlier than V tiles.  FP8 keeps two of each.
+// one, so K tiles are wanted earlier than V tiles.  The one-tile kernel over
+// an FP8 cache keeps two of each beside its code staging tiles.
 template <bool SINGLE, bool FP8>
 constexpr int ring_k() {
-  return FP8 ? 2 : 3;
+  return SINGLE && FP8 ? 2 : 3;
 }
 template <bool SINGLE, bool FP8>
 constexpr int ring_v() {
   return SINGLE && !FP8 ? 3 : 2;
 }
 
-// Two query tiles over a bf16 cache: queries in tensor memory, P in shared
-// memory, one S buffer the two tiles take turns on.  Every other variant (one
-// query tile; the FP8 cache, whose code staging leaves no shared memory for P)
-// keeps its queries in shared memory and writes P over S in tensor memory.
+// Two query tiles: queries in tensor memory, P in shared memory, one S buffer
+// the two tiles take turns on.  One query tile: queries in shared memory, P
+// written over S in tensor memory.
 template <bool SINGLE, bool FP8>
 constexpr bool queries_in_tmem() {
-  return !SINGLE && !FP8;
+  return !SINGLE;
+}
+
+// FP8 cache, two query tiles: a K/V tile's E4M3 codes land in the second half of
+// its ring slot and are widened to f16 there (no staging tiles, which leaves the
+// shared memory the tensor-memory query layout needs).  One query tile: codes
+// are staged in tiles of their own and widened into the ring.
+template <bool SINGLE, bool FP8>
+constexpr bool widen_in_place() {
+  return FP8 && !SINGLE;
+}
+template <int D, bool SINGLE, bool FP8>
+constexpr size_t staging_bytes() {
+  return FP8 && !widen_in_place<SINGLE, FP8>() ? 2 * (size_t)kTileKeys * D : 0;
 }
 
 template <int D, bool SINGLE, bool FP8>
@@ -125,13 +139,13 @@ constexpr size_t query_region_bytes() {
                                         : (SINGLE ? 1 : 2) * (D / 64) * (size_t)kHalfBytes;
 }
 
-// The FP8 variant adds one staging tile of raw codes each for K and V.
+// The one-tile FP8 variant adds one staging tile of raw codes each for K and V.
 template <int D, bool SINGLE, bool FP8>
 constexpr size_t prefill_smem_bytes() {
   constexpr size_t need = query_region_bytes<D, SINGLE, FP8>() +
                           (ring_k<SINGLE, FP8>() + ring_v<SINGLE, FP8>()) * (D / 64) *
                               (size_t)kHalfBytes +
-                          (FP8 ? 2 * kTileKeys * D : 0) + 256 + 1024;
+                          staging_bytes<D, SINGLE, FP8>() + 256 + 1024;
   static_assert(need <= 227 * 1024, "shared memory per CTA");
   return need < 120 * 1024 ? 120 * 1024 : need;
 }
@@ -212,6 +226,42 @@ __device__ __forceinline__ void widen_tile(const uint8_t* src, uint8_t* dst, int
   }
 }
 
+// In-place variant: the codes of one tile sit in the second half of the ring slot
+// (rows of D bytes) and are widened into the whole slot, in the layout above.  A
+// row's f16 output overwrites code bytes that other threads read, so every thread
+// first loads all of its codes, the 64 widening threads meet at named barrier 1,
+// and only then write.
+template <int D>
+__device__ __forceinline__ void widen_tile_in_place(uint8_t* slot, int ct) {
+  constexpr int kCols = D / 16;
+  constexpr int kRowStep = kConvThreads / kCols;
+  constexpr int kRows = kTileKeys / kRowStep;
+  static_assert(kRowStep % 8 == 0, "rows of one thread must share the swizzle phase");
+  const int j = ct % kCols, r0 = ct / kCols;
+  const uint8_t* s = slot + (D / 64) * kHalfBytes / 2 + r0 * D + 16 * j;
+  uint4 w[kRows];
+#pragma unroll
+  for (int k = 0; k < kRows; ++k) w[k] = *reinterpret_cast<const uint4*>(s + k * kRowStep * D);
+  ptx::named_barrier(1, kConvThreads);
+  const int sw = r0 & 7, c0 = (j & 3) * 2;
+  uint8_t* d = slot + (j >> 2) * kHalfBytes + r0 * 128;
+  const int o0 = (c0 ^ sw) << 4, o1 = ((c0 + 1) ^ sw) << 4;
+#pragma unroll
+  for (int k = 0; k < kRows; ++k) {
+    uint4 lo, hi;
+    lo.x = ptx::e4m3x2_to_f16x2(w[k].x);
+    lo.y = ptx::e4m3x2_to_f16x2(w[k].x >> 16);
+    lo.z = ptx::e4m3x2_to_f16x2(w[k].y);
+    lo.w = ptx::e4m3x2_to_f16x2(w[k].y >> 16);
+    hi.x = ptx::e4m3x2_to_f16x2(w[k].z);
+    hi.y = ptx::e4m3x2_to_f16x2(w[k].z >> 16);
+    hi.z = ptx::e4m3x2_to_f16x2(w[k].w);
+    hi.w = ptx::e4m3x2_to_f16x2(w[k].w >> 16);
+    *reinterpret_cast<uint4*>(d + k * kRowStep * 128 + o0) = lo;
+    *reinterpret_cast<uint4*>(d + k * kRowStep * 128 + o1) = hi;
+  }
+}
+
 // SINGLE: every item of the launch has queries in its first query tile only
 // (the planner lists those items last and launches them separately, so each
 // instantiation keeps its own register allocation).
@@ -240,9 +290,10 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
   uint8_t* sQ = sm;
   uint8_t* sK = sm + query_region_bytes<D, SINGLE, FP8>();
   uint8_t* sV = sK + RK * TILE;
-  uint8_t* sStK = sV + RV * TILE;           // FP8: raw code tile of K
-  uint8_t* sStV = sStK + kTileKeys * D;     // FP8: raw code tile of V
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + RV * TILE + (FP8 ? 2 * kTileKeys * D : 0));
+  constexpr bool INPLACE = widen_in_place<SINGLE, FP8>();
+  uint8_t* sStK = sV + RV * TILE;           // FP8, one tile: raw code tile of K
+  uint8_t* sStV = sStK + kTileKeys * D;     // FP8, one tile: raw code tile of V
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + RV * TILE + staging_bytes<D, SINGLE, FP8>());
   uint64_t* q_full = bars + 0;
   uint64_t* k_full = bars + 1;    // [RK]
   uint64_t* k_empty = bars + 4;   // [RK]
@@ -252,10 +303,12 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
   uint64_t* p_full = bars + 15;   // [2]
   uint64_t* o_full = bars + 17;   // [2]
   uint64_t* mma_done = bars + 19;
-  uint64_t* kst_full = bars + 20;   // FP8: code staging of K filled (TMA bytes)
-  uint64_t* kst_empty = bars + 21;  // FP8: code staging of K read by the converters
+  uint64_t* kst_full = bars + 20;   // FP8, one tile: code staging of K filled (TMA bytes)
+  uint64_t* kst_empty = bars + 21;  // FP8, one tile: code staging of K read by the converters
   uint64_t* vst_full = bars + 22;
   uint64_t* vst_empty = bars + 23;
+  uint64_t* code_k = bars + 20;     // FP8 in place: [RK] codes landed in a K ring slot
+  uint64_t* code_v = bars + 30;     // FP8 in place: [RV] the same for V
   uint64_t* q_conv = bars + 24;     // queries ready: in TMEM (two tiles), converted (FP8)
   uint64_t* s_free = bars + 25;     // two tiles: the shared S buffer read by its softmax
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 28);
@@ -299,7 +352,10 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
     mbar_init(mma_done, 1);
     mbar_init(s_free, 4);  // one arrival per softmax warp of the tile that read S
     mbar_init(q_conv, (SINGLE ? 1 : 2) * 128);
-    if (FP8) {
+    if (INPLACE) {
+      for (int s = 0; s < RK; ++s) mbar_init(code_k + s, 1);
+      for (int s = 0; s < RV; ++s) mbar_init(code_v + s, 1);
+    } else if (FP8) {
       mbar_init(kst_full, 1);
       mbar_init(kst_empty, kConvThreads);
       mbar_init(vst_full, 1);
@@ -409,7 +465,10 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
         if (!__all_sync(0xffffffffu, mbar_wait(k_empty + st, ((i / RK) & 1) ^ 1, abort_flag,
                                                wait_limit, true)))
           return false;
-        load_tile(tr, sK + st * TILE, &tm_k3, &tm_k, k_full + st);
+        if (INPLACE)  // codes into the slot's second half, widened there by warps 10-11
+          load_codes(tr, sK + st * TILE + TILE / 2, &tm_k3, &tm_k, code_k + st);
+        else
+          load_tile(tr, sK + st * TILE, &tm_k3, &tm_k, k_full + st);
         ++k_issued;
         return true;
       };
@@ -418,11 +477,14 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
         if (!__all_sync(0xffffffffu, mbar_wait(v_empty + st, ((i / RV) & 1) ^ 1, abort_flag,
                                                wait_limit, true)))
           return false;
-        load_tile(tr, sV + st * TILE, &tm_v3, &tm_v, v_full + st);
+        if (INPLACE)
+          load_codes(tr, sV + st * TILE + TILE / 2, &tm_v3, &tm_v, code_v + st);
+        else
+          load_tile(tr, sV + st * TILE, &tm_v3, &tm_v, v_full + st);
         ++v_issued;
         return true;
       };
-      if (FP8) {
+      if (FP8 && !INPLACE) {
         // codes of K tile i, then of V tile i, through one staging tile each
         for (int i = 0; i < n_tiles; ++i) {
           TileRows tr;
@@ -452,16 +514,17 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
           if (!(run = load_v(i, cur))) break;
           cur = nxt;
         }
-        // never leave the CTA with copies in flight
+        // never leave the CTA with copies in flight (the copies' own barriers: in
+        // place, the ring slots' full barriers wait for the widening threads too)
         for (int s = 0; s < RK; ++s)
           if (k_issued > s) {
             const int last = s + RK * ((k_issued - 1 - s) / RK);
-            mbar_wait(k_full + s, (last / RK) & 1, nullptr, wait_limit);
+            mbar_wait((INPLACE ? code_k : k_full) + s, (last / RK) & 1, nullptr, wait_limit);
           }
         for (int s = 0; s < RV; ++s)
           if (v_issued > s) {
             const int last = s + RV * ((v_issued - 1 - s) / RV);
-            mbar_wait(v_full + s, (last / RV) & 1, nullptr, wait_limit);
+            mbar_wait((INPLACE ? code_v : v_full) + s, (last / RV) & 1, nullptr, wait_limit);
           }
       }
       if (lane == 0) mbar_wait(q_full, 0, nullptr, wait_limit);
@@ -566,45 +629,6 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
             mma_commit_warp(k_empty + ks);
           }
         }
-      } else if (!QT) {
-        // Two tiles, P over S (FP8 cache): per K tile i the order is
-        //   PV_0(i), QK_0(i + 1), PV_1(i), QK_1(i + 1)
-        // so one tile's softmax overlaps the other tile's MMAs.
-        if (ok) {
-          tc_fence_after();
-          issue_qk(0, 0, 0);
-          mma_commit_warp(s_full + 0);
-          issue_qk(1, 1, 0);
-          mma_commit_warp(s_full + 1);
-          mma_commit_warp(k_empty + 0);
-        }
-        for (int i = 0; ok && i < n_tiles; ++i) {
-          const int st = i % RV;  // V stage of K tile i
-          const uint32_t ph = (i / RV) & 1;
-          const bool more = i + 1 < n_tiles;
-          const int st1 = (i + 1) % RK;  // K stage of K tile i + 1
-          const uint32_t ph1 = ((i + 1) / RK) & 1;
-          if (!(ok = wait_all(v_full + st, ph) && wait_all(p_full + 0, i & 1))) break;
-          tc_fence_after();
-          issue_pv(0, 0, st, i > 0);
-          mma_commit_warp(o_full + 0);
-          if (more) {
-            if (!(ok = wait_all(k_full + st1, ph1))) break;
-            tc_fence_after();
-            issue_qk(0, 0, st1);
-            mma_commit_warp(s_full + 0);
-          }
-          if (!(ok = wait_all(p_full + 1, i & 1))) break;
-          tc_fence_after();
-          issue_pv(1, 1, st, i > 0);
-          mma_commit_warp(o_full + 1);
-          mma_commit_warp(v_empty + st);
-          if (more) {
-            issue_qk(1, 1, st1);
-            mma_commit_warp(s_full + 1);
-            mma_commit_warp(k_empty + st1);
-          }
-        }
       } else {
         // Two tiles, one S buffer.  Use u of the buffer is QK of K tile u / 2 for
         // query tile u % 2; it may start once the softmax has read use u - 1
@@ -667,11 +691,33 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
     __syncwarp();
   } else if (FP8 && warp >= 10) {
     // ------------------------------------------------------------ FP8 code widening
-    // Staged E4M3 tile -> f16 K (V) ring slot, then make the generic-proxy
-    // writes visible to the tensor cores before signalling the ring slot full.
+    // E4M3 tile -> f16 K (V) ring slot, then make the generic-proxy writes
+    // visible to the tensor cores before signalling the ring slot full.
     const int ct = threadIdx.x - 10 * 32;
     bool ok = true;
-    for (int i = 0; ok && i < n_tiles; ++i) {
+    if (INPLACE) {
+      // codes in the slot's second half, in the producer's order: K tile 0, then
+      // K tile i + 1 before V tile i.  The 64 threads agree on every wait's outcome
+      // at a barrier (all or none go on), since the widening meets at another one.
+      auto widen = [&](uint8_t* slot, uint64_t* landed, uint32_t parity, uint64_t* full) -> bool {
+        const bool got = mbar_wait(landed, parity, abort_flag, wait_limit);
+        if (!named_barrier_and(1, kConvThreads, got)) return false;
+        widen_tile_in_place<D>(slot, ct);
+        fence_proxy_async_smem();
+        mbar_arrive(full);
+        return true;
+      };
+      if (n_tiles > 0) ok = widen(sK, code_k, 0, k_full);
+      for (int i = 0; ok && i < n_tiles; ++i) {
+        if (i + 1 < n_tiles) {
+          const int sk = (i + 1) % RK;
+          if (!(ok = widen(sK + sk * TILE, code_k + sk, ((i + 1) / RK) & 1, k_full + sk))) break;
+        }
+        const int sv = i % RV;
+        ok = widen(sV + sv * TILE, code_v + sv, (i / RV) & 1, v_full + sv);
+      }
+    }
+    for (int i = 0; !INPLACE && ok && i < n_tiles; ++i) {
       const int sk = i % RK, sv = i % RV;
       if (!(ok = mbar_wait(kst_full, i & 1, abort_flag, wait_limit) &&
                  mbar_wait(k_empty + sk, ((i / RK) & 1) ^ 1, abort_flag, wait_limit)))

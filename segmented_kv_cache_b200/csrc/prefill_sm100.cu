@@ -28,16 +28,17 @@
 //                the max grows by more than 2^8 (the final O / l uses the same
 //                reference max, so the result is unchanged), epilogue O / l ->
 //                bf16 and lse.
-// Two query tiles (the usual item): the softmax threads copy their query rows
-// into tensor memory once, so
-//                  S   = Q_t K^T   (TS: Q from TMEM, K from the ring)
-//                  O_t += P_t V    (SS: P from shared memory, V MN-major)
+// Two query tiles (the usual item):
+//                  S   = Q_t K^T   (SS: Q tile and K stage from shared memory)
+//                  O_t += P_t V    (TS: P from tensor memory, V MN-major)
 // and the two tiles take turns on one S buffer.  A softmax thread loads its
 // whole S row, releases the buffer (the other tile's QK can go), and writes P
-// to shared memory, so the next K tile's S of a query tile is computed while
-// this tile's softmax still runs, and no MMA writes tensor memory that the MMA
-// before it reads (such a write waits for the tensor pipe to drain).
-// TMEM columns: O0 [0,128) O1 [128,256) S [256,384) Q0 [384,448) Q1 [448,512).
+// into tensor-memory columns of its own, so the next K tile's S of a query
+// tile is computed while this tile's softmax still runs, and no MMA writes
+// tensor memory that an earlier MMA reads (such a write waits for the tensor
+// pipe to drain).  P stays out of shared memory, whose bandwidth the SS QK,
+// the V reads of PV and the TMA writes already share.
+// TMEM columns: O0 [0,128) O1 [128,256) S [256,384) P0 [384,448) P1 [448,512).
 // One query tile: Q stays in shared memory (SS QK) and P is written over S in
 // TMEM (TS PV), with S double-buffered.
 // TMEM columns: O [0,128) S0/P0 [256,384) S1/P1 [384,512).
@@ -75,7 +76,6 @@ std::atomic<int> g_stall_tile{-1};
 std::atomic<uint64_t> g_stall_wait_ns{kWaitLimitNs};
 constexpr float kRescaleLog2 = 8.0f;
 constexpr uint32_t kHalfBytes = 128 * 128;  // 128 rows x 64 bf16 (one swizzle-128B panel)
-constexpr uint32_t kPTile = 2 * kHalfBytes;   // P of one query tile: 128 rows x 128 keys
 
 struct PrefillParams {
   __nv_bfloat16* out;
@@ -98,11 +98,11 @@ struct PrefillParams {
 // variant asks for more than half the SM's shared memory as well, so one CTA
 // owns an SM and its 512 tensor-memory columns.
 // K/V ring depths (stages of K, of V).  Over a bf16 cache the one-tile kernel
-// spends the second query tile's space on a third K and V stage, and the
-// two-tile kernels, whose query tiles live in tensor memory, on a third K
-// stage: its QK of a K tile runs a softmax ahead of the PV of the previous
-// one, so K tiles are wanted earlier than V tiles.  The one-tile kernel over
-// an FP8 cache keeps two of each beside its code staging tiles.
+// spends the second query tile's space on a third K and V stage; the two-tile
+// kernels, whose P tiles live in tensor memory, have room for a third K stage:
+// their QK of a K tile runs a softmax ahead of the PV of the previous one, so K
+// tiles are wanted earlier than V tiles.  The one-tile kernel over an FP8 cache
+// keeps two of each beside its code staging tiles.
 template <bool SINGLE, bool FP8>
 constexpr int ring_k() {
   return SINGLE && FP8 ? 2 : 3;
@@ -112,11 +112,12 @@ constexpr int ring_v() {
   return SINGLE && !FP8 ? 3 : 2;
 }
 
-// Two query tiles: queries in tensor memory, P in shared memory, one S buffer
-// the two tiles take turns on.  One query tile: queries in shared memory, P
-// written over S in tensor memory.
+// Two query tiles: P in tensor memory columns of its own (so no MMA ever writes
+// tensor memory that an earlier MMA reads), one S buffer the two tiles take
+// turns on.  One query tile: P written over S, S double-buffered.  Queries stay
+// in shared memory as the TMA loaded them in both.
 template <bool SINGLE, bool FP8>
-constexpr bool queries_in_tmem() {
+constexpr bool two_tiles() {
   return !SINGLE;
 }
 
@@ -135,8 +136,7 @@ constexpr size_t staging_bytes() {
 
 template <int D, bool SINGLE, bool FP8>
 constexpr size_t query_region_bytes() {
-  return queries_in_tmem<SINGLE, FP8>() ? 2 * (size_t)kPTile
-                                        : (SINGLE ? 1 : 2) * (D / 64) * (size_t)kHalfBytes;
+  return (SINGLE ? 1 : 2) * (D / 64) * (size_t)kHalfBytes;
 }
 
 // The one-tile FP8 variant adds one staging tile of raw codes each for K and V.
@@ -283,10 +283,10 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
   constexpr int RK = ring_k<SINGLE, FP8>(), RV = ring_v<SINGLE, FP8>();
-  // Q tiles at sQ + t * TILE; with queries in tensor memory, P_t at sQ + t * kPTile,
-  // which holds Q tile t until its softmax threads have copied it there.
-  constexpr bool QT = queries_in_tmem<SINGLE, FP8>();
-  constexpr uint32_t QSTRIDE = QT ? kPTile : TILE;
+  // Q tiles at sQ + t * TILE.  Two query tiles (QT): P_t in tensor memory columns
+  // [384 + 64 t, 448 + 64 t).
+  constexpr bool QT = two_tiles<SINGLE, FP8>();
+  constexpr uint32_t QSTRIDE = TILE;
   uint8_t* sQ = sm;
   uint8_t* sK = sm + query_region_bytes<D, SINGLE, FP8>();
   uint8_t* sV = sK + RK * TILE;
@@ -309,7 +309,7 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
   uint64_t* vst_empty = bars + 23;
   uint64_t* code_k = bars + 20;     // FP8 in place: [RK] codes landed in a K ring slot
   uint64_t* code_v = bars + 30;     // FP8 in place: [RV] the same for V
-  uint64_t* q_conv = bars + 24;     // queries ready: in TMEM (two tiles), converted (FP8)
+  uint64_t* q_conv = bars + 24;     // FP8: queries converted to f16 in place
   uint64_t* s_free = bars + 25;     // two tiles: the shared S buffer read by its softmax
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 28);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -548,7 +548,7 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
           FP8 ? idesc_f16_f32(128, 128, false) : idesc_bf16_f32(128, 128, false);
       const uint32_t idesc_pv = FP8 ? idesc_f16_f32(128, D, true) : idesc_bf16_f32(128, D, true);
       const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
-      const uint32_t tS0 = tmem + 256, tO0 = tmem, tQ0 = tmem + 384;
+      const uint32_t tS0 = tmem + 256, tO0 = tmem, tP0 = tmem + 384;
       // S buffer `sb` = Q tile `qt` . K stage `st`^T;  O tile `ot` += P (in S buffer `sb`) . V stage `st`
       // Shared-memory descriptors are built once: a ring stage or P tile moves the
       // start address (16-byte units, the low 14 bits) by a multiple of its size,
@@ -556,7 +556,7 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
       // issue loop measured ~1.8x slower MMA issue than the tensor core's rate.
       const uint64_t dq = sdesc_sw128(q_addr, 16, 1024), dk = sdesc_sw128(k_addr, 16, 1024);
       const uint64_t dv = sdesc_sw128(v_addr, kHalfBytes, 1024);
-      constexpr uint32_t kTileU = TILE >> 4, kPTileU = kPTile >> 4;
+      constexpr uint32_t kTileU = TILE >> 4;
       // K-step k of a K-major operand: panel k / 4, 32 bytes per step inside it
       auto kstep = [](int k) -> uint32_t { return ((k >> 2) * kHalfBytes + (k & 3) * 32) >> 4; };
       // S buffer `sb` = Q tile `qt` . K stage `st`^T;  O tile `ot` += P (in S buffer `sb`) . V stage `st`
@@ -574,24 +574,23 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
         for (int k = 0; k < kTileKeys / 16; ++k)
           mma_ts_warp(d, a + 8 * k, b0 + ((k * 2048) >> 4), idesc_pv, (acc || k > 0) ? 1u : 0u);
       };
-      // two tiles: S = Q tile `qt` (in TMEM) . K stage `st`^T into the shared S buffer;
-      // O tile `ot` += P tile `ot` (shared memory) . V stage `st`
+      // two tiles: S = Q tile `qt` . K stage `st`^T into the shared S buffer (SS);
+      // O tile `ot` += P tile `ot` (its own tensor-memory columns) . V stage `st` (TS)
       auto issue_qk_t = [&](int qt, int st) {
-        const uint64_t b0 = dk + st * kTileU;
-        const uint32_t a = tQ0 + 64 * qt;
+        const uint64_t a0 = dq + qt * kTileU, b0 = dk + st * kTileU;
 #pragma unroll
         for (int k = 0; k < KSTEPS; ++k)
-          mma_ts_warp(tS0, a + 8 * k, b0 + kstep(k), idesc_qk, k > 0 ? 1u : 0u);
+          mma_ss_warp(tS0, a0 + kstep(k), b0 + kstep(k), idesc_qk, k > 0 ? 1u : 0u);
       };
       auto issue_pv_s = [&](int ot, int st, bool acc) {
-        const uint64_t a0 = dq + ot * kPTileU, b0 = dv + st * kTileU;
-        const uint32_t d = tO0 + 128 * ot;
+        const uint64_t b0 = dv + st * kTileU;
+        const uint32_t d = tO0 + 128 * ot, a = tP0 + 64 * ot;
 #pragma unroll
         for (int k = 0; k < kTileKeys / 16; ++k)
-          mma_ss_warp(d, a0 + kstep(k), b0 + ((k * 2048) >> 4), idesc_pv, (acc || k > 0) ? 1u : 0u);
+          mma_ts_warp(d, a + 8 * k, b0 + ((k * 2048) >> 4), idesc_pv, (acc || k > 0) ? 1u : 0u);
       };
-      bool ok = wait_all((FP8 || QT) ? q_conv : q_full, 0) &&
-                wait_all(k_full + 0, 0);
+      // FP8: the softmax threads convert the query tiles to f16 in place first
+      bool ok = wait_all(FP8 ? q_conv : q_full, 0) && wait_all(k_full + 0, 0);
       if (single) {
         // one query tile, S double-buffered: K tile i uses S buffer i & 1.  While the
         // softmax works on buffer i & 1, S of tile i + 1 is already in the other one;
@@ -745,21 +744,21 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
     const int vis = p.causal ? min(k_len, k_len - q_len + qi + 1) : k_len;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     uint32_t tS = lane_base + 256 + 128 * t;  // S buffer of the current K tile (SINGLE)
-    if (QT) tS = lane_base + 256;             // queries in TMEM: the shared S buffer
+    if (QT) tS = lane_base + 256;             // two tiles: the shared S buffer
     const uint32_t tO = lane_base + 128 * t;
+    const uint32_t tP = lane_base + 384 + 64 * t;  // two tiles: this tile's P
     // FP8: scores are q . code * k_scale, so the K scale joins the softmax scale
     const float sl2 = FP8 ? p.scale_log2 * __ldg(p.k_scale + g) : p.scale_log2;
     float m_ref = -INFINITY;  // raw score units
     float l = 0.f;
     bool ok = true;
-    if (n_tiles > 0 && (FP8 || QT)) {
-      // This thread's query row of tile t (visiting chunk c ^ (row & 7), the
-      // place of the row's logical chunk c, spreads a warp's 32 rows over all
-      // shared-memory banks).  One tile: bf16 -> f16 in place (FP8 cache).  Two
-      // tiles: into this row's TMEM lane, 2 elements per column (f16 over an
-      // FP8 cache), the layout of a tensor-memory A operand.
+    if (n_tiles > 0 && FP8) {
+      // FP8 cache: this thread's query row of tile t, bf16 -> f16 in place (exact
+      // for |q| < 65504), so that both MMA operands are f16.  Visiting chunk
+      // c ^ (row & 7), the place of the row's logical chunk c, spreads a warp's
+      // 32 rows over all shared-memory banks.
       ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, abort_flag, wait_limit));
-      if (ok && !QT) {
+      if (ok) {
 #pragma unroll
         for (int h = 0; h < HALVES; ++h)
 #pragma unroll
@@ -771,26 +770,6 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
             *chunk = v;
           }
         fence_proxy_async_smem();
-        mbar_arrive(q_conv);
-      } else if (ok) {
-        const uint32_t tQ = lane_base + 384 + 64 * t;
-#pragma unroll
-        for (int h = 0; h < HALVES; ++h) {
-          uint32_t qv[32];
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            uint4 v = *reinterpret_cast<const uint4*>(sQ + t * QSTRIDE + h * kHalfBytes +
-                                                      row * 128 + ((c ^ (row & 7)) << 4));
-            if (FP8) bf16x8_to_f16x8(v);
-            qv[4 * c] = v.x;
-            qv[4 * c + 1] = v.y;
-            qv[4 * c + 2] = v.z;
-            qv[4 * c + 3] = v.w;
-          }
-          tmem_st32(tQ + 32 * h, qv);
-        }
-        tmem_wait_st();
-        tc_fence_before();
         mbar_arrive(q_conv);
       }
     }
@@ -844,18 +823,9 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
       float ls0 = 0.f, ls1 = 0.f;
       const uint64_t sl2x2 = f2_pack(sl2, sl2), nbase2 = f2_pack(-base, -base);
       uint32_t pk[4][16];
-      // queries in TMEM: P row into the K-major 128-byte-swizzled A-operand layout of
-      // P_t in shared memory (keys [64h, 64h + 64) in panel h, logical 16-byte
-      // chunk c at c ^ (row & 7)); 32 keys (4 chunks) per call
-      auto store_p = [&](int c) {
-        uint8_t* prow = sQ + t * kPTile + (c >> 1) * kHalfBytes + row * 128;
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          *reinterpret_cast<uint4*>(prow + (((4 * (c & 1) + j) ^ (row & 7)) << 4)) =
-              make_uint4(pk[c][4 * j], pk[c][4 * j + 1], pk[c][4 * j + 2], pk[c][4 * j + 3]);
-      };
-      // queries in TMEM: P(i) replaces P(i - 1) in shared memory once PV(i - 1) has read it
-      // (complete by now as a rule: it was issued when this tile's S was)
+      // two tiles: P(i) replaces P(i - 1) in this tile's tensor-memory columns once
+      // PV(i - 1) has read it (complete by now as a rule: it was issued when this
+      // tile's S was)
       bool waited = false;
       if (QT && i > 0) {
         if (!__all_sync(0xffffffffu,
@@ -883,11 +853,9 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
           }
           pk[c][e] = FP8 ? pack_f16x2(pa, pb) : pack_bf16(pa, pb);
         }
-        if (!QT) {
-          tmem_st16(tS + 16 * c, pk[c]);  // P over the first 64 columns of this S buffer
-        } else {
-          store_p(c);
-        }
+        // 32 keys as 16 columns of 2 (the tensor-memory A-operand layout): over the
+        // first 64 columns of this S buffer (one tile), or into P_t (two tiles)
+        tmem_st16((QT ? tP : tS) + 16 * c, pk[c]);
       }
       if constexpr (QT) f2_unpack(ls, ls0, ls1);
       l = l * alpha + (ls0 + ls1);
@@ -907,7 +875,6 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
           tmem_st32(tO + 32 * c, o);
         }
       }
-      if (QT) fence_proxy_async_smem();
       return true;
     };
     // A warp whose 32 rows hold no query (past the end of the chunk) only keeps

@@ -39,9 +39,9 @@
 // pipe to drain).  P stays out of shared memory, whose bandwidth the SS QK,
 // the V reads of PV and the TMA writes already share.
 // TMEM columns: O0 [0,128) O1 [128,256) S [256,384) P0 [384,448) P1 [448,512).
-// One query tile: Q stays in shared memory (SS QK) and P is written over S in
-// TMEM (TS PV), with S double-buffered.
-// TMEM columns: O [0,128) S0/P0 [256,384) S1/P1 [384,512).
+// One query tile: S double-buffered, each buffer with a P region of its own, so
+// the QK that refills an S buffer never overwrites what the PV before it reads.
+// TMEM columns: O [0,128) P0 [128,192) P1 [192,256) S0 [256,384) S1 [384,512).
 // Over an FP8 cache two more warps widen the E4M3 codes to f16: with two query
 // tiles in place, inside the ring slot whose second half the codes were loaded
 // into; with one, from staging tiles of their own.
@@ -114,8 +114,8 @@ constexpr int ring_v() {
 
 // Two query tiles: P in tensor memory columns of its own (so no MMA ever writes
 // tensor memory that an earlier MMA reads), one S buffer the two tiles take
-// turns on.  One query tile: P written over S, S double-buffered.  Queries stay
-// in shared memory as the TMA loaded them in both.
+// turns on.  One query tile: S double-buffered, a P region per S buffer.  Queries
+// stay in shared memory as the TMA loaded them in both.
 template <bool SINGLE, bool FP8>
 constexpr bool two_tiles() {
   return !SINGLE;
@@ -567,9 +567,10 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
         for (int k = 0; k < KSTEPS; ++k)
           mma_ss_warp(d, a0 + kstep(k), b0 + kstep(k), idesc_qk, k > 0 ? 1u : 0u);
       };
+      // one tile: O += P (region `sb`, columns [128 + 64 sb, 192 + 64 sb)) . V stage `st`
       auto issue_pv = [&](int ot, int sb, int st, bool acc) {
         const uint64_t b0 = dv + st * kTileU;
-        const uint32_t d = tO0 + 128 * ot, a = tS0 + 128 * sb;
+        const uint32_t d = tO0 + 128 * ot, a = tmem + 128 + 64 * sb;
 #pragma unroll
         for (int k = 0; k < kTileKeys / 16; ++k)
           mma_ts_warp(d, a + 8 * k, b0 + ((k * 2048) >> 4), idesc_pv, (acc || k > 0) ? 1u : 0u);
@@ -592,10 +593,12 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
       // FP8: the softmax threads convert the query tiles to f16 in place first
       bool ok = wait_all(FP8 ? q_conv : q_full, 0) && wait_all(k_full + 0, 0);
       if (single) {
-        // one query tile, S double-buffered: K tile i uses S buffer i & 1.  While the
-        // softmax works on buffer i & 1, S of tile i + 1 is already in the other one;
-        // right after PV(i) has read P(i), S of tile i + 2 goes into the freed buffer
-        // (tensor-core operations of one CTA run in issue order).
+        // one query tile, S double-buffered: K tile i uses S buffer and P region i & 1.
+        // While the softmax works on buffer i & 1, S of tile i + 1 is already in the
+        // other one; right after PV(i), S of tile i + 2 goes into buffer i & 1 (the PV
+        // reads P region i & 1, not the S columns).  Tensor-core operations of one CTA
+        // run in issue order, so S of tile i + 2 being complete also means PV(i) is, and
+        // the softmax may then overwrite P region i & 1.
         if (ok) {
           tc_fence_after();
           issue_qk(0, 0, 0);
@@ -746,7 +749,9 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
     uint32_t tS = lane_base + 256 + 128 * t;  // S buffer of the current K tile (SINGLE)
     if (QT) tS = lane_base + 256;             // two tiles: the shared S buffer
     const uint32_t tO = lane_base + 128 * t;
-    const uint32_t tP = lane_base + 384 + 64 * t;  // two tiles: this tile's P
+    // P of the current K tile: two tiles, this tile's region; one tile, the region of
+    // the current S buffer (set per K tile)
+    uint32_t tP = lane_base + 384 + 64 * t;
     // FP8: scores are q . code * k_scale, so the K scale joins the softmax scale
     const float sl2 = FP8 ? p.scale_log2 * __ldg(p.k_scale + g) : p.scale_log2;
     float m_ref = -INFINITY;  // raw score units
@@ -853,9 +858,8 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
           }
           pk[c][e] = FP8 ? pack_f16x2(pa, pb) : pack_bf16(pa, pb);
         }
-        // 32 keys as 16 columns of 2 (the tensor-memory A-operand layout): over the
-        // first 64 columns of this S buffer (one tile), or into P_t (two tiles)
-        tmem_st16((QT ? tP : tS) + 16 * c, pk[c]);
+        // 32 keys as 16 columns of 2 (the tensor-memory A-operand layout)
+        tmem_st16(tP + 16 * c, pk[c]);
       }
       if constexpr (QT) f2_unpack(ls, ls0, ls1);
       l = l * alpha + (ls0 + ls1);
@@ -882,7 +886,10 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
     const bool warp_live = __any_sync(0xffffffffu, row_valid);
     // one K tile of softmax on S buffer sb (phase sph of its barriers)
     auto run_tile = [&](int i, int sb, uint32_t sph) -> bool {
-      if (single) tS = lane_base + 256 + 128 * sb;
+      if (single) {
+        tS = lane_base + 256 + 128 * sb;
+        tP = lane_base + 128 + 64 * sb;
+      }
       if (!__all_sync(0xffffffffu, mbar_wait(s_full + sb, sph, abort_flag, wait_limit, true)))
         return false;
       if (!warp_live) {

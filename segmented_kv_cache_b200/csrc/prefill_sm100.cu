@@ -55,6 +55,7 @@
 
 #include <atomic>
 #include <mutex>
+#include <type_traits>
 
 #include "ptx_sm100.cuh"
 #include "seg_attn_internal.h"
@@ -270,11 +271,12 @@ __device__ __forceinline__ void widen_tile_in_place(uint8_t* slot, int ct) {
 // and 11 into the K/V rings; queries are converted bf16 -> f16 in shared memory
 // and P is f16, so every product is f16 x f16 -> f32.  The K scale is folded
 // into the softmax scale, the V scale into the output.
-template <int D, bool SINGLE, bool FP8>
+template <int D, bool SINGLE, bool FP8, bool TMA_OUT>
 __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_k3,
-                   const __grid_constant__ CUtensorMap tm_v3, const PrefillParams p) {
+                   const __grid_constant__ CUtensorMap tm_v3, const __grid_constant__ CUtensorMap tm_o,
+                   const PrefillParams p) {
   using namespace ptx;
   constexpr int HALVES = D / 64;
   constexpr uint32_t TILE = HALVES * kHalfBytes;
@@ -371,6 +373,7 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
     prefetch_tensormap(&tm_v);
     prefetch_tensormap(&tm_k3);
     prefetch_tensormap(&tm_v3);
+    prefetch_tensormap(&tm_o);
   }
   if (warp == 1) tmem_alloc(tmem_slot, 512);
   tc_fence_before();
@@ -948,12 +951,13 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
     if (ok && n_tiles > 0)
       ok = __all_sync(0xffffffffu,
                       mbar_wait(o_full + t, (n_tiles - 1) & 1, abort_flag, wait_limit));
-    // Results leave through shared memory so that a warp stores whole rows: a thread
+    // Results leave through shared memory so that whole rows are stored: a thread
     // owns one row, and its own 16-byte pieces of it would put every warp store on 32
-    // different lines.  Each warp stages its 32 rows in a quarter of the tile's query
-    // / P region (free: the commit of the tile's last PV covers every earlier MMA),
-    // 16-byte chunk c of row-local r at ((c & ~7) | ((c ^ r) & 7)), then copies rows
-    // out with consecutive lanes on consecutive chunks.
+    // different lines.  The tile's query region is free (the commit of the tile's
+    // last PV covers every earlier MMA).  Partials of a split piece: each warp stages
+    // its 32 rows in a quarter of it, 16-byte chunk c of row-local r at
+    // ((c & ~7) | ((c ^ r) & 7)), and copies rows out with consecutive lanes on
+    // consecutive chunks.
     uint8_t* stage_w = sQ + t * QSTRIDE + quad * (QSTRIDE / 4);
     auto swz = [](int c, int r) { return (c & ~7) | ((c ^ r) & 7); };
     if (ok && slot >= 0) {
@@ -990,7 +994,8 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
         __syncwarp();
       }
       if (row_valid) p.part_lse[prow0 + lane] = l > 0.f ? m_ref * sl2 + log2f(l) : -INFINITY;
-    } else if (ok) {
+    } else if (!TMA_OUT && ok) {
+      // a pass whose pieces mostly write partials: rows staged per warp, copied out
       constexpr int CH = D / 8;    // 16-byte chunks of a bf16 row
       constexpr int RPI = 32 / CH; // rows per warp instruction of the copy
       const float inv = l > 0.f ? (FP8 ? __ldg(p.v_scale + g) : 1.f) / l : 0.f;
@@ -1022,6 +1027,67 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
       if (row_valid && p.lse)
         p.lse[(int64_t)(tok0 + qi) * p.q_heads + head] =
             l > 0.f ? (m_ref * sl2 + log2f(l)) * 0.69314718055994531f : -INFINITY;
+    }
+    if (TMA_OUT && slot < 0) {
+      // Final bf16 output, staged in the tile's query region in the layout of the
+      // queries' TMA box (64-column panels of 128-byte rows, chunk c of row r at
+      // c ^ (r & 7)).  A full query tile then leaves in two TMA stores issued by one
+      // thread (the rows of one tile are qpt consecutive tokens x G heads, the box of
+      // the output map); a tile with fewer queries than qpt is copied out a row per
+      // D / 8 lanes, since a box would reach into the next request's rows.  The
+      // tile's four warps agree at a barrier (an AND of their outcomes) before
+      // staging, so a give-up anywhere leaves no warp waiting at the second one.
+      constexpr int CH = D / 8;    // 16-byte chunks of a bf16 row
+      constexpr int RPI = 32 / CH; // rows per warp instruction of the copy
+      uint8_t* stage_t = sQ + t * QSTRIDE;
+      const bool full = q0 + (t + 1) * p.qpt <= q_len;
+      const bool go = full ? named_barrier_and(2 + t, 128, ok) : ok;
+      if (go) {
+        const float inv = l > 0.f ? (FP8 ? __ldg(p.v_scale + g) : 1.f) / l : 0.f;
+        uint32_t o[D / 32][32];
+        load_o(o);
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 8) {
+            uint4 v;
+            v.x = pack_bf16(__uint_as_float(o[c][e]) * inv, __uint_as_float(o[c][e + 1]) * inv);
+            v.y = pack_bf16(__uint_as_float(o[c][e + 2]) * inv, __uint_as_float(o[c][e + 3]) * inv);
+            v.z = pack_bf16(__uint_as_float(o[c][e + 4]) * inv, __uint_as_float(o[c][e + 5]) * inv);
+            v.w = pack_bf16(__uint_as_float(o[c][e + 6]) * inv, __uint_as_float(o[c][e + 7]) * inv);
+            const int ch = (32 * c + e) / 8;  // logical 16-byte chunk of the row
+            *reinterpret_cast<uint4*>(stage_t + (ch >> 3) * kHalfBytes + row * 128 +
+                                      (((ch & 7) ^ (row & 7)) << 4)) = v;
+          }
+        }
+        if (full) {
+          fence_proxy_async_smem();
+          named_barrier(2 + t, 128);
+          if (quad == 0 && lane == 0) {
+#pragma unroll
+            for (int h = 0; h < HALVES; ++h)
+              tma_store_3d(&tm_o, stage_t + h * kHalfBytes, 64 * h, g * p.group,
+                           tok0 + q0 + t * p.qpt);
+            bulk_commit_group();
+            bulk_wait_group_read0();  // the staging must be read before the CTA exits
+          }
+        } else {
+          __syncwarp();
+#pragma unroll
+          for (int k = 0; k < 32; k += RPI) {
+            const int rr = quad * 32 + k + lane / CH, c = lane % CH;
+            const int qi_r = q0 + t * p.qpt + rr / p.group;
+            if (qi_r < q_len)
+              *reinterpret_cast<uint4*>(p.out + ((int64_t)(tok0 + qi_r) * p.q_heads + g * p.group +
+                                                 rr % p.group) * D + 8 * c) =
+                  *reinterpret_cast<const uint4*>(stage_t + (c >> 3) * kHalfBytes + rr * 128 +
+                                                  (((c & 7) ^ (rr & 7)) << 4));
+          }
+        }
+        if (row_valid && p.lse)
+          p.lse[(int64_t)(tok0 + qi) * p.q_heads + head] =
+              l > 0.f ? (m_ref * sl2 + log2f(l)) * 0.69314718055994531f : -INFINITY;
+      }
     }
   }
 
@@ -1106,16 +1172,17 @@ bool encode(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, bool SINGLE, bool FP8>
+template <int D, bool SINGLE, bool FP8, bool TMA_OUT>
 int launch_items(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                 const CUtensorMap& tk3, const CUtensorMap& tv3, const PrefillParams& p, int n,
+                 const CUtensorMap& tk3, const CUtensorMap& tv3, const CUtensorMap& to,
+                 const PrefillParams& p, int n,
                  cudaStream_t stream) {
   constexpr size_t smem = prefill_smem_bytes<D, SINGLE, FP8>();
-  if (cudaFuncSetAttribute(prefill_kernel<D, SINGLE, FP8>,
+  if (cudaFuncSetAttribute(prefill_kernel<D, SINGLE, FP8, TMA_OUT>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return SEG_ATTN_ERR_CUDA;
-  prefill_kernel<D, SINGLE, FP8><<<n, FP8 ? kThreadsFp8 : kThreads, smem, stream>>>(tq, tk, tv, tk3,
-                                                                                  tv3, p);
+  prefill_kernel<D, SINGLE, FP8, TMA_OUT><<<n, FP8 ? kThreadsFp8 : kThreads, smem, stream>>>(tq, tk, tv, tk3,
+                                                                                  tv3, to, p);
   return cudaGetLastError() == cudaSuccess ? SEG_ATTN_OK : SEG_ATTN_ERR_CUDA;
 }
 
@@ -1123,12 +1190,15 @@ template <int D, bool FP8>
 int launch_prefill_d(const PrefillLaunch& a, cudaStream_t stream) {
   const seg_attn_table_desc& d = *a.desc;
   const int group = d.q_heads / d.kv_heads;
-  CUtensorMap tq, tk, tv, tk3, tv3;
+  CUtensorMap tq, tk, tv, tk3, tv3, to;
   {
     const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)d.q_heads, (cuuint64_t)d.total_q};
     const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)d.q_heads * D * 2};
     const cuuint32_t box[3] = {64, (cuuint32_t)group, (cuuint32_t)d.queries_per_tile};
     if (!encode(&tq, a.q, 3, dims, strides, box)) return SEG_ATTN_ERR_CUDA;
+    // the output has the queries' shape: full query tiles leave by TMA stores of the
+    // same boxes (a pass that only writes partials has no output: no store is issued)
+    if (!encode(&to, a.out ? a.out : a.q, 3, dims, strides, box)) return SEG_ATTN_ERR_CUDA;
   }
   {
     const int64_t rows = d.num_slots * d.kv_heads;
@@ -1168,16 +1238,25 @@ int launch_prefill_d(const PrefillLaunch& a, cudaStream_t stream) {
   p.v_scale = a.v_scale;
   p.wait_ns = g_stall_wait_ns.load();
   p.withhold_tile = g_stall_tile.load();
-  // two-tile items first, then the single-tile items listed at the end
+  // two-tile items first, then the single-tile items listed at the end.  A pass in
+  // which some piece writes final rows runs the instantiation whose epilogue stores
+  // full query tiles by TMA; a pass of partials only (every item split, or a pass
+  // over shared prefixes) keeps the leaner epilogue, which measured faster there.
   const int n_single = d.num_single, n_two = d.num_work - d.num_single;
+  const bool any_final = d.num_parts < d.num_work;
+  auto launch = [&](auto single_tag, auto tma_tag, int base, int n) {
+    p.work_base = base;
+    return launch_items<D, decltype(single_tag)::value, FP8, decltype(tma_tag)::value>(
+        tq, tk, tv, tk3, tv3, to, p, n, stream);
+  };
+  using T = std::true_type;
+  using F = std::false_type;
   if (n_two > 0) {
-    p.work_base = 0;
-    const int rc = launch_items<D, false, FP8>(tq, tk, tv, tk3, tv3, p, n_two, stream);
+    const int rc = any_final ? launch(F{}, T{}, 0, n_two) : launch(F{}, F{}, 0, n_two);
     if (rc != SEG_ATTN_OK) return rc;
   }
   if (n_single > 0) {
-    p.work_base = n_two;
-    const int rc = launch_items<D, true, FP8>(tq, tk, tv, tk3, tv3, p, n_single, stream);
+    const int rc = any_final ? launch(T{}, T{}, n_two, n_single) : launch(T{}, F{}, n_two, n_single);
     if (rc != SEG_ATTN_OK) return rc;
   }
   if (d.num_merge > 0) {

@@ -74,7 +74,7 @@ enum { SEG_ATTN_MODE_PREFILL = 0, SEG_ATTN_MODE_DECODE = 1 };
 #define SEG_ATTN_SHARE_PREFIX 0x100
 
 #define SEG_ATTN_TABLE_MAGIC 0x53454741u /* "SEGA" */
-#define SEG_ATTN_TABLE_VERSION 4u
+#define SEG_ATTN_TABLE_VERSION 5u
 
 /*
  * Description of a built segment table.  Filled by seg_attn_build_table; the
@@ -105,7 +105,7 @@ typedef struct seg_attn_table_desc {
   int64_t off_seg_kstart;  /* [num_segments] logical index of each segment's first key */
   int64_t off_seg_len;     /* [num_segments] */
   int64_t off_work;        /* work items, 16-byte aligned: decode [num_work][4],
-                              prefill [num_work][12] */
+                              prefill [num_work][16] */
   int64_t off_req_chunks;  /* decode: [batch+1] first chunk of each request */
   int64_t off_merge;       /* prefill: [num_merge][8] split items and their partial slots */
   uint64_t table_bytes;    /* size of the table buffer */
@@ -134,7 +134,7 @@ typedef struct seg_attn_table_desc {
   int64_t off_group_seg_start;  /* [num_group_segments] */
   int64_t off_group_seg_kstart; /* [num_group_segments] */
   int64_t off_group_seg_len;    /* [num_group_segments] */
-  int64_t off_group_work;       /* [num_group_work][12] */
+  int64_t off_group_work;       /* [num_group_work][16] */
   int64_t off_citem;            /* [num_citems][4] first slot, pieces, first query of the item */
   int64_t off_cascade;          /* [num_cascade][8] row, request, prefix item, row in group,
                                    suffix item, row in request */

@@ -324,8 +324,8 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
   // row also carries the request's first query row, queries, keys and the segment
   // of the piece's first key, so no dependent table load precedes the first copies.
   const int item = p.work_base + blockIdx.x;
-  const int4 w0 = p.tab.work[3 * item], w1 = p.tab.work[3 * item + 1];
-  const int4 w2 = p.tab.work[3 * item + 2];
+  const int4 w0 = p.tab.work[4 * item], w1 = p.tab.work[4 * item + 1];
+  const int4 w2 = p.tab.work[4 * item + 2], w3 = p.tab.work[4 * item + 3];
   const int g = w0.y, q0 = w0.z, kt0 = w0.w, slot = w1.y;
   const int n_tiles = w1.x - kt0;
   const int tok0 = w2.x, q_len = w2.y, k_len = w2.z;
@@ -385,6 +385,10 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
     // ------------------------------------------------------------ producer
     int k_issued = 0, v_issued = 0;
     if (n_tiles > 0) {
+      // bf16 cache: when the table gives the slot of a first K tile that lies inside
+      // one segment, that tile goes with the query tiles, ahead of any table lookup
+      // (a stage of the fresh ring is free)
+      const bool k0_early = !FP8 && w3.x >= 0 && p.withhold_tile != 0;
       if (lane == 0) {
         const int q_tiles = single ? 1 : 2;
         mbar_expect_tx(q_full, q_tiles * TILE);
@@ -392,6 +396,11 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
           for (int h = 0; h < HALVES; ++h)
             tma_load_3d(sQ + t * QSTRIDE + h * kHalfBytes, &tm_q, q_full, 64 * h, g * p.group,
                         tok0 + q0 + t * p.qpt);
+        if (k0_early) {
+          mbar_expect_tx(k_full, TILE);
+          for (int h = 0; h < HALVES; ++h)
+            tma_load_3d(sK + h * kHalfBytes, &tm_k3, k_full, 64 * h, g, w3.x);
+        }
       }
       int seg = w2.w;
       const int seg_end = w1.w;
@@ -508,7 +517,8 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
         // K tile i + 1 before V tile i: the MMA warp takes them in that order
         TileRows cur, nxt;
         tile_rows(0, cur);
-        bool run = load_k(0, cur);
+        if (k0_early) ++k_issued;
+        bool run = k0_early || load_k(0, cur);
         for (int i = 0; run && i < n_tiles; ++i) {
           if (i + 1 < n_tiles) {
             tile_rows(i + 1, nxt);

@@ -30,7 +30,7 @@ struct TableView {
   const int32_t* seg_start;   // [nseg]
   const int32_t* seg_kstart;  // [nseg]
   const int32_t* seg_len;     // [nseg]
-  const int4* work;           // decode [num_work]; prefill [num_work][3]
+  const int4* work;           // decode [num_work]; prefill [num_work][4]
   const int4* merge;          // prefill [num_merge][2]
   const int32_t* req_chunks;  // [B+1] (decode)
 };

@@ -38,9 +38,11 @@ using Row8 = std::array<int32_t, 8>;
 using Row4 = std::array<int32_t, 4>;
 // prefill piece: request, kv head, first query, first K tile | end K tile, partial
 // slot (-1: none), one-tile flag, end of the request's segments | first packed query
-// row, queries and keys of the request, segment holding the piece's first key
-constexpr int kWorkInts = 12;
-using Row12 = std::array<int32_t, kWorkInts>;
+// row, queries and keys of the request, segment holding the piece's first key | pool
+// slot of the piece's first key when its first K tile lies inside that segment (-1:
+// it does not), three zero words
+constexpr int kWorkInts = 16;
+using Row16 = std::array<int32_t, kWorkInts>;
 
 bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 
@@ -107,7 +109,7 @@ struct PItem {
 };
 
 struct Pieces {
-  std::vector<Row12> work;      // two-tile pieces longest first, then single-tile ones
+  std::vector<Row16> work;      // two-tile pieces longest first, then single-tile ones
   std::vector<Row8> merge;      // split items that are not cascade items
   std::vector<int32_t> citem;   // per item: its index in `citems`, or -1
   int32_t slots = 0;            // partial-result slots
@@ -177,7 +179,7 @@ void plan_pieces(const std::vector<PItem>& items, int max_split, std::vector<Row
       const int32_t kt0 = (int32_t)((int64_t)it.tiles * j / p);
       const int32_t kt1 = (int32_t)((int64_t)it.tiles * (j + 1) / p);
       out.work.push_back({it.r, it.g, it.q0, kt0, kt1, slotted ? slot0 + j : -1,
-                          it.single ? 1 : 0, 0, 0, 0, 0, 0});
+                          it.single ? 1 : 0, 0, 0, 0, 0, 0, -1, 0, 0, 0});
       out.single += it.single ? 1 : 0;
     }
   }
@@ -187,9 +189,9 @@ void plan_pieces(const std::vector<PItem>& items, int max_split, std::vector<Row
   // query block, so the CTAs running at one time share their K/V tiles through L2
   // instead of each streaming its own range from HBM.
   int32_t max_len = 1;
-  for (const Row12& w : out.work) max_len = std::max(max_len, w[4] - w[3]);
-  auto cls = [&](const Row12& w) { return (int64_t)(w[4] - w[3]) * 16 / max_len; };
-  std::stable_sort(out.work.begin(), out.work.end(), [&](const Row12& a, const Row12& b) {
+  for (const Row16& w : out.work) max_len = std::max(max_len, w[4] - w[3]);
+  auto cls = [&](const Row16& w) { return (int64_t)(w[4] - w[3]) * 16 / max_len; };
+  std::stable_sort(out.work.begin(), out.work.end(), [&](const Row16& a, const Row16& b) {
     if (a[6] != b[6]) return a[6] < b[6];
     if (cls(a) != cls(b)) return cls(a) > cls(b);
     if (a[0] != b[0]) return a[0] < b[0];  // request
@@ -204,10 +206,10 @@ void plan_pieces(const std::vector<PItem>& items, int max_split, std::vector<Row
 // the request's segments, first packed query row, queries, keys, and the
 // segment that holds the piece's first key (the last segment whose logical
 // start is <= that key, as the device's segment walk finds it).
-void fill_request_words(std::vector<Row12>& work, const std::vector<int32_t>& q_off,
+void fill_request_words(std::vector<Row16>& work, const std::vector<int32_t>& q_off,
                         const std::vector<int32_t>& k_len, const std::vector<Segs>& lists,
                         const std::vector<int32_t>& seg_off) {
-  for (Row12& w : work) {
+  for (Row16& w : work) {
     const int r = w[0];
     const int64_t first_key = (int64_t)w[3] * segattn::kTileKeys;
     int32_t seg = seg_off[r];
@@ -222,6 +224,15 @@ void fill_request_words(std::vector<Row12>& work, const std::vector<int32_t>& q_
     w[9] = q_off[r + 1] - q_off[r];
     w[10] = k_len[r];
     w[11] = seg;
+    // the first K tile in one segment: its slot (the producer loads it before
+    // anything else of the CTA is set up)
+    w[12] = -1;
+    if (seg < seg_end && w[4] > w[3]) {
+      const int32_t local = seg - seg_off[r];
+      const int64_t ks = kstart_next - lists[r].len[local];
+      if (first_key + segattn::kTileKeys <= kstart_next && first_key >= ks)
+        w[12] = (int32_t)(lists[r].start[local] + (first_key - ks));
+    }
   }
 }
 

@@ -119,7 +119,7 @@ def test_prefill_table_contents():
     assert view(tab, d.off_seg_kstart, 5) == [0, 2, 0, 0, 20]
     assert view(tab, d.off_seg_len, 5) == [2, 5, 3, 20, 30]
     assert d.off_work % 4 == 0 and d.queries_per_tile == 32  # 128 rows / group 4
-    work = np.array(view(tab, d.off_work, 12 * d.num_work)).reshape(-1, 12)
+    work = np.array(view(tab, d.off_work, 16 * d.num_work)).reshape(-1, 16)
     # request 0: one pair x 2 kv heads; request 2: 40 queries -> 1 pair (64 per pair) x 2 heads
     assert len(work) == 4 and sorted(set(work[:, 0])) == [0, 2]
     # causal tile count: last query of request 2 sees all 50 keys -> tiles [0, 1), unsplit
@@ -130,6 +130,9 @@ def test_prefill_table_contents():
     for w in work:
         r = w[0]
         assert list(w[7:12]) == [s_off[r + 1], q_off[r], q_off[r + 1] - q_off[r], k_len[r], s_off[r]]
+        # first K tile in one segment: its first slot; otherwise -1 (here every request's
+        # first tile spans more than one segment, or the request has no tile at all)
+        assert w[12] == -1 and list(w[13:16]) == [0, 0, 0]
 
 
 def test_prefill_first_segment_of_split_pieces():
@@ -140,13 +143,16 @@ def test_prefill_first_segment_of_split_pieces():
     starts = [0, 10, 400, 500, 2000, 2000, 3000]
     tab = build([1], [list(zip(starts, lens))], num_slots=6000, causal=False, hq=8, hkv=1)
     d = tab.desc
-    work = np.array(view(tab, d.off_work, 12 * d.num_work)).reshape(-1, 12)
+    work = np.array(view(tab, d.off_work, 16 * d.num_work)).reshape(-1, 16)
     assert d.num_work > 1 and d.num_merge == 1  # split into several pieces
     kstart = np.cumsum([0] + lens)[:-1]
     for w in work:
         j = w[3] * 128
         want = max(i for i in range(len(lens)) if kstart[i] <= j)
         assert w[11] == want and w[7] == len(lens) and list(w[8:11]) == [0, 1, 4000]
+        # the slot of the first key when the piece's first tile lies inside that segment
+        inside = j + 128 <= kstart[want] + lens[want]
+        assert w[12] == (starts[want] + j - kstart[want] if inside else -1)
 
 
 def test_decode_chunks_cover_each_request():
@@ -205,7 +211,7 @@ def test_prefill_split_plan_covers_every_item_once():
     tab = build([64], [[(0, 20000)]], num_slots=20000, hq=16, hkv=2)
     d = tab.desc
     assert d.num_merge > 0 and d.num_parts > d.num_merge and d.workspace_bytes > 0
-    work = np.array(view(tab, d.off_work, 12 * d.num_work)).reshape(-1, 12)
+    work = np.array(view(tab, d.off_work, 16 * d.num_work)).reshape(-1, 16)
     merge = np.array(view(tab, d.off_merge, 8 * d.num_merge)).reshape(-1, 8)
     seen_slots = set()
     for r, g, q0, slot0, parts, *_ in merge:
@@ -230,7 +236,7 @@ def test_prefill_without_split_needs_no_workspace():
     tab = build([40, 3], [[(20, 20), (60, 30)], [(0, 7)]], num_slots=100, hq=8, hkv=2)
     d = tab.desc
     assert d.num_merge == 0 and d.num_parts == 0 and d.workspace_bytes == 0
-    work = np.array(view(tab, d.off_work, 12 * d.num_work)).reshape(-1, 12)
+    work = np.array(view(tab, d.off_work, 16 * d.num_work)).reshape(-1, 16)
     assert (work[:, 5] == -1).all() and (work[:, 3] == 0).all()
 
 
@@ -239,7 +245,7 @@ def test_prefill_one_tile_kernel_only_for_all_single_tile_passes():
     # Requests of 10 and 7 queries: every item holds queries in its first tile only.
     tab = build([10, 7], [[(0, 300)], [(400, 200)]], num_slots=900, hq=16, hkv=2)
     d = tab.desc
-    work = np.array(view(tab, d.off_work, 12 * d.num_work)).reshape(-1, 12)
+    work = np.array(view(tab, d.off_work, 16 * d.num_work)).reshape(-1, 16)
     assert d.num_single == d.num_work == 4 and (work[:, 6] == 1).all()
     lens = work[:, 4] - work[:, 3]
     assert list(lens) == sorted(lens, reverse=True)
@@ -247,7 +253,7 @@ def test_prefill_one_tile_kernel_only_for_all_single_tile_passes():
     tab = build([40, 10, 7], [[(0, 300)], [(400, 200)], [(700, 100)]], num_slots=900, hq=16,
                 hkv=2)
     d = tab.desc
-    work = np.array(view(tab, d.off_work, 12 * d.num_work)).reshape(-1, 12)
+    work = np.array(view(tab, d.off_work, 16 * d.num_work)).reshape(-1, 16)
     assert d.num_single == 0 and (work[:, 6] == 0).all()
 
 

@@ -69,7 +69,7 @@ def test_decode_group_wider_than_one_item_and_split_prefix_pass():
     case = _group_case(40, 5000, 700, seed=1, decode=True)
     _, tab = _check(case, True, "decode 40 members")
     d = tab.desc
-    gw = tab.host[d.off_group_work: d.off_group_work + 12 * d.num_group_work].view(-1, 12)
+    gw = tab.host[d.off_group_work: d.off_group_work + 16 * d.num_group_work].view(-1, 16)
     assert set(gw[:, 2].tolist()) == {0, 32}           # two query blocks
     assert d.num_group_work > 2 * d.kv_heads            # pieces along the prefix
 

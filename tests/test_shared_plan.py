@@ -129,7 +129,7 @@ def check_plan(tab, reqs, q, decode, causal=True, hq=16, hkv=2):
     assert d.group_total_k == int(P.sum())
     # the prefix pass: every (group, query block, kv head) item covers its tiles once,
     # every piece writes a partial into its own slot
-    gw = arr(tab, d.off_group_work, d.num_group_work, 12)
+    gw = arr(tab, d.off_group_work, d.num_group_work, 16)
     cit = arr(tab, d.off_citem, d.num_citems, 4)
     used = set()
     for p in range(d.num_groups):
@@ -261,7 +261,7 @@ def test_shared_prefix_configs_share_every_group(cfg):
     plain = sa.SegTable.build(None if decode else b.q_lens, b.seg_starts, b.seg_lens, wl.num_slots,
                               True, mode & 0xff, wl.q_heads, wl.kv_heads, wl.head_dim)
     if not decode:
-        tiles = lambda t, off, n: int((arr(t, off, n, 12)[:, 4] - arr(t, off, n, 12)[:, 3]).sum())
+        tiles = lambda t, off, n: int((arr(t, off, n, 16)[:, 4] - arr(t, off, n, 16)[:, 3]).sum())
         shared_tiles = tiles(tab, d.off_work, d.num_work) + tiles(tab, d.off_group_work,
                                                                   d.num_group_work)
         assert shared_tiles < 0.8 * tiles(plain, plain.desc.off_work, plain.desc.num_work)

@@ -798,8 +798,7 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
       auto f = [](uint32_t bits) { return __uint_as_float(bits); };
       // the whole S row in registers: one round trip to tensor memory
       uint32_t sv[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, sv[c]);
+      tmem_ld128(tS, sv);
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_wait_ld(sv[c]);
       if (QT) {
@@ -871,9 +870,9 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
           }
           pk[c][e] = FP8 ? pack_f16x2(pa, pb) : pack_bf16(pa, pb);
         }
-        // 32 keys as 16 columns of 2 (the tensor-memory A-operand layout)
-        tmem_st16(tP + 16 * c, pk[c]);
       }
+      // 128 keys as 64 columns of 2 (the tensor-memory A-operand layout), one store
+      tmem_st64(tP, pk);
       if constexpr (QT) f2_unpack(ls, ls0, ls1);
       l = l * alpha + (ls0 + ls1);
       if (__any_sync(0xffffffffu, rescale)) {
@@ -941,8 +940,12 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
     auto load_o = [&](uint32_t (&o)[D / 32][32]) {
       if (n_tiles > 0) {
         tc_fence_after();
+        if constexpr (D == 128) {
+          tmem_ld128(tO, o);
+        } else {
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) tmem_ld32(tO + 32 * c, o[c]);
+          for (int c = 0; c < D / 32; ++c) tmem_ld32(tO + 32 * c, o[c]);
+        }
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) tmem_wait_ld(o[c]);
       } else {

@@ -318,6 +318,14 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
       : "r"(taddr));
 }
 
+// 128 consecutive 32-bit columns of this thread's lane in one load.
+__device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t (&v)[4][32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x128.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63, %64, %65, %66, %67, %68, %69, %70, %71, %72, %73, %74, %75, %76, %77, %78, %79, %80, %81, %82, %83, %84, %85, %86, %87, %88, %89, %90, %91, %92, %93, %94, %95, %96, %97, %98, %99, %100, %101, %102, %103, %104, %105, %106, %107, %108, %109, %110, %111, %112, %113, %114, %115, %116, %117, %118, %119, %120, %121, %122, %123, %124, %125, %126, %127}, [%128];"
+      : "=r"(v[0][0]), "=r"(v[0][1]), "=r"(v[0][2]), "=r"(v[0][3]), "=r"(v[0][4]), "=r"(v[0][5]), "=r"(v[0][6]), "=r"(v[0][7]), "=r"(v[0][8]), "=r"(v[0][9]), "=r"(v[0][10]), "=r"(v[0][11]), "=r"(v[0][12]), "=r"(v[0][13]), "=r"(v[0][14]), "=r"(v[0][15]), "=r"(v[0][16]), "=r"(v[0][17]), "=r"(v[0][18]), "=r"(v[0][19]), "=r"(v[0][20]), "=r"(v[0][21]), "=r"(v[0][22]), "=r"(v[0][23]), "=r"(v[0][24]), "=r"(v[0][25]), "=r"(v[0][26]), "=r"(v[0][27]), "=r"(v[0][28]), "=r"(v[0][29]), "=r"(v[0][30]), "=r"(v[0][31]), "=r"(v[1][0]), "=r"(v[1][1]), "=r"(v[1][2]), "=r"(v[1][3]), "=r"(v[1][4]), "=r"(v[1][5]), "=r"(v[1][6]), "=r"(v[1][7]), "=r"(v[1][8]), "=r"(v[1][9]), "=r"(v[1][10]), "=r"(v[1][11]), "=r"(v[1][12]), "=r"(v[1][13]), "=r"(v[1][14]), "=r"(v[1][15]), "=r"(v[1][16]), "=r"(v[1][17]), "=r"(v[1][18]), "=r"(v[1][19]), "=r"(v[1][20]), "=r"(v[1][21]), "=r"(v[1][22]), "=r"(v[1][23]), "=r"(v[1][24]), "=r"(v[1][25]), "=r"(v[1][26]), "=r"(v[1][27]), "=r"(v[1][28]), "=r"(v[1][29]), "=r"(v[1][30]), "=r"(v[1][31]), "=r"(v[2][0]), "=r"(v[2][1]), "=r"(v[2][2]), "=r"(v[2][3]), "=r"(v[2][4]), "=r"(v[2][5]), "=r"(v[2][6]), "=r"(v[2][7]), "=r"(v[2][8]), "=r"(v[2][9]), "=r"(v[2][10]), "=r"(v[2][11]), "=r"(v[2][12]), "=r"(v[2][13]), "=r"(v[2][14]), "=r"(v[2][15]), "=r"(v[2][16]), "=r"(v[2][17]), "=r"(v[2][18]), "=r"(v[2][19]), "=r"(v[2][20]), "=r"(v[2][21]), "=r"(v[2][22]), "=r"(v[2][23]), "=r"(v[2][24]), "=r"(v[2][25]), "=r"(v[2][26]), "=r"(v[2][27]), "=r"(v[2][28]), "=r"(v[2][29]), "=r"(v[2][30]), "=r"(v[2][31]), "=r"(v[3][0]), "=r"(v[3][1]), "=r"(v[3][2]), "=r"(v[3][3]), "=r"(v[3][4]), "=r"(v[3][5]), "=r"(v[3][6]), "=r"(v[3][7]), "=r"(v[3][8]), "=r"(v[3][9]), "=r"(v[3][10]), "=r"(v[3][11]), "=r"(v[3][12]), "=r"(v[3][13]), "=r"(v[3][14]), "=r"(v[3][15]), "=r"(v[3][16]), "=r"(v[3][17]), "=r"(v[3][18]), "=r"(v[3][19]), "=r"(v[3][20]), "=r"(v[3][21]), "=r"(v[3][22]), "=r"(v[3][23]), "=r"(v[3][24]), "=r"(v[3][25]), "=r"(v[3][26]), "=r"(v[3][27]), "=r"(v[3][28]), "=r"(v[3][29]), "=r"(v[3][30]), "=r"(v[3][31])
+      : "r"(taddr));
+}
+
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
@@ -328,6 +336,14 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32
       "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]),
       "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]),
       "r"(v[30]), "r"(v[31])
+      : "memory");
+}
+
+// 64 consecutive 32-bit columns of this thread's lane in one store.
+__device__ __forceinline__ void tmem_st64(uint32_t taddr, const uint32_t (&v)[4][16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x64.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63, %64};" ::"r"(taddr),
+      "r"(v[0][0]), "r"(v[0][1]), "r"(v[0][2]), "r"(v[0][3]), "r"(v[0][4]), "r"(v[0][5]), "r"(v[0][6]), "r"(v[0][7]), "r"(v[0][8]), "r"(v[0][9]), "r"(v[0][10]), "r"(v[0][11]), "r"(v[0][12]), "r"(v[0][13]), "r"(v[0][14]), "r"(v[0][15]), "r"(v[1][0]), "r"(v[1][1]), "r"(v[1][2]), "r"(v[1][3]), "r"(v[1][4]), "r"(v[1][5]), "r"(v[1][6]), "r"(v[1][7]), "r"(v[1][8]), "r"(v[1][9]), "r"(v[1][10]), "r"(v[1][11]), "r"(v[1][12]), "r"(v[1][13]), "r"(v[1][14]), "r"(v[1][15]), "r"(v[2][0]), "r"(v[2][1]), "r"(v[2][2]), "r"(v[2][3]), "r"(v[2][4]), "r"(v[2][5]), "r"(v[2][6]), "r"(v[2][7]), "r"(v[2][8]), "r"(v[2][9]), "r"(v[2][10]), "r"(v[2][11]), "r"(v[2][12]), "r"(v[2][13]), "r"(v[2][14]), "r"(v[2][15]), "r"(v[3][0]), "r"(v[3][1]), "r"(v[3][2]), "r"(v[3][3]), "r"(v[3][4]), "r"(v[3][5]), "r"(v[3][6]), "r"(v[3][7]), "r"(v[3][8]), "r"(v[3][9]), "r"(v[3][10]), "r"(v[3][11]), "r"(v[3][12]), "r"(v[3][13]), "r"(v[3][14]), "r"(v[3][15])
       : "memory");
 }
 

@@ -149,13 +149,16 @@ __global__ void __launch_bounds__(kThreads) la_chunk_state_kernel(
     const float w = t < len ? ex2(glast - gt) : 0.f;
     if (t == 0) p.gamma[unit] = ex2(glast);
     // K row t *= exp(G_last - G_t): the row's 16-byte pieces are permuted by the
-    // swizzle but stay inside the row, so scaling in place is layout-blind
+    // swizzle but stay inside the row, so scaling in place is layout-blind.  Thread
+    // t starts at piece t & 7, so the 8 rows of one shared-memory phase use 8
+    // different banks.
     bool ok = mbar_wait(&kv_full, 0, &abort_flag, kWaitNs);
     if (ok) {
       for (int hh = 0; hh < 2; ++hh) {
         uint4* row = reinterpret_cast<uint4*>(sK + hh * kHalf + t * 128);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
+        for (int e0 = 0; e0 < 8; ++e0) {
+          const int e = e0 ^ (t & 7);
           uint4 x = row[e];
           uint32_t* wd = reinterpret_cast<uint32_t*>(&x);
 #pragma unroll
@@ -174,19 +177,30 @@ __global__ void __launch_bounds__(kThreads) la_chunk_state_kernel(
     ok = ok && mbar_wait(&mma_done, 0, &abort_flag, kWaitNs);
     if (ok) {
       tc_fence_after();
-      // row t of U (key index i = t): 128 fp32 columns
-      float* dst = p.u + ((int64_t)unit * kDim + t) * kDim;
+      // Row t of U (key index i = t) is 128 fp32 columns = 32 pieces of 16 bytes.
+      // The K and V tiles are idle once the MMA is done: row t goes there at
+      // 512 * t, piece c at position (c & ~7) | ((c ^ t) & 7), and then each warp
+      // writes its own 32 rows out, one whole 512-byte row per store instruction.
+      uint4* stage = reinterpret_cast<uint4*>(sm);
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t a[32];
-        tmem_ld32(lane_base + 32 * cc, a);
-        tmem_wait_ld(a);
+      for (int half = 0; half < 2; ++half) {
+        uint32_t a[2][32];
+        tmem_ld64(lane_base + 64 * half, a);
+        tmem_wait_ld(a[0]);
+        tmem_wait_ld(a[1]);
 #pragma unroll
-        for (int e = 0; e < 32; e += 4)
-          *reinterpret_cast<float4*>(dst + 32 * cc + e) =
-              make_float4(__uint_as_float(a[e]), __uint_as_float(a[e + 1]),
-                          __uint_as_float(a[e + 2]), __uint_as_float(a[e + 3]));
+        for (int j = 0; j < 16; ++j) {
+          const int c = 16 * half + j;
+          const uint32_t* w4 = &a[j >> 3][4 * (j & 7)];
+          stage[32 * t + ((c & ~7) | ((c ^ t) & 7))] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        }
       }
+      __syncwarp();
+      const int r0 = t - lane;
+      uint4* dst = reinterpret_cast<uint4*>(p.u + ((int64_t)unit * kDim + r0) * kDim);
+#pragma unroll 4
+      for (int r = 0; r < 32; ++r)
+        dst[32 * r + lane] = stage[32 * (r0 + r) + ((lane & ~7) | ((lane ^ (r0 + r)) & 7))];
     }
   }
   tc_fence_before();
@@ -334,24 +348,27 @@ __global__ void __launch_bounds__(kThreads) la_chunk_out_kernel(
     bool ok = __all_sync(0xffffffffu, mbar_wait(&qk_done, 0, &abort_flag, kWaitNs));
     if (ok) {
       tc_fence_after();
-      // P[t][s] = S[t][s] * exp(G_t - G_s) for s <= t (rows past the chunk: 0)
+      // P[t][s] = S[t][s] * exp(G_t - G_s) for s <= t (rows past the chunk: 0):
+      // the whole S row in one load, the 64 packed bf16 pairs back in one store
+      uint32_t a[4][32], pk[4][16];
+      tmem_ld128(tS + (lane_base - tmem), a);
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) tmem_wait_ld(a[cc]);
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
-        uint32_t a[32];
-        tmem_ld32(tS + (lane_base - tmem) + 32 * cc, a);
-        tmem_wait_ld(a);
-        uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const int s0 = 32 * cc + 2 * e;
-          const float p0 = (row_valid && s0 <= t) ? __uint_as_float(a[2 * e]) * ex2(gt - g2[s0]) : 0.f;
-          const float p1 =
-              (row_valid && s0 + 1 <= t) ? __uint_as_float(a[2 * e + 1]) * ex2(gt - g2[s0 + 1]) : 0.f;
+          const float p0 =
+              (row_valid && s0 <= t) ? __uint_as_float(a[cc][2 * e]) * ex2(gt - g2[s0]) : 0.f;
+          const float p1 = (row_valid && s0 + 1 <= t)
+                               ? __uint_as_float(a[cc][2 * e + 1]) * ex2(gt - g2[s0 + 1])
+                               : 0.f;
           __nv_bfloat162 b = __floats2bfloat162_rn(p0, p1);
-          pk[e] = *reinterpret_cast<uint32_t*>(&b);
+          pk[cc][e] = *reinterpret_cast<uint32_t*>(&b);
         }
-        tmem_st16(tS + (lane_base - tmem) + 16 * cc, pk);
       }
+      tmem_st64(tS + (lane_base - tmem), pk);
       tmem_wait_st();
       tc_fence_before();
     }
@@ -360,30 +377,45 @@ __global__ void __launch_bounds__(kThreads) la_chunk_out_kernel(
     if (ok) {
       tc_fence_after();
       const float decay_t = ex2(gt);
-      __nv_bfloat16* orow = p.out + ((int64_t)(row0 + t) * p.heads + h) * kDim;
+      // Row t of out is 128 bf16 = 16 pieces of 16 bytes.  The Q tile is idle once
+      // every MMA is done: row t goes there at 256 * t, piece c at position
+      // (c & 8) | ((c ^ t) & 7), and each warp then writes its own 32 rows out, two
+      // whole 256-byte rows per store instruction (rows past the chunk stay unwritten).
+      uint4* stage = reinterpret_cast<uint4*>(sQ);
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t a[32], b[32];
-        tmem_ld32(tI + (lane_base - tmem) + 32 * cc, a);
-        tmem_ld32(tO + (lane_base - tmem) + 32 * cc, b);
-        tmem_wait_ld(a);
-        tmem_wait_ld(b);
-        if (row_valid) {
+      for (int half = 0; half < 2; ++half) {
+        uint32_t a[2][32], b[2][32];
+        tmem_ld64(tI + (lane_base - tmem) + 64 * half, a);
+        tmem_ld64(tO + (lane_base - tmem) + 64 * half, b);
+        tmem_wait_ld(a[0]);
+        tmem_wait_ld(a[1]);
+        tmem_wait_ld(b[0]);
+        tmem_wait_ld(b[1]);
 #pragma unroll
-          for (int e = 0; e < 32; e += 8) {
-            uint32_t wd[4];
+        for (int j = 0; j < 8; ++j) {  // piece c = 8 * half + j: columns 8c .. 8c + 7
+          uint32_t wd[4];
 #pragma unroll
-            for (int u2 = 0; u2 < 4; ++u2) {
-              const float o0 = p.scale * fmaf(decay_t, __uint_as_float(a[e + 2 * u2]),
-                                              __uint_as_float(b[e + 2 * u2]));
-              const float o1 = p.scale * fmaf(decay_t, __uint_as_float(a[e + 2 * u2 + 1]),
-                                              __uint_as_float(b[e + 2 * u2 + 1]));
-              __nv_bfloat162 v2 = __floats2bfloat162_rn(o0, o1);
-              wd[u2] = *reinterpret_cast<uint32_t*>(&v2);
-            }
-            *reinterpret_cast<uint4*>(orow + 32 * cc + e) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+          for (int u2 = 0; u2 < 4; ++u2) {
+            const int e = 8 * j + 2 * u2;
+            const float o0 = p.scale * fmaf(decay_t, __uint_as_float(a[e >> 5][e & 31]),
+                                            __uint_as_float(b[e >> 5][e & 31]));
+            const float o1 = p.scale * fmaf(decay_t, __uint_as_float(a[e >> 5][(e & 31) + 1]),
+                                            __uint_as_float(b[e >> 5][(e & 31) + 1]));
+            __nv_bfloat162 v2 = __floats2bfloat162_rn(o0, o1);
+            wd[u2] = *reinterpret_cast<uint32_t*>(&v2);
           }
+          const int c = 8 * half + j;
+          stage[16 * t + ((c & 8) | ((c ^ t) & 7))] = make_uint4(wd[0], wd[1], wd[2], wd[3]);
         }
+      }
+      __syncwarp();
+      const int r0 = t - lane, c = lane & 15;
+#pragma unroll 4
+      for (int r2 = 0; r2 < 16; ++r2) {
+        const int r = r0 + 2 * r2 + (lane >> 4);
+        if (r < len)
+          reinterpret_cast<uint4*>(p.out + ((int64_t)(row0 + r) * p.heads + h) * kDim)[c] =
+              stage[16 * r + ((c & 8) | ((c ^ r) & 7))];
       }
     }
   }

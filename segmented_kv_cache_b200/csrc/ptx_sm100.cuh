@@ -318,6 +318,14 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
       : "r"(taddr));
 }
 
+// 64 consecutive 32-bit columns of this thread's lane in one load.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&v)[2][32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%64];"
+      : "=r"(v[0][0]), "=r"(v[0][1]), "=r"(v[0][2]), "=r"(v[0][3]), "=r"(v[0][4]), "=r"(v[0][5]), "=r"(v[0][6]), "=r"(v[0][7]), "=r"(v[0][8]), "=r"(v[0][9]), "=r"(v[0][10]), "=r"(v[0][11]), "=r"(v[0][12]), "=r"(v[0][13]), "=r"(v[0][14]), "=r"(v[0][15]), "=r"(v[0][16]), "=r"(v[0][17]), "=r"(v[0][18]), "=r"(v[0][19]), "=r"(v[0][20]), "=r"(v[0][21]), "=r"(v[0][22]), "=r"(v[0][23]), "=r"(v[0][24]), "=r"(v[0][25]), "=r"(v[0][26]), "=r"(v[0][27]), "=r"(v[0][28]), "=r"(v[0][29]), "=r"(v[0][30]), "=r"(v[0][31]), "=r"(v[1][0]), "=r"(v[1][1]), "=r"(v[1][2]), "=r"(v[1][3]), "=r"(v[1][4]), "=r"(v[1][5]), "=r"(v[1][6]), "=r"(v[1][7]), "=r"(v[1][8]), "=r"(v[1][9]), "=r"(v[1][10]), "=r"(v[1][11]), "=r"(v[1][12]), "=r"(v[1][13]), "=r"(v[1][14]), "=r"(v[1][15]), "=r"(v[1][16]), "=r"(v[1][17]), "=r"(v[1][18]), "=r"(v[1][19]), "=r"(v[1][20]), "=r"(v[1][21]), "=r"(v[1][22]), "=r"(v[1][23]), "=r"(v[1][24]), "=r"(v[1][25]), "=r"(v[1][26]), "=r"(v[1][27]), "=r"(v[1][28]), "=r"(v[1][29]), "=r"(v[1][30]), "=r"(v[1][31])
+      : "r"(taddr));
+}
+
 // 128 consecutive 32-bit columns of this thread's lane in one load.
 __device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t (&v)[4][32]) {
   asm volatile(

@@ -574,7 +574,23 @@ def time_cold_calls(path, leg, steps, warmup, flush):
         path.run_leg(leg)
     e1.record(stream)
     torch.cuda.synchronize()
-    return statistics.mean(cold), statistics.median(cold), min(cold), e0.elapsed_time(e1) / steps
+    b2b = e0.elapsed_time(e1) / steps
+    # cold inside a stream of work: `steps` x (flush, call) between one event pair, less
+    # `steps` flushes alone.  An event pair around a lone call also holds the launch of
+    # the call, which the GPU front end only starts once the first event is written;
+    # in a stream of kernels that launch overlaps the work before it.
+    def loop(with_call):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            flush.zero_()
+            if with_call:
+                path.run_leg(leg)
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / steps
+    in_stream = statistics.median(loop(True) - loop(False) for _ in range(3))
+    return (statistics.mean(cold), statistics.median(cold), min(cold), b2b, in_stream)
 
 
 def run_sub_configs(args, device, peaks, peak_kind, with_oracle=True):
@@ -589,10 +605,12 @@ def run_sub_configs(args, device, peaks, peak_kind, with_oracle=True):
         path = Path(wl, device, args.kv_dtype, share=False)
         leg = path.legs[0]
         b = leg["batch"]
-        mean_ms, med_ms, min_ms, b2b_ms = time_cold_calls(path, leg, steps, warmup, flush)
+        mean_ms, med_ms, min_ms, b2b_ms, stream_ms = time_cold_calls(path, leg, steps, warmup,
+                                                                     flush)
         assert sa.seg_attn_take_device_error() == 0
         rec = {"workload": workload_name(wl), "mode": b.mode, "ms": mean_ms,
                "ms_median": med_ms, "ms_min": min_ms, "ms_back_to_back": b2b_ms,
+               "ms_cold_in_stream": stream_ms,
                "launches": leg["launches"], "steps": steps,
                "l2": "flushed before every timed call (256 MB write)"}
         if leg["mode"] == sa.MODE_PREFILL:
@@ -601,12 +619,16 @@ def run_sub_configs(args, device, peaks, peak_kind, with_oracle=True):
             rec.update({"flops": f, "tflops": tf, "frac_burst": tf / peaks["bf16_tflops"],
                         "frac_sustained": tf / peaks["bf16_tflops_sustained"],
                         "tflops_back_to_back": f / (b2b_ms * 1e-3) / 1e12,
+                        "tflops_cold_in_stream": f / (stream_ms * 1e-3) / 1e12,
+                        "frac_burst_cold_in_stream":
+                            f / (stream_ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
                         "peak_kind": f"{peak_kind} burst bf16"})
         else:
             kvb = 1 if args.kv_dtype == "fp8" else 2
             by = decode_bytes(b, wl, leg["tab"].desc.table_bytes, kvb)
             gbs = by / (mean_ms * 1e-3) / 1e9
             rec.update({"bytes": by, "gbs": gbs, "frac_hbm": gbs / peaks["hbm_gbs"],
+                        "gbs_cold_in_stream": by / (stream_ms * 1e-3) / 1e9,
                         "tflops": decode_flops(b, wl) / (mean_ms * 1e-3) / 1e12,
                         "peak_kind": f"{peak_kind} copy bandwidth"})
         if with_oracle:

@@ -270,6 +270,19 @@ int seg_attn_wait_selftest(int wait_us, void* stream);
 int seg_attn_stall_test(int withhold_k_tile, int wait_us);
 
 /*
+ * seg_attn_order_test -- diagnostic (no counterpart on the source pages): every
+ * softmax warp of later prefill launches sleeps about delay_ns nanoseconds
+ * right after it signals P of its item's last K tile, so the last P.V product
+ * has completed before the warp waits for it at the end of the item -- the
+ * order a slow warp meets there (an instruction-cache miss, a profiler's
+ * instrumentation).  Results must not change and no wait may give up.
+ *   delay_ns       0 .. 1000000; 0 is off (the default).
+ * Host-side setting read at each launch (process-wide, not thread-safe with
+ * concurrent prefill calls).  delay_ns out of range: SEG_ATTN_ERR_INVALID_ARG.
+ */
+int seg_attn_order_test(int delay_ns);
+
+/*
  * seg_attn_decode_noalloc -- seg_attn_decode for callers that cannot allocate
  * device memory (no counterpart on the source pages; this is a library
  * convenience).  Typical callers: a plugin inside another runtime that owns

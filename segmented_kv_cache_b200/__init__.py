@@ -21,7 +21,7 @@ from ._build import LIB as LIB_PATH
 __all__ = [
     "SegAttnError", "seg_attn_table_desc", "seg_attn_build_table", "seg_attn_workspace_size",
     "seg_attn_prefill", "seg_attn_decode", "seg_attn_status_string", "seg_attn_version",
-    "seg_attn_take_device_error", "seg_attn_wait_selftest", "seg_attn_stall_test", "SegTable", "load_library", "LIB_PATH",
+    "seg_attn_take_device_error", "seg_attn_wait_selftest", "seg_attn_stall_test", "seg_attn_order_test", "SegTable", "load_library", "LIB_PATH",
     "MODE_PREFILL", "MODE_DECODE", "STATUS", "SegPool", "seg_attn_kv_append",
     "seg_attn_decode_fp8", "seg_attn_prefill_fp8", "seg_attn_kv_append_fp8", "SHARE_PREFIX",
     "seg_la_table_desc", "seg_la_build_table", "seg_la_workspace_size", "seg_la_prefill",
@@ -130,6 +130,8 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         lib.seg_attn_wait_selftest.restype = I
         lib.seg_attn_stall_test.argtypes = [I, I]
         lib.seg_attn_stall_test.restype = I
+        lib.seg_attn_order_test.argtypes = [I]
+        lib.seg_attn_order_test.restype = I
         PP = ctypes.POINTER(ctypes.c_void_p)
         lib.seg_attn_pool_create.argtypes = [I64, PP]
         lib.seg_attn_pool_destroy.argtypes = [P]
@@ -253,6 +255,14 @@ def seg_attn_stall_test(withhold_k_tile: int, wait_us: int = 1000000) -> None:
     rc = load_library().seg_attn_stall_test(int(withhold_k_tile), int(wait_us))
     if rc != 0:
         raise SegAttnError("seg_attn_stall_test", rc)
+
+
+def seg_attn_order_test(delay_ns: int) -> None:
+    """Order test switch of later prefill launches: every softmax warp sleeps ``delay_ns``
+    after signalling P of its item's last K tile (0: off)."""
+    rc = load_library().seg_attn_order_test(int(delay_ns))
+    if rc != 0:
+        raise SegAttnError("seg_attn_order_test", rc)
 
 
 def seg_attn_take_device_error() -> int:

@@ -217,6 +217,11 @@ extern "C" int seg_attn_stall_test(int withhold_k_tile, int wait_us) {
   return segattn::set_stall_test(withhold_k_tile, wait_us);
 }
 
+extern "C" int seg_attn_order_test(int delay_ns) {
+  if (delay_ns < 0 || delay_ns > 1000000) return SEG_ATTN_ERR_INVALID_ARG;
+  return segattn::set_order_test(delay_ns);
+}
+
 extern "C" int seg_attn_take_device_error(int* value) {
   if (!value) return SEG_ATTN_ERR_INVALID_ARG;
   int wait_err = 0, append_err = 0;

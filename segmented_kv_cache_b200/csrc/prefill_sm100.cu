@@ -75,6 +75,9 @@ constexpr uint64_t kWaitLimitNs = 1000000000ull;  // default limit of a bounded 
 // producer stops loading (-1: none), and the limit of its bounded waits.
 std::atomic<int> g_stall_tile{-1};
 std::atomic<uint64_t> g_stall_wait_ns{kWaitLimitNs};
+// Order test (off by default): every softmax warp sleeps this long after it
+// signals P of its item's last K tile.
+std::atomic<int> g_order_delay_ns{0};
 constexpr float kRescaleLog2 = 8.0f;
 constexpr uint32_t kHalfBytes = 128 * 128;  // 128 rows x 64 bf16 (one swizzle-128B panel)
 
@@ -91,6 +94,7 @@ struct PrefillParams {
   const float* v_scale;
   uint64_t wait_ns;      // limit of every bounded wait (1 s unless a stall test shortens it)
   int withhold_tile;     // stall test: the producer stops before loading this K tile (-1: off)
+  int p_delay_ns;        // order test: softmax sleep after the last P is signalled (0: off)
 };
 
 // Query region + K ring + V ring + barriers + alignment slack.  The query
@@ -896,6 +900,17 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
     // A warp whose 32 rows hold no query (past the end of the chunk) only keeps
     // step with the barriers: its P rows feed only output rows nobody reads.
     const bool warp_live = __any_sync(0xffffffffu, row_valid);
+    // One tile: before P of the last K tile n - 1 is signalled, PV(n - 2) must be
+    // complete.  The S of tile n - 1 proves only PV(n - 3), and once P(n - 1) is
+    // signalled PV(n - 1) may complete at any time; a later wait for PV(n - 2) could
+    // then meet o_full at completion n, whose parity is that of n - 2, and wait for
+    // a completion that never comes.  Confirmed here, o_full is at completion n - 1
+    // or n when the epilogue waits for PV(n - 1), which one parity wait tells apart.
+    auto last_pv_order = [&](int i) -> bool {
+      if (!single || i != n_tiles - 1 || i == 0) return true;
+      return __all_sync(0xffffffffu,
+                        mbar_wait(o_full + t, (i - 1) & 1, abort_flag, wait_limit)) != 0;
+    };
     // one K tile of softmax on S buffer sb (phase sph of its barriers)
     auto run_tile = [&](int i, int sb, uint32_t sph) -> bool {
       if (single) {
@@ -914,6 +929,7 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
               !__all_sync(0xffffffffu, mbar_wait(o_full + t, (i - 1) & 1, abort_flag, wait_limit)))
             return false;
         }
+        if (!last_pv_order(i)) return false;
         mbar_arrive(p_full + sb);
         return true;
       }
@@ -921,8 +937,11 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
       const bool masked = __any_sync(0xffffffffu, (kt0 + i + 1) * kTileKeys > vis);
       if (!softmax_tile(i, masked)) return false;
       tmem_wait_st();
+      if (!last_pv_order(i)) return false;
       tc_fence_before();
       mbar_arrive(p_full + sb);
+      // order test: the last PV completes before this warp reaches the end of the item
+      if (p.p_delay_ns > 0 && i == n_tiles - 1) __nanosleep(p.p_delay_ns);
       return true;
     };
     if (single) {
@@ -955,12 +974,9 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
           for (int e = 0; e < 32; ++e) o[c][e] = 0u;
       }
     };
-    // S of the last tile ready proves PV complete up to tile n - 2, or only up to
-    // n - 3 with the two S buffers of one query tile: then wait for O phase n - 2
-    // first, since a parity wait tells apart just two consecutive phases
-    if (ok && single && n_tiles > 1)
-      ok = __all_sync(0xffffffffu,
-                      mbar_wait(o_full + t, (n_tiles - 2) & 1, abort_flag, wait_limit));
+    // PV complete up to tile n - 2 (two tiles: P(n - 1) was written after it; one
+    // tile: confirmed before P(n - 1) was signalled), so o_full is at completion
+    // n - 1 or n and a parity wait for PV(n - 1) is unambiguous
     if (ok && n_tiles > 0)
       ok = __all_sync(0xffffffffu,
                       mbar_wait(o_full + t, (n_tiles - 1) & 1, abort_flag, wait_limit));
@@ -1251,6 +1267,7 @@ int launch_prefill_d(const PrefillLaunch& a, cudaStream_t stream) {
   p.v_scale = a.v_scale;
   p.wait_ns = g_stall_wait_ns.load();
   p.withhold_tile = g_stall_tile.load();
+  p.p_delay_ns = g_order_delay_ns.load();
   // two-tile items first, then the single-tile items listed at the end.  A pass in
   // which some piece writes final rows runs the instantiation whose epilogue stores
   // full query tiles by TMA; a pass of partials only (every item split, or a pass
@@ -1311,6 +1328,11 @@ __global__ void __launch_bounds__(32) wait_selftest_kernel(uint64_t limit_ns) {
 }
 
 }  // namespace
+
+int set_order_test(int delay_ns) {
+  g_order_delay_ns.store(delay_ns);
+  return SEG_ATTN_OK;
+}
 
 int set_stall_test(int withhold_k_tile, int wait_us) {
   g_stall_tile.store(withhold_k_tile < 0 ? -1 : withhold_k_tile);

@@ -118,6 +118,8 @@ int launch_decode(const DecodeLaunch& a, cudaStream_t stream);
 int launch_wait_selftest(int wait_us, cudaStream_t stream);
 // Stall test of the prefill kernel (seg_attn_stall_test).
 int set_stall_test(int withhold_k_tile, int wait_us);
+// Order test of the prefill kernel (seg_attn_order_test).
+int set_order_test(int delay_ns);
 int take_device_error(int* value);
 int take_append_error(int* value);
 

@@ -9,7 +9,7 @@ import torch
 import oracle
 import segmented_kv_cache_b200 as sa
 
-from helpers import compare, random_case, run_cuda
+from helpers import compare, random_case, run_cuda, shared_case, shared_values
 
 S = sa.STATUS
 
@@ -21,6 +21,9 @@ def test_wait_selftest_rejects_out_of_range_limits():
         assert lib.seg_attn_wait_selftest(bad, None) == S["INVALID_ARG"]
         assert lib.seg_attn_stall_test(-1, bad) == S["INVALID_ARG"]
     assert lib.seg_attn_stall_test(-1, 1000000) == 0  # the defaults
+    for bad in (-1, 1000001):
+        assert lib.seg_attn_order_test(bad) == S["INVALID_ARG"]
+    assert lib.seg_attn_order_test(0) == 0  # off, the default
 
 
 def _stall_case(q_per_req, hq=8, hkv=2, d=128):
@@ -113,3 +116,54 @@ def test_stalled_wait_is_reported_and_the_context_survives():
                                     case["q"], case["k_pool"], case["v_pool"], case["scale"], True)
     compare(out, lse, ref_o, ref_l, "after a reported stall")
     assert sa.seg_attn_take_device_error() == 0
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("variant", ["two-tile", "one-tile", "e4m3", "shared-prefix decode"])
+def test_late_softmax_at_the_end_of_an_item_keeps_results(variant):
+    """Every softmax warp sleeps 30 us after signalling P of its item's last K tile (the
+    order test switch), so the last P.V product has completed before the warp waits for
+    it.  No wait may give up and the results must match the oracle: a one-tile item's
+    end wait used to take that state for an earlier one and wait out its limit."""
+    from segmented_kv_cache_b200 import synth
+    if variant == "shared-prefix decode":
+        # the pass over the shared prefixes runs the one-tile kernel on pieces of many K tiles
+        reqs, q_lens, S_ = shared_case(3, B=8, decode=True, max_prefix=5000)
+        case = shared_values(reqs, q_lens, S_, 64, 8, 128, seed=20)
+        mode, causal = sa.MODE_DECODE | sa.SHARE_PREFIX, True
+        q_arg = None
+    else:
+        case = _stall_case(20 if variant == "one-tile" else 50)
+        mode, causal = sa.MODE_PREFILL, False
+        q_arg = case["q_lens"]
+    c = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in case.items()}
+    assert sa.seg_attn_take_device_error() == 0
+    try:
+        sa.seg_attn_order_test(30000)
+        if variant == "e4m3":
+            tab = sa.SegTable.build(q_arg, case["seg_starts"], case["seg_lens"], case["num_slots"],
+                                    causal, mode, 8, 2, 128).to("cuda")
+            k8, v8, ks, vs = synth.fp8_pools(case["k_pool"], case["v_pool"])
+            out = torch.full_like(c["q"], float("nan"))
+            lse = torch.full(c["q"].shape[:2], float("nan"), dtype=torch.float32, device="cuda")
+            sa.seg_attn_prefill_fp8(c["q"], k8.cuda(), v8.cuda(), ks.cuda(), vs.cuda(), out, lse,
+                                    tab.device, tab.desc, case["scale"], None)
+            ref_o, ref_l = oracle.attention_fp8(case["q_lens"], case["seg_starts"],
+                                                case["seg_lens"], case["q"], k8, v8, ks, vs,
+                                                case["scale"], causal)
+        else:
+            out, lse, tab = run_cuda(c["q"], c["k_pool"], c["v_pool"], q_arg, case["seg_starts"],
+                                     case["seg_lens"], case["num_slots"], causal, mode,
+                                     case["scale"])
+            ref_o, ref_l = oracle.attention(case["q_lens"], case["seg_starts"], case["seg_lens"],
+                                            case["q"], case["k_pool"], case["v_pool"],
+                                            case["scale"], causal)
+        torch.cuda.synchronize()
+    finally:
+        sa.seg_attn_order_test(0)
+    if variant == "one-tile":
+        assert tab.desc.num_single == tab.desc.num_work
+    if variant == "shared-prefix decode":
+        assert tab.desc.shared == 1
+    assert sa.seg_attn_take_device_error() == 0
+    compare(out, lse, ref_o, ref_l, f"late softmax ({variant})")

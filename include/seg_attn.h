@@ -271,10 +271,11 @@ int seg_attn_stall_test(int withhold_k_tile, int wait_us);
 
 /*
  * seg_attn_order_test -- diagnostic (no counterpart on the source pages): every
- * softmax warp of later prefill launches sleeps about delay_ns nanoseconds
- * right after it signals P of its item's last K tile, so the last P.V product
- * has completed before the warp waits for it at the end of the item -- the
- * order a slow warp meets there (an instruction-cache miss, a profiler's
+ * softmax warp of a one-query-tile item (a short chunk, a pass over shared
+ * prefixes) in later prefill launches sleeps about delay_ns nanoseconds right
+ * after it signals P of the item's last K tile, so the last P.V product has
+ * completed before the warp waits for it at the end of the item -- the order a
+ * slow warp meets there (an instruction-cache miss, a profiler's
  * instrumentation).  Results must not change and no wait may give up.
  *   delay_ns       0 .. 1000000; 0 is off (the default).
  * Host-side setting read at each launch (process-wide, not thread-safe with

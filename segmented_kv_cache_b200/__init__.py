@@ -258,8 +258,8 @@ def seg_attn_stall_test(withhold_k_tile: int, wait_us: int = 1000000) -> None:
 
 
 def seg_attn_order_test(delay_ns: int) -> None:
-    """Order test switch of later prefill launches: every softmax warp sleeps ``delay_ns``
-    after signalling P of its item's last K tile (0: off)."""
+    """Order test switch of later prefill launches: every softmax warp of a one-tile item
+    sleeps ``delay_ns`` after signalling P of the item's last K tile (0: off)."""
     rc = load_library().seg_attn_order_test(int(delay_ns))
     if rc != 0:
         raise SegAttnError("seg_attn_order_test", rc)

@@ -12,7 +12,11 @@
 //                          stored as a bf16 tile, and the final state;
 //   la_chunk_out_kernel    per (chunk, head): Q K^T, Q S_c and P V on the tensor
 //                          cores (P = Q K^T . D, written to tensor memory as bf16
-//                          by the math warps), combined in the epilogue.
+//                          by the math warps), combined in the epilogue.  P V runs
+//                          before the entering state is known, and Q S_c then goes
+//                          into the columns of S and P, which P V has read: 256
+//                          tensor-memory columns and 97 KB of shared memory (S_c
+//                          lands where K was), so two CTAs share an SM.
 // Tiles come in with TMA (128 tokens x 64 columns per box, 128-byte swizzle),
 // accumulators live in tensor memory.  Warp roles: warp 0 lane 0 issues the
 // copies and the MMAs, warp 1 owns the tensor memory, warps 2-5 (one TMEM lane
@@ -244,7 +248,7 @@ __global__ void __launch_bounds__(256) la_scan_kernel(const Params p) {
 }
 
 // ---------------------------------------------------------------- pass 3
-__global__ void __launch_bounds__(kThreads) la_chunk_out_kernel(
+__global__ void __launch_bounds__(kThreads, 2) la_chunk_out_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_s,
     const Params p) {
@@ -254,7 +258,7 @@ __global__ void __launch_bounds__(kThreads) la_chunk_out_kernel(
   uint8_t* sQ = sm;
   uint8_t* sK = sm + kTile;
   uint8_t* sV = sm + 2 * kTile;
-  uint8_t* sS = sm + 3 * kTile;
+  uint8_t* sS = sK;  // the entering state, loaded once Q K^T has read K
   __shared__ uint64_t qk_full, s_full, v_full, qk_done, p_full, mma_done;
   __shared__ uint32_t tmem_slot;
   __shared__ volatile int abort_flag;
@@ -275,13 +279,13 @@ __global__ void __launch_bounds__(kThreads) la_chunk_out_kernel(
     abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 1) tmem_alloc(&tmem_slot, 512);
+  if (warp == 1) tmem_alloc(&tmem_slot, 256);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
-  // tensor memory: S = Q K^T, then P over it [0,128); Q S_c [128,256); P V [256,384)
-  const uint32_t tS = tmem, tI = tmem + 128, tO = tmem + 256;
+  // tensor memory: S = Q K^T, then P over it, then Q S_c [0,128); P V [128,256)
+  const uint32_t tS = tmem, tI = tmem, tO = tmem + 128;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -306,12 +310,17 @@ __global__ void __launch_bounds__(kThreads) la_chunk_out_kernel(
         }
         mma_commit(&qk_done);
       }
-      // Only the entering state comes from the scan: everything above (and the
-      // math warps' P) runs while the scan is still going when this grid was
-      // launched as its programmatic dependent.
-      grid_dependency_wait();
-      mbar_expect_tx(&s_full, kTile);
-      for (int hh = 0; hh < 2; ++hh) tma_load_3d(sS + hh * kHalf, &tm_s, &s_full, 64 * hh, 0, unit);
+      // P V needs nothing from the scan; Q S_c follows once the entering state has
+      // landed (warp 1 loads it), into the columns of S and P: tensor-core operations
+      // of one CTA run in issue order, so P V has read P by then
+      ok = ok && mbar_wait(&v_full, 0, &abort_flag, kWaitNs) &&
+           mbar_wait(&p_full, 0, &abort_flag, kWaitNs);
+      if (ok) {
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < kChunk / 16; ++k)
+          mma_ts(tO, tS + 8 * k, sdesc_sw128(va + k * 2048, kHalf, 1024), id_mn, k > 0 ? 1u : 0u);
+      }
       ok = ok && mbar_wait(&s_full, 0, &abort_flag, kWaitNs);
       if (ok) {
         tc_fence_after();
@@ -322,20 +331,25 @@ __global__ void __launch_bounds__(kThreads) la_chunk_out_kernel(
                  id_mn, k > 0 ? 1u : 0u);
         }
       }
-      ok = ok && mbar_wait(&v_full, 0, &abort_flag, kWaitNs) &&
-           mbar_wait(&p_full, 0, &abort_flag, kWaitNs);
-      if (ok) {
-        tc_fence_after();
-#pragma unroll
-        for (int k = 0; k < kChunk / 16; ++k)
-          mma_ts(tO, tS + 8 * k, sdesc_sw128(va + k * 2048, kHalf, 1024), id_mn, k > 0 ? 1u : 0u);
-      }
       mma_commit(&mma_done);
       mbar_wait(&mma_done, 0, nullptr, kWaitNs);
-      if (!ok) {  // leave no copy in flight
+      if (!ok) {  // leave no copy in flight (warp 1 waits for the state's)
         mbar_wait(&qk_full, 0, nullptr, kWaitNs);
-        mbar_wait(&s_full, 0, nullptr, kWaitNs);
         mbar_wait(&v_full, 0, nullptr, kWaitNs);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // Only the entering state comes from the scan: everything else runs while the
+      // scan is still going when this grid was launched as its programmatic
+      // dependent.  It lands where K was, once the Q K^T products have read K.
+      grid_dependency_wait();
+      if (mbar_wait(&qk_done, 0, &abort_flag, kWaitNs)) {
+        mbar_expect_tx(&s_full, kTile);
+        for (int hh = 0; hh < 2; ++hh)
+          tma_load_3d(sS + hh * kHalf, &tm_s, &s_full, 64 * hh, 0, unit);
+        mbar_wait(&s_full, 0, nullptr, kWaitNs);  // no copy left in flight at exit
       }
     }
     __syncwarp();
@@ -370,41 +384,38 @@ __global__ void __launch_bounds__(kThreads) la_chunk_out_kernel(
       }
       tmem_st64(tS + (lane_base - tmem), pk);
       tmem_wait_st();
-      tc_fence_before();
     }
+    tc_fence_before();
     mbar_arrive(&p_full);
     ok = ok && __all_sync(0xffffffffu, mbar_wait(&mma_done, 0, &abort_flag, kWaitNs));
     if (ok) {
       tc_fence_after();
-      const float decay_t = ex2(gt);
       // Row t of out is 128 bf16 = 16 pieces of 16 bytes.  The Q tile is idle once
       // every MMA is done: row t goes there at 256 * t, piece c at position
       // (c & 8) | ((c ^ t) & 7), and each warp then writes its own 32 rows out, two
       // whole 256-byte rows per store instruction (rows past the chunk stay unwritten).
+      const float decay_t = ex2(gt);
       uint4* stage = reinterpret_cast<uint4*>(sQ);
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t a[2][32], b[2][32];
-        tmem_ld64(tI + (lane_base - tmem) + 64 * half, a);
-        tmem_ld64(tO + (lane_base - tmem) + 64 * half, b);
-        tmem_wait_ld(a[0]);
-        tmem_wait_ld(a[1]);
-        tmem_wait_ld(b[0]);
-        tmem_wait_ld(b[1]);
+      for (int q4 = 0; q4 < 4; ++q4) {
+        uint32_t a[32], b[32];
+        tmem_ld32(tI + (lane_base - tmem) + 32 * q4, a);
+        tmem_ld32(tO + (lane_base - tmem) + 32 * q4, b);
+        tmem_wait_ld(a);
+        tmem_wait_ld(b);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {  // piece c = 8 * half + j: columns 8c .. 8c + 7
+        for (int j = 0; j < 4; ++j) {  // piece c = 4 * q4 + j: columns 8c .. 8c + 7
           uint32_t wd[4];
 #pragma unroll
           for (int u2 = 0; u2 < 4; ++u2) {
             const int e = 8 * j + 2 * u2;
-            const float o0 = p.scale * fmaf(decay_t, __uint_as_float(a[e >> 5][e & 31]),
-                                            __uint_as_float(b[e >> 5][e & 31]));
-            const float o1 = p.scale * fmaf(decay_t, __uint_as_float(a[e >> 5][(e & 31) + 1]),
-                                            __uint_as_float(b[e >> 5][(e & 31) + 1]));
+            const float o0 = p.scale * fmaf(decay_t, __uint_as_float(a[e]), __uint_as_float(b[e]));
+            const float o1 =
+                p.scale * fmaf(decay_t, __uint_as_float(a[e + 1]), __uint_as_float(b[e + 1]));
             __nv_bfloat162 v2 = __floats2bfloat162_rn(o0, o1);
             wd[u2] = *reinterpret_cast<uint32_t*>(&v2);
           }
-          const int c = 8 * half + j;
+          const int c = 4 * q4 + j;
           stage[16 * t + ((c & 8) | ((c ^ t) & 7))] = make_uint4(wd[0], wd[1], wd[2], wd[3]);
         }
       }
@@ -423,7 +434,7 @@ __global__ void __launch_bounds__(kThreads) la_chunk_out_kernel(
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, 256);
   }
   if (threadIdx.x == 0 && abort_flag) atomicOr(&g_la_error, 1);
 }
@@ -478,12 +489,17 @@ int launch_la_prefill(const Launch& a, cudaStream_t stream) {
     if (!encode3(&tq, a.q, d.heads, d.total_q, false) || !encode3(&tk, a.k, d.heads, d.total_q, false) ||
         !encode3(&tv, a.v, d.heads, d.total_q, false) || !encode3(&ts, p.s_in, kDim, units, true))
       return SEG_ATTN_ERR_CUDA;
-    constexpr int smem1 = 2 * kTile + 1024, smem3 = 4 * kTile + 1024;
+    constexpr int smem1 = 2 * kTile + 1024, smem3 = 3 * kTile + 1024;
+    // The output pass fits two CTAs per SM; a grid that fills at most one CTA per SM
+    // asks for more shared memory than two could share, so no SM takes two of them
+    // while others idle.
+    constexpr int kSms = 148, smem3_spread = 4 * kTile + 1024;
+    const int smem3_launch = units <= kSms ? smem3_spread : smem3;
     // function attributes are per device: set them for the current one on every call
     if (cudaFuncSetAttribute(la_chunk_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              smem1) != cudaSuccess ||
         cudaFuncSetAttribute(la_chunk_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem3) != cudaSuccess)
+                             smem3_spread) != cudaSuccess)
       return SEG_ATTN_ERR_CUDA;
     const dim3 grid(d.num_chunks, d.heads);
     la_chunk_state_kernel<<<grid, kThreads, smem1, stream>>>(tk, tv, p);
@@ -504,7 +520,7 @@ int launch_la_prefill(const Launch& a, cudaStream_t stream) {
     if (cudaLaunchKernelEx(&cfg, la_scan_kernel, p) != cudaSuccess) return SEG_ATTN_ERR_CUDA;
     cfg.gridDim = grid;
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = smem3;
+    cfg.dynamicSmemBytes = smem3_launch;
     if (cudaLaunchKernelEx(&cfg, la_chunk_out_kernel, tq, tk, tv, ts, p) != cudaSuccess)
       return SEG_ATTN_ERR_CUDA;
   } else if (d.batch > 0) {

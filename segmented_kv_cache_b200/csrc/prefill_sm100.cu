@@ -75,8 +75,8 @@ constexpr uint64_t kWaitLimitNs = 1000000000ull;  // default limit of a bounded 
 // producer stops loading (-1: none), and the limit of its bounded waits.
 std::atomic<int> g_stall_tile{-1};
 std::atomic<uint64_t> g_stall_wait_ns{kWaitLimitNs};
-// Order test (off by default): every softmax warp sleeps this long after it
-// signals P of its item's last K tile.
+// Order test (off by default): every softmax warp of a one-tile item sleeps this
+// long after it signals P of the item's last K tile.
 std::atomic<int> g_order_delay_ns{0};
 constexpr float kRescaleLog2 = 8.0f;
 constexpr uint32_t kHalfBytes = 128 * 128;  // 128 rows x 64 bf16 (one swizzle-128B panel)
@@ -94,7 +94,7 @@ struct PrefillParams {
   const float* v_scale;
   uint64_t wait_ns;      // limit of every bounded wait (1 s unless a stall test shortens it)
   int withhold_tile;     // stall test: the producer stops before loading this K tile (-1: off)
-  int p_delay_ns;        // order test: softmax sleep after the last P is signalled (0: off)
+  int p_delay_ns;        // order test: one-tile softmax sleep after the last P is signalled (0: off)
 };
 
 // Query region + K ring + V ring + barriers + alignment slack.  The query
@@ -940,8 +940,6 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
       if (!last_pv_order(i)) return false;
       tc_fence_before();
       mbar_arrive(p_full + sb);
-      // order test: the last PV completes before this warp reaches the end of the item
-      if (p.p_delay_ns > 0 && i == n_tiles - 1) __nanosleep(p.p_delay_ns);
       return true;
     };
     if (single) {
@@ -953,6 +951,11 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreads, 1)
       }
     } else {
       for (int i = 0; ok && i < n_tiles; ++i) ok = run_tile(i, t, i & 1);
+    }
+    // order test (one tile): the last PV completes before this warp reaches the end
+    // of the item
+    if constexpr (SINGLE) {
+      if (p.p_delay_ns > 0 && ok) __nanosleep(p.p_delay_ns);
     }
     if (!warp_live) ok = false;  // nothing to write
     // this row's O (fp32, D columns) in registers: every load issued, one wait

@@ -119,12 +119,13 @@ def test_stalled_wait_is_reported_and_the_context_survives():
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("variant", ["two-tile", "one-tile", "e4m3", "shared-prefix decode"])
+@pytest.mark.parametrize("variant", ["one-tile", "one-tile e4m3", "shared-prefix decode"])
 def test_late_softmax_at_the_end_of_an_item_keeps_results(variant):
-    """Every softmax warp sleeps 30 us after signalling P of its item's last K tile (the
-    order test switch), so the last P.V product has completed before the warp waits for
-    it.  No wait may give up and the results must match the oracle: a one-tile item's
-    end wait used to take that state for an earlier one and wait out its limit."""
+    """Every softmax warp of a one-tile item sleeps 30 us after signalling P of the item's
+    last K tile (the order test switch), so the last P.V product has completed before the
+    warp waits for it.  No wait may give up and the results must match the oracle: the
+    end wait used to take that state for an earlier one and wait out its limit.  (The
+    two-tile kernel waits for PV(i - 1) before it writes P(i), so it never meets it.)"""
     from segmented_kv_cache_b200 import synth
     if variant == "shared-prefix decode":
         # the pass over the shared prefixes runs the one-tile kernel on pieces of many K tiles
@@ -133,14 +134,14 @@ def test_late_softmax_at_the_end_of_an_item_keeps_results(variant):
         mode, causal = sa.MODE_DECODE | sa.SHARE_PREFIX, True
         q_arg = None
     else:
-        case = _stall_case(20 if variant == "one-tile" else 50)
+        case = _stall_case(20)  # qpt = 32: one query tile per item
         mode, causal = sa.MODE_PREFILL, False
         q_arg = case["q_lens"]
     c = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in case.items()}
     assert sa.seg_attn_take_device_error() == 0
     try:
         sa.seg_attn_order_test(30000)
-        if variant == "e4m3":
+        if variant == "one-tile e4m3":
             tab = sa.SegTable.build(q_arg, case["seg_starts"], case["seg_lens"], case["num_slots"],
                                     causal, mode, 8, 2, 128).to("cuda")
             k8, v8, ks, vs = synth.fp8_pools(case["k_pool"], case["v_pool"])
@@ -161,7 +162,7 @@ def test_late_softmax_at_the_end_of_an_item_keeps_results(variant):
         torch.cuda.synchronize()
     finally:
         sa.seg_attn_order_test(0)
-    if variant == "one-tile":
+    if variant.startswith("one-tile"):
         assert tab.desc.num_single == tab.desc.num_work
     if variant == "shared-prefix decode":
         assert tab.desc.shared == 1

@@ -21,6 +21,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <cmath>
 #include <array>
 #include <functional>
 #include <limits>
@@ -127,13 +128,15 @@ void plan_pieces(const std::vector<PItem>& items, int max_split, std::vector<Row
     if (f <= 1 || tiles < 2 * segattn::kMinPieceTiles) return 1;
     return std::min(f, tiles / segattn::kMinPieceTiles);
   };
-  auto makespan = [&](int f) {
+  // Longest-first schedule of the pieces on the SMs (each piece costed at its K tiles
+  // plus the per-piece start-up and epilogue), for a piece count per item.
+  auto makespan = [&](const std::vector<int>& counts) {
     std::vector<int64_t> cost;
-    for (const PItem& it : items) {
-      const int p = pieces_of(it.tiles, f);
+    for (size_t i = 0; i < items.size(); ++i) {
+      const int64_t t = items[i].tiles;
+      const int p = counts[i];
       for (int j = 0; j < p; ++j)
-        cost.push_back((int64_t)it.tiles * (j + 1) / p - (int64_t)it.tiles * j / p +
-                       segattn::kPieceOverheadTiles);
+        cost.push_back(t * (j + 1) / p - t * j / p + segattn::kPieceOverheadTiles);
     }
     std::sort(cost.begin(), cost.end(), std::greater<int64_t>());
     std::priority_queue<int64_t, std::vector<int64_t>, std::greater<int64_t>> sm;
@@ -147,15 +150,49 @@ void plan_pieces(const std::vector<PItem>& items, int max_split, std::vector<Row
     }
     return span_max;
   };
-  int best_f = 1;
-  int64_t best = makespan(1);
-  for (int f = 2; f <= max_split; ++f) {
-    const int64_t m = makespan(f);
-    if (m * 100 < best * 98) {
-      best = m;
-      best_f = f;
-    }
+  // Candidate plans: every item cut into the same number of pieces f (1 .. max_split),
+  // or every item cut into pieces of about L = (all K tiles) / (k waves x SMs) tiles,
+  // k = 1 .. 8, so that items of different lengths end in pieces of one length that
+  // fill whole waves.  Both respect the shortest piece and the most pieces per item.
+  // The plan taken is the one with the fewest pieces among those whose simulated
+  // makespan is within 2 % of the best.
+  int64_t total_tiles = 0;
+  for (const PItem& it : items) total_tiles += it.tiles;
+  std::vector<std::vector<int>> cands;
+  for (int f = 1; f <= max_split; ++f) {
+    std::vector<int> c(items.size());
+    for (size_t i = 0; i < items.size(); ++i) c[i] = pieces_of(items[i].tiles, f);
+    cands.push_back(std::move(c));
   }
+  for (int k = 1; k <= 8 && total_tiles > 0; ++k) {
+    const double len = (double)total_tiles / ((double)k * segattn::kSmCount);
+    std::vector<int> c(items.size());
+    for (size_t i = 0; i < items.size(); ++i) {
+      const int32_t t = items[i].tiles;
+      if (t < 2 * segattn::kMinPieceTiles) {
+        c[i] = 1;
+        continue;
+      }
+      const int want = (int)std::lround((double)t / len);
+      c[i] = std::max(1, std::min({want, max_split, (int)(t / segattn::kMinPieceTiles)}));
+    }
+    cands.push_back(std::move(c));
+  }
+  std::vector<int64_t> spans(cands.size()), npieces(cands.size(), 0);
+  int64_t best_span = INT64_MAX;
+  for (size_t j = 0; j < cands.size(); ++j) {
+    spans[j] = makespan(cands[j]);
+    for (int p : cands[j]) npieces[j] += p;
+    best_span = std::min(best_span, spans[j]);
+  }
+  size_t pick = 0;
+  for (size_t j = 0; j < cands.size(); ++j) {
+    if (spans[j] * 100 > best_span * 102) continue;
+    if (spans[pick] * 100 > best_span * 102 || npieces[j] < npieces[pick] ||
+        (npieces[j] == npieces[pick] && spans[j] < spans[pick]))
+      pick = j;
+  }
+  const std::vector<int>& counts = cands[pick];
   // The one-tile kernel runs a pass only when every item of it is single-tile: a
   // second launch for a few single-tile items would serialise behind the first
   // launch's tail (those items then run two-tile, their empty tile's softmax skipped).
@@ -165,7 +202,7 @@ void plan_pieces(const std::vector<PItem>& items, int max_split, std::vector<Row
   for (size_t i = 0; i < items.size(); ++i) {
     PItem it = items[i];
     it.single = all_single;
-    const int p = pieces_of(it.tiles, best_f);
+    const int p = counts[i];
     const bool slotted = p > 1 || it.cascade;
     const int32_t slot0 = slotted ? out.slots : -1;
     if (slotted) out.slots += p;

@@ -19,7 +19,8 @@
 //                          lands where K was), so two CTAs share an SM.
 // Tiles come in with TMA (128 tokens x 64 columns per box, 128-byte swizzle),
 // accumulators live in tensor memory.  Warp roles: warp 0 lane 0 issues the
-// copies and the MMAs, warp 1 owns the tensor memory, warps 2-5 (one TMEM lane
+// copies and the MMAs, warp 1 owns the tensor memory (and in the output pass
+// loads the entering state once the scan has finished), warps 2-5 (one TMEM lane
 // quadrant each) do the per-row arithmetic.  Every mbarrier wait gives up after
 // one second and flags a device error instead of hanging.
 #include <cuda.h>

@@ -265,3 +265,34 @@ def test_shared_prefix_configs_share_every_group(cfg):
         shared_tiles = tiles(tab, d.off_work, d.num_work) + tiles(tab, d.off_group_work,
                                                                   d.num_group_work)
         assert shared_tiles < 0.8 * tiles(plain, plain.desc.off_work, plain.desc.num_work)
+
+
+def test_prefix_pass_of_unequal_groups_is_cut_into_pieces_of_one_length():
+    # The decode groups' prefixes run 8192..32768 keys (64..256 K tiles per item).  The
+    # planner may cut every item into the same number of pieces, or every item into
+    # pieces of about one length; whichever it takes, each item's pieces cover its K
+    # tiles once, in order, each piece writes its own partial slot, and the pieces are
+    # the fewest that keep the simulated schedule within 2 % of the best.  Here the
+    # equal-length cut wins: all pieces within 1.5x of each other (equal counts per item
+    # would leave 2x between the longest and the shortest).
+    wl = synth.make_workload(6, values=False)
+    b = wl.batches[0]
+    tab = sa.SegTable.build(None, b.seg_starts, b.seg_lens, wl.num_slots, True,
+                            sa.MODE_DECODE | sa.SHARE_PREFIX, wl.q_heads, wl.kv_heads,
+                            wl.head_dim)
+    d = tab.desc
+    w = arr(tab, d.off_group_work, d.num_group_work, 16)
+    lens = w[:, 4] - w[:, 3]
+    assert (lens >= 8).all()
+    items = {}
+    for row in w:
+        items.setdefault((row[0], row[1], row[2]), []).append(row)
+    totals = []
+    for rows in items.values():
+        rows = sorted(rows, key=lambda r: r[3])
+        assert rows[0][3] == 0
+        assert all(a[4] == b_[3] for a, b_ in zip(rows, rows[1:]))
+        totals.append(rows[-1][4])
+    assert max(totals) >= 2 * min(totals) - 1  # the items really differ in length
+    assert lens.max() <= 1.5 * lens.min()
+    assert sorted(w[:, 5].tolist()) == list(range(d.num_group_parts))
